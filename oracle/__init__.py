@@ -1,0 +1,237 @@
+"""CPU oracle for the SmoothQuant W8A8 smoothed linear layer.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and
+the CPU-baseline / reference legs of ``bench.py`` may import this package.
+It shares no code with the CUDA library: the arithmetic lives in
+``sq_oracle.c`` (plain single-threaded C, fp32, round-to-nearest-even, no
+FMA contraction); this module only compiles it with gcc and marshals numpy
+arrays into it.
+
+Method source: "SmoothQuant (activation smoothing quantization)", jisaku.com
+glossary (2023), sections "The mathematics of the smoothing transformation"
+(Y = (X diag(s)^-1)(diag(s) W)) and "Hyper-parameter alpha"
+(s_j = max|X_j|^alpha / max|W_j|^(1-alpha)).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "sq_oracle.c")
+_BUILD = os.path.join(_HERE, "_build")
+_LIB_PATH = os.path.join(_BUILD, "libsq_oracle.so")
+
+# -O2 without fast-math and without FMA contraction: every fp32 operation is
+# one IEEE-rounded operation in source order.
+CFLAGS = ["-O2", "-fno-fast-math", "-ffp-contract=off", "-fPIC", "-shared", "-std=gnu11"]
+
+LAYOUT_KN = 0
+LAYOUT_NK = 1
+
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile sq_oracle.c into _build/libsq_oracle.so (gcc)."""
+    os.makedirs(_BUILD, exist_ok=True)
+    stale = (not os.path.exists(_LIB_PATH)) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC)
+    if force or stale:
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        subprocess.run(["gcc", *CFLAGS, _SRC, "-o", tmp, "-lm"], check=True)
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        f32p = ctypes.POINTER(ctypes.c_float)
+        i8p = ctypes.POINTER(ctypes.c_int8)
+        i32p = ctypes.POINTER(ctypes.c_int32)
+        u16p = ctypes.POINTER(ctypes.c_uint16)
+        i64 = ctypes.c_int64
+        sig = {
+            "or_quantize_value": ([ctypes.c_float, ctypes.c_float], ctypes.c_int8),
+            "or_calib_absmax": ([f32p, i64, i64, f32p], None),
+            "or_weight_absmax": ([f32p, ctypes.c_int, i64, i64, f32p], None),
+            "or_smooth_factor": ([f32p, f32p, i64, ctypes.c_float, f32p, f32p], None),
+            "or_smooth_weight": ([f32p, ctypes.c_int, i64, i64, f32p, f32p], None),
+            "or_smooth_quant_weight": ([f32p, ctypes.c_int, i64, i64, f32p, i8p, f32p], None),
+            "or_smooth_act": ([f32p, i64, i64, f32p, f32p], None),
+            "or_quant_act": ([f32p, i64, i64, f32p, i8p, f32p], None),
+            "or_gemm_i8": ([i8p, i8p, i64, i64, i64, i32p], None),
+            "or_dequant": ([i32p, f32p, f32p, i64, i64, f32p], None),
+            "or_round_bf16": ([f32p, i64, u16p], None),
+            "or_round_f16": ([f32p, i64, u16p], None),
+        }
+        for name, (args, res) in sig.items():
+            fn = getattr(lib, name)
+            fn.argtypes = args
+            fn.restype = res
+        _lib = lib
+    return _lib
+
+
+def _f32(a) -> np.ndarray:
+    a = np.ascontiguousarray(np.asarray(a, dtype=np.float32))
+    return a
+
+
+def _ptr(a: np.ndarray, ctype):
+    return a.ctypes.data_as(ctypes.POINTER(ctype))
+
+
+# ---------------------------------------------------------------------------
+# numpy-facing wrappers, one per oracle step
+# ---------------------------------------------------------------------------
+
+def quantize_value(v: float, r: float) -> int:
+    """clamp(rne(v * r), -127, 127) in fp32."""
+    return int(_load().or_quantize_value(ctypes.c_float(v), ctypes.c_float(r)))
+
+
+def calib_absmax(x, amax=None) -> np.ndarray:
+    """Running per-channel max|X_j| over the tokens (rows) of x [T, K]."""
+    x = _f32(x)
+    T, K = x.shape
+    out = np.zeros(K, np.float32) if amax is None else _f32(amax).copy()
+    _load().or_calib_absmax(_ptr(x, ctypes.c_float), T, K, _ptr(out, ctypes.c_float))
+    return out
+
+
+def weight_absmax(w, layout: int) -> np.ndarray:
+    """w_j = max_n |W_jn| for W given as [K,N] (LAYOUT_KN) or [N,K] (LAYOUT_NK)."""
+    w = _f32(w)
+    K, N = _kn(w, layout)
+    out = np.zeros(K, np.float32)
+    _load().or_weight_absmax(_ptr(w, ctypes.c_float), layout, K, N, _ptr(out, ctypes.c_float))
+    return out
+
+
+def smooth_factor(amax, wmax, alpha: float):
+    """(s, inv_s) from the per-channel maxima and alpha."""
+    amax = _f32(amax)
+    wmax = _f32(wmax)
+    K = amax.shape[0]
+    s = np.zeros(K, np.float32)
+    inv = np.zeros(K, np.float32)
+    _load().or_smooth_factor(_ptr(amax, ctypes.c_float), _ptr(wmax, ctypes.c_float), K,
+                             ctypes.c_float(alpha), _ptr(s, ctypes.c_float), _ptr(inv, ctypes.c_float))
+    return s, inv
+
+
+def smooth_weight(w, layout: int, s) -> np.ndarray:
+    """W~ = diag(s) W, returned in W's own layout."""
+    w = _f32(w)
+    s = _f32(s)
+    K, N = _kn(w, layout)
+    out = np.zeros_like(w)
+    _load().or_smooth_weight(_ptr(w, ctypes.c_float), layout, K, N, _ptr(s, ctypes.c_float),
+                             _ptr(out, ctypes.c_float))
+    return out
+
+
+def smooth_quant_weight(w, layout: int, s):
+    """(Wq [N,K] int8, dw [N] fp32) from W and s."""
+    w = _f32(w)
+    s = _f32(s)
+    K, N = _kn(w, layout)
+    wq = np.zeros((N, K), np.int8)
+    dw = np.zeros(N, np.float32)
+    _load().or_smooth_quant_weight(_ptr(w, ctypes.c_float), layout, K, N, _ptr(s, ctypes.c_float),
+                                   _ptr(wq, ctypes.c_int8), _ptr(dw, ctypes.c_float))
+    return wq, dw
+
+
+def smooth_act(x, inv_s) -> np.ndarray:
+    """X~ = X diag(s)^-1 = X * inv_s (per column)."""
+    x = _f32(x)
+    inv_s = _f32(inv_s)
+    M, K = x.shape
+    out = np.zeros_like(x)
+    _load().or_smooth_act(_ptr(x, ctypes.c_float), M, K, _ptr(inv_s, ctypes.c_float),
+                          _ptr(out, ctypes.c_float))
+    return out
+
+
+def quant_act(x, inv_s):
+    """(Xq [M,K] int8, dx [M] fp32): smoothing then per-token quantization."""
+    x = _f32(x)
+    inv_s = _f32(inv_s)
+    M, K = x.shape
+    xq = np.zeros((M, K), np.int8)
+    dx = np.zeros(M, np.float32)
+    _load().or_quant_act(_ptr(x, ctypes.c_float), M, K, _ptr(inv_s, ctypes.c_float),
+                         _ptr(xq, ctypes.c_int8), _ptr(dx, ctypes.c_float))
+    return xq, dx
+
+
+def gemm_i8(xq, wq) -> np.ndarray:
+    """acc [M,N] int32 = Xq [M,K] . Wq[N,K]^T."""
+    xq = np.ascontiguousarray(np.asarray(xq, dtype=np.int8))
+    wq = np.ascontiguousarray(np.asarray(wq, dtype=np.int8))
+    M, K = xq.shape
+    N, K2 = wq.shape
+    assert K == K2
+    acc = np.zeros((M, N), np.int32)
+    _load().or_gemm_i8(_ptr(xq, ctypes.c_int8), _ptr(wq, ctypes.c_int8), M, N, K, _ptr(acc, ctypes.c_int32))
+    return acc
+
+
+def dequant(acc, dx, dw) -> np.ndarray:
+    """y [M,N] fp32 = ((float)acc * dx_t) * dw_n."""
+    acc = np.ascontiguousarray(np.asarray(acc, dtype=np.int32))
+    dx = _f32(dx)
+    dw = _f32(dw)
+    M, N = acc.shape
+    y = np.zeros((M, N), np.float32)
+    _load().or_dequant(_ptr(acc, ctypes.c_int32), _ptr(dx, ctypes.c_float), _ptr(dw, ctypes.c_float),
+                       M, N, _ptr(y, ctypes.c_float))
+    return y
+
+
+def round_to(y, dtype: str) -> np.ndarray:
+    """Round fp32 y to 'bf16' / 'f16' (returned as raw uint16 bit patterns) or keep 'f32'."""
+    y = _f32(y)
+    if dtype == "f32":
+        return y.copy()
+    out = np.zeros(y.shape, np.uint16)
+    fn = _load().or_round_bf16 if dtype == "bf16" else _load().or_round_f16
+    if dtype not in ("bf16", "f16"):
+        raise ValueError(dtype)
+    fn(_ptr(y, ctypes.c_float), y.size, _ptr(out, ctypes.c_uint16))
+    return out
+
+
+def linear(x, inv_s, wq, dw, out_dtype: str = "f32"):
+    """The runtime smoothed linear: quant_act -> gemm_i8 -> dequant -> round."""
+    xq, dx = quant_act(x, inv_s)
+    acc = gemm_i8(xq, wq)
+    y = dequant(acc, dx, dw)
+    return round_to(y, out_dtype), acc, xq, dx
+
+
+def pipeline(calib_chunks, w, layout: int, alpha: float, x, out_dtype: str = "f32"):
+    """Whole path in the usage order: calibrate -> smooth+quantize W -> linear."""
+    K = _kn(_f32(w), layout)[0]
+    amax = np.zeros(K, np.float32)
+    for c in calib_chunks:
+        amax = calib_absmax(c, amax)
+    wmax = weight_absmax(w, layout)
+    s, inv_s = smooth_factor(amax, wmax, alpha)
+    wq, dw = smooth_quant_weight(w, layout, s)
+    y, acc, xq, dx = linear(x, inv_s, wq, dw, out_dtype)
+    return dict(amax=amax, wmax=wmax, s=s, inv_s=inv_s, wq=wq, dw=dw, xq=xq, dx=dx, acc=acc, y=y)
+
+
+def _kn(w: np.ndarray, layout: int):
+    if layout == LAYOUT_KN:
+        return w.shape[0], w.shape[1]
+    if layout == LAYOUT_NK:
+        return w.shape[1], w.shape[0]
+    raise ValueError(f"layout {layout}")

@@ -1,0 +1,231 @@
+/*
+ * sq_oracle.c -- plain, slow CPU oracle for the SmoothQuant W8A8 smoothed
+ * linear layer.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the test suite, the smoke check and the
+ * benchmark's CPU-baseline leg may load this file.  It shares no code,
+ * header, table or helper with the CUDA library; neither side includes or
+ * links the other.  Every step is a single-threaded loop written in the
+ * order the method states it, with no blocking or fusion.
+ *
+ * Source of the method: "SmoothQuant (activation smoothing quantization)",
+ * jisaku.com glossary page (2023):
+ *   - section "Why activation quantization is hard": INT8 holds -128..127
+ *     and a token is scaled so that its largest magnitude maps to 127;
+ *   - section "The mathematics of the smoothing transformation":
+ *     Y = X W = (X diag(s)^-1)(diag(s) W) = X~ W~;
+ *   - section "Hyper-parameter alpha (migration strength)":
+ *     s_j = max|X_j|^alpha / max|W_j|^(1-alpha), alpha = 0.5 default;
+ *   - usage example: get_act_scales -> smooth_lm(alpha) -> quantize_model.
+ *
+ * Readings where the page is silent (all listed in the design notes):
+ *   - arithmetic is IEEE fp32 with round-to-nearest-even everywhere; build
+ *     with -ffp-contract=off so no multiply is fused into an add;
+ *   - channel maxima are floored at 1e-5 before s is formed;
+ *   - s^alpha is evaluated with sqrt for alpha in {0, .25, .5, .75, 1}
+ *     and with double pow otherwise;
+ *   - X~ = X * (1/s): the stored reciprocal is multiplied in;
+ *   - activations are quantized per token (dynamic), weights per output
+ *     channel: for a row v with absmax m, delta = m/127 and
+ *     q = clamp(rne(v * (127/m)), -127, 127); an all-zero row gives
+ *     delta = 0 and q = 0;
+ *   - the int32 product is dequantized as ((float)acc * dx_t) * dw_n and
+ *     then rounded to the output type.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#define OR_LAYOUT_KN 0 /* W[K][N]: Y = X W as the page writes it      */
+#define OR_LAYOUT_NK 1 /* W[N][K]: output-major, as torch's nn.Linear */
+
+/* Element W_jn (input channel j, output channel n) for either layout. */
+static float w_at(const float *w, int layout, int64_t K, int64_t N,
+                  int64_t j, int64_t n) {
+  return layout == OR_LAYOUT_KN ? w[j * N + n] : w[n * K + j];
+}
+
+/* ---- quantizer for one value --------------------------------------------
+ * Round half to even (rintf under the default rounding mode), then clamp to
+ * the symmetric range [-127, 127].  r is 127/absmax of the value's row. */
+int8_t or_quantize_value(float v, float r) {
+  float t = v * r;
+  float q = rintf(t);
+  if (q > 127.0f) q = 127.0f;
+  if (q < -127.0f) q = -127.0f;
+  return (int8_t)q;
+}
+
+/* ---- step 1: calibration ------------------------------------------------
+ * amax_j <- max(amax_j, max_t |x_tj|) over the tokens of one chunk; a
+ * running maximum across calls (get_act_scales in the usage example). */
+void or_calib_absmax(const float *x, int64_t T, int64_t K, float *amax) {
+  for (int64_t t = 0; t < T; ++t)
+    for (int64_t j = 0; j < K; ++j) {
+      float v = fabsf(x[t * K + j]);
+      if (v > amax[j]) amax[j] = v;
+    }
+}
+
+/* ---- step 2: weight maximum per input channel ---------------------------
+ * w_j = max_n |W_jn|: the max|W_j| of the alpha formula. */
+void or_weight_absmax(const float *w, int layout, int64_t K, int64_t N,
+                      float *wmax) {
+  for (int64_t j = 0; j < K; ++j) {
+    float m = 0.0f;
+    for (int64_t n = 0; n < N; ++n) {
+      float v = fabsf(w_at(w, layout, K, N, j, n));
+      if (v > m) m = v;
+    }
+    wmax[j] = m;
+  }
+}
+
+/* ---- step 3: smoothing factor -------------------------------------------
+ * s_j = max|X_j|^alpha / max|W_j|^(1-alpha), inv_s_j = 1/s_j. */
+void or_smooth_factor(const float *amax, const float *wmax, int64_t K,
+                      float alpha, float *s, float *inv_s) {
+  for (int64_t j = 0; j < K; ++j) {
+    float a = amax[j] > 1e-5f ? amax[j] : 1e-5f;
+    float w = wmax[j] > 1e-5f ? wmax[j] : 1e-5f;
+    float sj;
+    if (alpha == 1.0f) {
+      sj = a; /* a^1 / w^0 */
+    } else if (alpha == 0.0f) {
+      sj = 1.0f / w; /* a^0 / w^1 */
+    } else if (alpha == 0.5f) {
+      sj = sqrtf(a) / sqrtf(w);
+    } else if (alpha == 0.25f) {
+      float a14 = sqrtf(sqrtf(a));
+      float w34 = sqrtf(w) * sqrtf(sqrtf(w));
+      sj = a14 / w34;
+    } else if (alpha == 0.75f) {
+      float a34 = sqrtf(a) * sqrtf(sqrtf(a));
+      float w14 = sqrtf(sqrtf(w));
+      sj = a34 / w14;
+    } else {
+      double num = pow((double)a, (double)alpha);
+      double den = pow((double)w, 1.0 - (double)alpha);
+      sj = (float)(num / den);
+    }
+    s[j] = sj;
+    inv_s[j] = 1.0f / sj;
+  }
+}
+
+/* ---- step 4: weight fold W~ = diag(s) W ---------------------------------
+ * Output is W~ in W's own layout. */
+void or_smooth_weight(const float *w, int layout, int64_t K, int64_t N,
+                      const float *s, float *wt) {
+  for (int64_t j = 0; j < K; ++j)
+    for (int64_t n = 0; n < N; ++n) {
+      float v = s[j] * w_at(w, layout, K, N, j, n);
+      if (layout == OR_LAYOUT_KN)
+        wt[j * N + n] = v;
+      else
+        wt[n * K + j] = v;
+    }
+}
+
+/* ---- step 5: per-output-channel weight quantization ---------------------
+ * For output channel n: m_n = max_j |W~_jn|, dw_n = m_n/127,
+ * Wq[n][j] = clamp(rne(W~_jn * (127/m_n))).  Wq is stored [N][K]
+ * (K contiguous) whatever W's layout. */
+void or_smooth_quant_weight(const float *w, int layout, int64_t K, int64_t N,
+                            const float *s, int8_t *wq, float *dw) {
+  for (int64_t n = 0; n < N; ++n) {
+    float m = 0.0f;
+    for (int64_t j = 0; j < K; ++j) {
+      float v = fabsf(s[j] * w_at(w, layout, K, N, j, n));
+      if (v > m) m = v;
+    }
+    if (m == 0.0f) {
+      dw[n] = 0.0f;
+      for (int64_t j = 0; j < K; ++j) wq[n * K + j] = 0;
+      continue;
+    }
+    dw[n] = m / 127.0f;
+    float r = 127.0f / m;
+    for (int64_t j = 0; j < K; ++j)
+      wq[n * K + j] = or_quantize_value(s[j] * w_at(w, layout, K, N, j, n), r);
+  }
+}
+
+/* ---- step 6: activation smoothing X~ = X diag(s)^-1 ---------------------- */
+void or_smooth_act(const float *x, int64_t M, int64_t K, const float *inv_s,
+                   float *xt) {
+  for (int64_t t = 0; t < M; ++t)
+    for (int64_t j = 0; j < K; ++j) xt[t * K + j] = x[t * K + j] * inv_s[j];
+}
+
+/* ---- step 7: per-token dynamic activation quantization ------------------
+ * For token t: m_t = max_j |X~_tj|, dx_t = m_t/127,
+ * Xq[t][j] = clamp(rne(X~_tj * (127/m_t))). */
+void or_quant_act(const float *x, int64_t M, int64_t K, const float *inv_s,
+                  int8_t *xq, float *dx) {
+  for (int64_t t = 0; t < M; ++t) {
+    float m = 0.0f;
+    for (int64_t j = 0; j < K; ++j) {
+      float v = fabsf(x[t * K + j] * inv_s[j]);
+      if (v > m) m = v;
+    }
+    if (m == 0.0f) {
+      dx[t] = 0.0f;
+      for (int64_t j = 0; j < K; ++j) xq[t * K + j] = 0;
+      continue;
+    }
+    dx[t] = m / 127.0f;
+    float r = 127.0f / m;
+    for (int64_t j = 0; j < K; ++j)
+      xq[t * K + j] = or_quantize_value(x[t * K + j] * inv_s[j], r);
+  }
+}
+
+/* ---- step 8: INT8 x INT8 -> int32 matrix product ------------------------
+ * acc[t][n] = sum_j Xq[t][j] * Wq[n][j]: exact integer arithmetic. */
+void or_gemm_i8(const int8_t *xq, const int8_t *wq, int64_t M, int64_t N,
+                int64_t K, int32_t *acc) {
+  for (int64_t t = 0; t < M; ++t)
+    for (int64_t n = 0; n < N; ++n) {
+      int32_t sum = 0;
+      for (int64_t j = 0; j < K; ++j)
+        sum += (int32_t)xq[t * K + j] * (int32_t)wq[n * K + j];
+      acc[t * N + n] = sum;
+    }
+}
+
+/* ---- step 9: dequantization ---------------------------------------------
+ * y[t][n] = ((float)acc[t][n] * dx_t) * dw_n, fp32. */
+void or_dequant(const int32_t *acc, const float *dx, const float *dw,
+                int64_t M, int64_t N, float *y) {
+  for (int64_t t = 0; t < M; ++t)
+    for (int64_t n = 0; n < N; ++n) {
+      float a = (float)acc[t * N + n];
+      y[t * N + n] = (a * dx[t]) * dw[n];
+    }
+}
+
+/* ---- output rounding ----------------------------------------------------
+ * fp32 -> bfloat16, round to nearest even on the dropped 16 bits
+ * (NaN kept quiet). */
+void or_round_bf16(const float *y, int64_t count, uint16_t *out) {
+  for (int64_t i = 0; i < count; ++i) {
+    uint32_t u;
+    memcpy(&u, &y[i], 4);
+    if ((u & 0x7fffffffu) > 0x7f800000u) {
+      out[i] = (uint16_t)((u >> 16) | 0x40u);
+      continue;
+    }
+    uint32_t lsb = (u >> 16) & 1u;
+    u += 0x7fffu + lsb;
+    out[i] = (uint16_t)(u >> 16);
+  }
+}
+
+/* fp32 -> IEEE binary16 with the compiler's round-to-nearest-even cast. */
+void or_round_f16(const float *y, int64_t count, uint16_t *out) {
+  for (int64_t i = 0; i < count; ++i) {
+    _Float16 h = (_Float16)y[i];
+    memcpy(&out[i], &h, 2);
+  }
+}

@@ -1,0 +1,321 @@
+"""Pins for the CPU oracle: checks against what the SmoothQuant glossary page
+(jisaku.com, "SmoothQuant (activation smoothing quantization)") and plain
+mathematics fix, never against the oracle itself.
+
+- worked examples built from the page's printed channel values ("Why
+  activation quantization is hard"), worked by hand (tests/golden/);
+- the smoothing identity Y = (X diag(s)^-1)(diag(s) W) ("The mathematics of
+  the smoothing transformation") to fp32 rounding;
+- closed-form invariants of s_j = max|X_j|^a / max|W_j|^(1-a) ("Hyper-
+  parameter alpha") including the alpha = 0 and alpha = 1 limits;
+- the defining property of round-to-nearest quantization on a uniform grid;
+- brute-force integer matrix products and library reductions/conversions.
+"""
+from decimal import Decimal, getcontext
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from tests.golden.load import load
+
+getcontext().prec = 40
+KN, NK = oracle.LAYOUT_KN, oracle.LAYOUT_NK
+F32_EPS = float(np.finfo(np.float32).eps)  # 2^-23
+
+
+def _fl(rows):
+    if rows and isinstance(rows[0], list):
+        return np.array([[float(v) for v in r] for r in rows], np.float64)
+    return np.array([float(v) for v in rows], np.float64)
+
+
+def _int(rows):
+    if rows and isinstance(rows[0], list):
+        return np.array([[int(v) for v in r] for r in rows], np.int64)
+    return np.array([int(v) for v in rows], np.int64)
+
+
+def _ulps(got, exact):
+    """Distance of fp32 'got' from the exact value, in fp32 ulps of exact."""
+    got = np.asarray(got, np.float64)
+    exact = np.asarray(exact, np.float64)
+    ulp = np.spacing(np.abs(exact).astype(np.float32)).astype(np.float64)
+    return np.abs(got - exact) / ulp
+
+
+# ---------------------------------------------------------------------------
+# worked examples (tests/golden)
+# ---------------------------------------------------------------------------
+
+def test_p5_page_channels_worked_example():
+    g = load("p5_outlier_channel_example.txt")
+    x = _fl(g["x"]).astype(np.float32)
+    w = _fl(g["w_kn"]).astype(np.float32)
+    alpha = float(g["alpha"][0])
+    r = oracle.pipeline([x], w, KN, alpha, x, "f32")
+
+    # channel maxima are exact selections of input values
+    np.testing.assert_array_equal(r["amax"], _fl(g["a"]).astype(np.float32))
+    np.testing.assert_array_equal(r["wmax"], _fl(g["wmax"]).astype(np.float32))
+    # s from three IEEE-rounded operations on rounded inputs: a few ulps
+    assert _ulps(r["s"], _fl(g["s"])).max() <= 4
+    smoothed_x_max = r["amax"].astype(np.float64) * r["inv_s"]
+    assert _ulps(smoothed_x_max, _fl(g["smoothed_channel_max"])).max() <= 8
+    assert _ulps(r["dw"], _fl(g["dw"])).max() <= 8
+    assert _ulps(r["dx"], _fl(g["dx"])).max() <= 8
+    # integer codes and accumulators: exact
+    np.testing.assert_array_equal(r["wq"], _int(g["wq_nk"]))
+    np.testing.assert_array_equal(r["xq"], _int(g["xq"]))
+    np.testing.assert_array_equal(r["acc"], _int(g["acc"]))
+    # without smoothing (s = 1) the normal channel collapses as the page says
+    xq0, _ = oracle.quant_act(x, np.ones(2, np.float32))
+    np.testing.assert_array_equal(xq0, _int(g["xq_unsmoothed"]))
+
+    # Y against the exact product, within the rounding-error bound of
+    # quantizing both smoothed operands to their grids
+    y_exact = _fl(g["y_exact"])
+    xt = x.astype(np.float64) / _fl(g["s"])[None, :]
+    wt = _fl(g["s"])[:, None] * w.astype(np.float64)
+    dx = _fl(g["dx"])
+    dw = _fl(g["dw"])
+    bound = (np.abs(xt) @ np.ones_like(wt)) * dw[None, :] / 2 \
+        + dx[:, None] * (np.ones_like(xt) @ np.abs(wt)) / 2 \
+        + dx[:, None] * dw[None, :] * x.shape[1] / 4
+    assert np.all(np.abs(r["y"] - y_exact) <= bound * 1.001 + 1e-6)
+
+
+def test_p4_round_half_to_even_ties():
+    g = load("p4_rne_ties.txt")
+    x = _fl(g["x"]).astype(np.float32)[None, :]
+    xq, dx = oracle.quant_act(x, np.ones(x.shape[1], np.float32))
+    np.testing.assert_array_equal(xq[0], _int(g["xq"]))
+    assert dx[0] == np.float32(float(g["dx"][0]))
+
+
+def test_p6_outlier_x100_spread_and_codes():
+    g = load("p6_outlier_x100.txt")
+    x = _fl(g["x"]).astype(np.float32)
+    w = _fl(g["w_kn"]).astype(np.float32)
+    r = oracle.pipeline([x], w, KN, float(g["alpha"][0]), x, "f32")
+    np.testing.assert_array_equal(r["amax"], _fl(g["a"]).astype(np.float32))
+    np.testing.assert_array_equal(r["wmax"], _fl(g["wmax"]).astype(np.float32))
+    smoothed = r["amax"].astype(np.float64) * r["inv_s"]
+    assert _ulps(smoothed, _fl(g["smoothed_channel_max"])).max() <= 8
+    # the outlier channel's spread drops from 100x to 10x
+    assert abs(smoothed[3] / smoothed[0] - 10.0) < 1e-5
+    np.testing.assert_array_equal(r["xq"][0], _int(g["xq_token0"]))
+    xq0, _ = oracle.quant_act(x, np.ones(4, np.float32))
+    np.testing.assert_array_equal(xq0[0], _int(g["xq_token0_unsmoothed"]))
+    # every non-outlier code of an outlier token collapses to |q| <= 1
+    assert np.abs(xq0[0, :3]).max() <= 1
+
+
+# ---------------------------------------------------------------------------
+# smoothing identity and alpha invariants
+# ---------------------------------------------------------------------------
+
+ALPHAS = [0.0, 0.25, 0.5, 0.75, 1.0, 0.3, 0.85]
+
+
+@pytest.mark.parametrize("alpha", ALPHAS)
+@pytest.mark.parametrize("layout", [KN, NK])
+def test_p1_smoothing_identity(alpha, layout):
+    rng = np.random.default_rng(11)
+    x = rng.standard_normal((4, 8)).astype(np.float32)
+    x[:, 3] *= 100.0
+    w_kn = (rng.standard_normal((8, 3)) * 0.02).astype(np.float32)
+    w = w_kn if layout == KN else np.ascontiguousarray(w_kn.T)
+    amax = oracle.calib_absmax(x)
+    wmax = oracle.weight_absmax(w, layout)
+    s, inv_s = oracle.smooth_factor(amax, wmax, alpha)
+    xt = oracle.smooth_act(x, inv_s).astype(np.float64)
+    wt = oracle.smooth_weight(w, layout, s).astype(np.float64)
+    wt_kn = wt if layout == KN else wt.T
+    y = x.astype(np.float64) @ w_kn.astype(np.float64)
+    yt = xt @ wt_kn
+    # three fp32 roundings per term (1/s, x*inv_s, s*w) -> <= ~4 ulp per term
+    bound = 4 * F32_EPS * (np.abs(x).astype(np.float64) @ np.abs(w_kn).astype(np.float64))
+    assert np.all(np.abs(y - yt) <= bound + 1e-30)
+    # and a mistaken axis would break it by O(1): guard the bound is tight
+    assert bound.max() < 1e-4 * np.abs(y).max() + 1e-30
+
+
+@pytest.mark.parametrize("alpha", ALPHAS)
+def test_p2_alpha_invariants(alpha):
+    rng = np.random.default_rng(5)
+    K = 257
+    a = np.exp(rng.uniform(-3, 5, K)).astype(np.float32)
+    w = np.exp(rng.uniform(-6, 0, K)).astype(np.float32)
+    s, inv_s = oracle.smooth_factor(a, w, alpha)
+    a64, w64 = a.astype(np.float64), w.astype(np.float64)
+    xmax = a64 * inv_s.astype(np.float64)  # max|X~_j|
+    wmax_t = s.astype(np.float64) * w64     # max|W~_j|
+    # product of the two smoothed maxima is invariant for every alpha
+    np.testing.assert_allclose(xmax * wmax_t, a64 * w64, rtol=8 * F32_EPS)
+    # s against the formula evaluated in fp64 at the fp32 value of alpha
+    a32 = float(np.float32(alpha))
+    s_exact = a64 ** a32 / w64 ** (1 - a32)
+    assert _ulps(s, s_exact).max() <= (1 if alpha not in (0.25, 0.5, 0.75) else 4)
+    if alpha == 1.0:    # all difficulty moved to W: activations max to 1
+        np.testing.assert_allclose(xmax, 1.0, rtol=2 * F32_EPS)
+    if alpha == 0.0:    # all difficulty kept on X: weights max to 1
+        np.testing.assert_allclose(wmax_t, 1.0, rtol=2 * F32_EPS)
+    if alpha == 0.5:    # even split: both equal sqrt(a w)
+        np.testing.assert_allclose(xmax, np.sqrt(a64 * w64), rtol=6 * F32_EPS)
+        np.testing.assert_allclose(wmax_t, np.sqrt(a64 * w64), rtol=6 * F32_EPS)
+    np.testing.assert_array_equal(inv_s, (np.float32(1) / s).astype(np.float32))
+
+
+def test_smooth_factor_floor_on_empty_channels():
+    a = np.array([0.0, 3.0, 0.0], np.float32)
+    w = np.array([0.2, 0.0, 0.0], np.float32)
+    s, inv_s = oracle.smooth_factor(a, w, 0.5)
+    assert np.all(np.isfinite(s)) and np.all(np.isfinite(inv_s)) and np.all(s > 0)
+    np.testing.assert_allclose(s, np.sqrt([1e-5 / 0.2, 3.0 / 1e-5, 1.0]), rtol=1e-6)
+
+
+# ---------------------------------------------------------------------------
+# reductions against library routines
+# ---------------------------------------------------------------------------
+
+def test_calib_absmax_matches_library_and_is_running():
+    rng = np.random.default_rng(1)
+    x = rng.standard_normal((300, 96)).astype(np.float32)
+    x[:, 7] *= -100
+    full = oracle.calib_absmax(x)
+    np.testing.assert_array_equal(full, np.abs(x).max(axis=0))
+    run = oracle.calib_absmax(x[:100])
+    run = oracle.calib_absmax(x[100:250], run)
+    run = oracle.calib_absmax(x[250:], run)
+    np.testing.assert_array_equal(run, full)
+
+
+def test_weight_absmax_both_layouts():
+    rng = np.random.default_rng(2)
+    w_kn = rng.standard_normal((40, 24)).astype(np.float32)
+    np.testing.assert_array_equal(oracle.weight_absmax(w_kn, KN), np.abs(w_kn).max(axis=1))
+    np.testing.assert_array_equal(oracle.weight_absmax(np.ascontiguousarray(w_kn.T), NK),
+                                  np.abs(w_kn).max(axis=1))
+
+
+# ---------------------------------------------------------------------------
+# quantizers: defining property of rounding to a uniform symmetric grid
+# ---------------------------------------------------------------------------
+
+def test_quantize_value_saturation_and_ties():
+    assert oracle.quantize_value(200.0, 1.0) == 127
+    assert oracle.quantize_value(-200.0, 1.0) == -127
+    assert oracle.quantize_value(-128.0, 1.0) == -127
+    assert oracle.quantize_value(126.5, 1.0) == 126
+    assert oracle.quantize_value(-125.5, 1.0) == -126
+    assert oracle.quantize_value(0.49999997, 1.0) == 0
+
+
+def test_quant_act_grid_property_and_zero_rows():
+    rng = np.random.default_rng(3)
+    M, K = 37, 160
+    x = rng.standard_normal((M, K)).astype(np.float32)
+    x[:, [3, 77]] *= 100
+    x[5] = 0.0
+    inv_s = np.exp(rng.uniform(-2, 2, K)).astype(np.float32)
+    xq, dx = oracle.quant_act(x, inv_s)
+    xt = x.astype(np.float64) * inv_s.astype(np.float64)
+    for t in range(M):
+        if t == 5:
+            assert dx[t] == 0 and not xq[t].any()
+            continue
+        assert np.abs(xq[t]).max() == 127       # per-token: each row reaches 127
+        err = np.abs(xt[t] - xq[t].astype(np.float64) * dx[t])
+        assert err.max() <= dx[t] * 0.5 * (1 + 1e-5) + 1e-12
+        np.testing.assert_allclose(dx[t], np.abs(xt[t]).max() / 127, rtol=4 * F32_EPS)
+
+
+@pytest.mark.parametrize("layout", [KN, NK])
+def test_weight_quant_grid_property_per_output_channel(layout):
+    rng = np.random.default_rng(4)
+    K, N = 96, 48
+    w_kn = (rng.standard_normal((K, N)) * 0.02).astype(np.float32)
+    w_kn[:, 9] = 0.0
+    w = w_kn if layout == KN else np.ascontiguousarray(w_kn.T)
+    s = np.exp(rng.uniform(-2, 2, K)).astype(np.float32)
+    wq, dw = oracle.smooth_quant_weight(w, layout, s)
+    assert wq.shape == (N, K)
+    wt = s.astype(np.float64)[:, None] * w_kn.astype(np.float64)  # [K, N]
+    for n in range(N):
+        if n == 9:
+            assert dw[n] == 0 and not wq[n].any()
+            continue
+        assert np.abs(wq[n]).max() == 127
+        err = np.abs(wt[:, n] - wq[n].astype(np.float64) * dw[n])
+        assert err.max() <= dw[n] * 0.5 * (1 + 1e-5) + 1e-12
+    # both layouts give the same codes
+    other = np.ascontiguousarray(w.T)
+    wq2, dw2 = oracle.smooth_quant_weight(other, NK if layout == KN else KN, s)
+    np.testing.assert_array_equal(wq, wq2)
+    np.testing.assert_array_equal(dw, dw2)
+
+
+# ---------------------------------------------------------------------------
+# integer product and epilogue
+# ---------------------------------------------------------------------------
+
+def test_p3_gemm_brute_force_small():
+    rng = np.random.default_rng(6)
+    M, N, K = 3, 4, 5
+    xq = rng.integers(-127, 128, (M, K), dtype=np.int8)
+    wq = rng.integers(-127, 128, (N, K), dtype=np.int8)
+    acc = oracle.gemm_i8(xq, wq)
+    for t in range(M):
+        for n in range(N):
+            assert acc[t, n] == sum(int(xq[t, j]) * int(wq[n, j]) for j in range(K))
+
+
+def test_p3_gemm_against_int64_matmul_and_extremes():
+    rng = np.random.default_rng(7)
+    M, N, K = 33, 40, 272
+    xq = rng.integers(-127, 128, (M, K), dtype=np.int8)
+    wq = rng.integers(-127, 128, (N, K), dtype=np.int8)
+    np.testing.assert_array_equal(oracle.gemm_i8(xq, wq), xq.astype(np.int64) @ wq.astype(np.int64).T)
+    K = 28672  # largest K in the workloads: 127*127*K still fits in int32
+    xe = np.full((2, K), 127, np.int8)
+    xe[1] = -127
+    we = np.full((1, K), 127, np.int8)
+    np.testing.assert_array_equal(oracle.gemm_i8(xe, we)[:, 0], [127 * 127 * K, -127 * 127 * K])
+
+
+def test_dequant_exact_on_power_of_two_scales():
+    acc = np.array([[1, -2, 3], [40000, -7, 0]], np.int32)
+    dx = np.array([0.5, 2.0 ** -10], np.float32)
+    dw = np.array([4.0, 2.0 ** -3, 1.0], np.float32)
+    y = oracle.dequant(acc, dx, dw)
+    np.testing.assert_array_equal(y, acc.astype(np.float64) * dx[:, None] * dw[None, :])
+
+
+def test_dequant_order_of_rounding():
+    # (float)acc * dx is rounded before * dw: values chosen so the two
+    # groupings differ in fp32
+    acc = np.array([[16777217]], np.int32)  # 2^24 + 1 -> rounds to 2^24 (even)
+    dx = np.array([1.0], np.float32)
+    dw = np.array([1.0], np.float32)
+    assert oracle.dequant(acc, dx, dw)[0, 0] == np.float32(16777216.0)
+    acc = np.array([[3]], np.int32)
+    dx = np.array([np.float32(1.0) / np.float32(3.0)], np.float32)
+    dw = np.array([3.0], np.float32)
+    left = (np.float32(3.0) * dx[0]) * np.float32(3.0)
+    assert oracle.dequant(acc, dx, dw)[0, 0] == left
+
+
+def test_output_rounding_matches_library_conversions():
+    rng = np.random.default_rng(8)
+    y = (rng.standard_normal(4000) * np.exp(rng.uniform(-20, 20, 4000))).astype(np.float32)
+    # exact ties for bf16 (low 16 bits = 0x8000) and for f16
+    ties = np.array([1.0 + 2.0 ** -8, 1.0 + 3 * 2.0 ** -8, -(1.0 + 2.0 ** -8),
+                     1.0 + 2.0 ** -11, 1.0 + 3 * 2.0 ** -11, 65504.0, 1e-8], np.float32)
+    y = np.concatenate([y, ties])
+    bf = oracle.round_to(y, "bf16")
+    ref_bf = torch.from_numpy(y).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    np.testing.assert_array_equal(bf, ref_bf)
+    h = oracle.round_to(y, "f16")
+    np.testing.assert_array_equal(h, y.astype(np.float16).view(np.uint16))
