@@ -1,0 +1,165 @@
+/*
+ * sq.h -- C ABI of libsq.so, the sm_100a (B200) implementation of the
+ * SmoothQuant W8A8 smoothed linear layer.
+ *
+ * Method ("SmoothQuant (activation smoothing quantization)", jisaku.com
+ * glossary page):
+ *   - "The mathematics of the smoothing transformation":
+ *       Y = X W = (X diag(s)^-1)(diag(s) W) = X~ W~
+ *   - "Hyper-parameter alpha (migration strength)":
+ *       s_j = max|X_j|^alpha / max|W_j|^(1-alpha), alpha = 0.5 by default
+ *   - "Why activation quantization is hard": INT8 codes, a row is scaled so
+ *     that its largest magnitude maps to 127
+ *   - comparison table: the product runs directly on INT8 tensor cores
+ *   - usage example: get_act_scales (calibration) -> smooth_lm(alpha)
+ *     -> quantize_model.
+ * The four compute calls below follow that order.
+ *
+ * Conventions shared by every call
+ *   - Every data pointer is DEVICE memory on the current device, allocated
+ *     and owned by the caller.  The library allocates nothing, never
+ *     synchronises, and enqueues all work on `stream` (asynchronous with
+ *     respect to the host).  Buffers must stay alive until the work ends.
+ *   - Matrices are row-major with a leading dimension `ld*` counted in
+ *     ELEMENTS of the matrix's own type.
+ *   - Alignment: every pointer 16-byte aligned; every leading dimension a
+ *     multiple of 16 bytes; K and N multiples of 16.
+ *   - Arithmetic is IEEE fp32 with round-to-nearest-even; no operation is
+ *     contracted into an FMA.  INT8 codes, scales, s and int32 sums are
+ *     therefore reproducible bit for bit on any input.
+ *   - Quantization of a row v with absmax m: scale = m / 127 and
+ *     q = clamp(rne(v * (127 / m)), -127, 127); an all-zero row gives
+ *     scale 0 and codes 0.  -128 is never produced.
+ *   - Inputs must be finite; NaN/Inf give unspecified results.
+ *   - Errors: argument checks run on the host before anything is enqueued
+ *     and return SQ_ERR_INVALID_ARG / SQ_ERR_UNSUPPORTED with no side
+ *     effect.  A failed launch returns SQ_ERR_CUDA.  Work that is empty
+ *     (T == 0 or M == 0) returns SQ_OK and enqueues nothing.  Every wait
+ *     inside a kernel is bounded in time; a wait that runs out makes the
+ *     kernel stop and records SQ_ERR_TIMEOUT, which sq_check_device_error
+ *     reports.  No C++ exception crosses this interface.
+ */
+#ifndef SQ_H_
+#define SQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t / CUstream; NULL is the legacy default stream. */
+typedef struct CUstream_st *sq_stream_t;
+
+typedef enum {
+  SQ_OK = 0,
+  SQ_ERR_INVALID_ARG = 1, /* null pointer, bad size, alignment or alpha   */
+  SQ_ERR_UNSUPPORTED = 2, /* valid request this build does not implement  */
+  SQ_ERR_CUDA = 3,        /* a CUDA runtime/driver call failed            */
+  SQ_ERR_TIMEOUT = 4      /* a bounded in-kernel wait ran out             */
+} sq_status;
+
+typedef enum { SQ_F32 = 0, SQ_F16 = 1, SQ_BF16 = 2 } sq_dtype;
+
+/* Layout of the weight matrix W (input channel j, output channel n). */
+typedef enum {
+  SQ_W_KN = 0, /* W[K][N]: Y = X W as the page writes it            */
+  SQ_W_NK = 1  /* W[N][K]: output-major, as torch.nn.Linear stores it */
+} sq_wlayout;
+
+/*
+ * Calibration: running per-input-channel activation maximum
+ * (get_act_scales in the page's usage example; the max|X_j| of the alpha
+ * formula).
+ *   x     [T][ldx] of type xt (f32/f16/bf16), T tokens of K channels.
+ *   amax  [K] fp32, in-out: amax_j <- max(amax_j, max_t |x_tj|).  The caller
+ *         zero-fills it once and then calls this once per calibration chunk;
+ *         max is exact and order-free, so any chunking gives the same bits.
+ * T == 0 is a no-op.  K % 16 == 0, ldx >= K.
+ */
+sq_status sq_calib_absmax(const void *x, sq_dtype xt, int64_t T, int64_t K,
+                          int64_t ldx, float *amax, sq_stream_t stream);
+
+/*
+ * Smoothing and weight quantization (smooth_lm(alpha) then quantize_model).
+ *   w         weights of type wt; layout SQ_W_KN: [K][ldw], SQ_W_NK: [N][ldw].
+ *   amax      [K] fp32 calibration maxima from sq_calib_absmax.
+ *   alpha     migration strength in [0, 1].
+ *   wq        [N][K] int8 OUT, K contiguous (row n = output channel n):
+ *             Wq = clamp(rne(W~ * 127 / max_j|W~_jn|)), W~ = diag(s) W.
+ *   w_scale   [N] fp32 OUT, per-output-channel scale max_j|W~_jn| / 127.
+ *   smooth    [K] fp32 OUT, s_j (also used as scratch during the call).
+ *   inv_smooth[K] fp32 OUT, 1/s_j (what sq_quant_act multiplies by).
+ * s_j uses a_j and w_j = max_n |W_jn| floored at 1e-5.  For alpha in
+ * {0, 0.25, 0.5, 0.75, 1} the power is formed from IEEE square roots
+ * (bit-reproducible); other alphas use double-precision pow, rounded once.
+ * K % 16 == 0, N % 16 == 0, ldw >= K (NK) or >= N (KN).
+ */
+sq_status sq_smooth_quant_weight(const void *w, sq_dtype wt, sq_wlayout layout,
+                                 int64_t K, int64_t N, int64_t ldw,
+                                 const float *amax, float alpha, int8_t *wq,
+                                 float *w_scale, float *smooth,
+                                 float *inv_smooth, sq_stream_t stream);
+
+/*
+ * Runtime activation smoothing and per-token dynamic quantization
+ * (X~ = X diag(s)^-1, then INT8 with the largest magnitude mapped to 127).
+ *   x          [M][ldx] of type xt.
+ *   inv_smooth [K] fp32 (from sq_smooth_quant_weight).
+ *   xq         [M][K] int8 OUT (row stride K).
+ *   x_scale    [M] fp32 OUT, max_j |x_tj * inv_s_j| / 127.
+ * M == 0 is a no-op.  K % 16 == 0, ldx >= K.
+ */
+sq_status sq_quant_act(const void *x, sq_dtype xt, int64_t M, int64_t K,
+                       int64_t ldx, const float *inv_smooth, int8_t *xq,
+                       float *x_scale, sq_stream_t stream);
+
+/*
+ * W8A8 linear on the tensor cores (tcgen05, kind::i8): exact int32
+ * accumulation acc_tn = sum_j xq_tj * wq_nj, then the dequant epilogue
+ * y_tn = round_yt(((float)acc_tn * x_scale_t) * w_scale_n).
+ *   xq [M][K] int8, wq [N][K] int8, x_scale [M], w_scale [N] fp32.
+ *   y  [M][ldy] of type yt (f32/f16/bf16) OUT.
+ *   workspace / workspace_bytes: device scratch of at least
+ *         sq_w8a8_linear_workspace_size(M, N, K) bytes, which must be ZERO
+ *         on the first call; the library leaves it zero again when each
+ *         call ends.  May be NULL when that size is 0.  Calls that share a
+ *         workspace must be stream-ordered.
+ * M == 0 is a no-op.  K % 16 == 0, N % 16 == 0, ldy >= N.
+ */
+sq_status sq_w8a8_linear(const int8_t *xq, const float *x_scale,
+                         const int8_t *wq, const float *w_scale, int64_t M,
+                         int64_t N, int64_t K, void *y, sq_dtype yt,
+                         int64_t ldy, void *workspace, size_t workspace_bytes,
+                         sq_stream_t stream);
+
+/* Bytes of workspace sq_w8a8_linear needs for this shape (0 if none). */
+size_t sq_w8a8_linear_workspace_size(int64_t M, int64_t N, int64_t K);
+
+/*
+ * The integer product alone: acc[M][ldacc] int32 OUT = xq . wq^T, computed
+ * by the same tensor-core kernels as sq_w8a8_linear (same tiling and
+ * dispatch on M), for verifying the exact accumulators.  Same workspace
+ * contract as sq_w8a8_linear.
+ */
+sq_status sq_w8a8_accumulate(const int8_t *xq, const int8_t *wq, int64_t M,
+                             int64_t N, int64_t K, int32_t *acc, int64_t ldacc,
+                             void *workspace, size_t workspace_bytes,
+                             sq_stream_t stream);
+
+/*
+ * Synchronises `stream`, then reports (and clears) a timeout that any
+ * kernel of this library recorded on the current device since the last
+ * check: SQ_ERR_TIMEOUT, else SQ_OK (or SQ_ERR_CUDA if the sync failed).
+ */
+sq_status sq_check_device_error(sq_stream_t stream);
+
+/* Static, human-readable name of a status code. */
+const char *sq_status_string(sq_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SQ_H_ */

@@ -1,0 +1,118 @@
+"""The C ABI without a GPU: the library loads, exports every function the
+header declares, and rejects invalid arguments on the host before touching
+CUDA (each call below returns before its first CUDA call)."""
+import ctypes
+
+import pytest
+
+import w8a8_post_quantization_channel_b200 as sq
+
+INV = sq.SQ_ERR_INVALID_ARG
+A16 = 1 << 20          # a fake, 16-byte aligned address (never dereferenced)
+MIS = (1 << 20) + 4    # misaligned
+
+
+def test_library_exports_every_header_function():
+    names = sq.header_functions()
+    assert {"sq_calib_absmax", "sq_smooth_quant_weight", "sq_quant_act", "sq_w8a8_linear",
+            "sq_w8a8_linear_workspace_size", "sq_w8a8_accumulate", "sq_check_device_error",
+            "sq_status_string"} <= set(names)
+    L = sq.lib()
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_status_strings():
+    for code in range(5):
+        s = sq.sq_status_string(code)
+        assert s.startswith("SQ_")
+    assert "unknown" in sq.sq_status_string(99)
+
+
+def test_calib_argument_checks():
+    L = sq.lib()
+    f = L.sq_calib_absmax
+    assert f(A16, sq.SQ_BF16, 0, 256, 256, A16, None) == sq.SQ_OK        # empty stream: no-op
+    assert f(None, sq.SQ_BF16, 0, 256, 256, A16, None) == sq.SQ_OK       # x unused when T == 0
+    assert f(None, sq.SQ_BF16, 4, 256, 256, A16, None) == INV             # null x
+    assert f(A16, sq.SQ_BF16, 4, 256, 256, None, None) == INV             # null amax
+    assert f(A16, sq.SQ_BF16, 4, 250, 256, A16, None) == INV              # K % 16
+    assert f(A16, sq.SQ_BF16, 4, 256, 255, A16, None) == INV              # ld < K / unaligned rows
+    assert f(A16, sq.SQ_BF16, 4, 256, 260, A16, None) == INV              # row stride 520 B not 16-B multiple
+    assert f(MIS, sq.SQ_BF16, 4, 256, 256, A16, None) == INV              # misaligned x
+    assert f(A16, 7, 4, 256, 256, A16, None) == INV                       # bad dtype
+    assert f(A16, sq.SQ_F32, -1, 256, 256, A16, None) == INV              # negative T
+    assert f(A16, sq.SQ_F32, 4, 0, 256, A16, None) == INV                 # K == 0
+
+
+def test_smooth_quant_weight_argument_checks():
+    f = sq.lib().sq_smooth_quant_weight
+    ok = dict(w=A16, wt=sq.SQ_F16, lay=sq.SQ_W_NK, K=256, N=512, ld=256, amax=A16, alpha=0.5,
+              wq=A16, ws=A16, s=A16, inv=A16)
+
+    def call(**kw):
+        a = dict(ok)
+        a.update(kw)
+        return f(a["w"], a["wt"], a["lay"], a["K"], a["N"], a["ld"], a["amax"], ctypes.c_float(a["alpha"]),
+                 a["wq"], a["ws"], a["s"], a["inv"], None)
+
+    assert call(alpha=-0.1) == INV
+    assert call(alpha=1.5) == INV
+    assert call(alpha=float("nan")) == INV
+    assert call(lay=3) == INV
+    assert call(N=500) == INV
+    assert call(K=248) == INV
+    assert call(ld=128) == INV                 # NK: ld >= K
+    assert call(lay=sq.SQ_W_KN, ld=256) == INV  # KN: ld >= N = 512
+    assert call(w=None) == INV
+    assert call(wq=None) == INV
+    assert call(ws=MIS) == INV
+    assert call(s=None) == INV
+    assert call(inv=None) == INV
+    assert call(amax=None) == INV
+
+
+def test_quant_act_argument_checks():
+    f = sq.lib().sq_quant_act
+    assert f(None, sq.SQ_BF16, 0, 256, 256, A16, None, None, None) == sq.SQ_OK
+    assert f(A16, sq.SQ_BF16, 8, 256, 256, None, A16, A16, None) == INV
+    assert f(A16, sq.SQ_BF16, 8, 256, 256, A16, None, A16, None) == INV
+    assert f(A16, sq.SQ_BF16, 8, 256, 256, A16, A16, None, None) == INV
+    assert f(A16, sq.SQ_BF16, 8, 24, 24, A16, A16, A16, None) == INV
+    assert f(MIS, sq.SQ_F32, 8, 256, 256, A16, A16, A16, None) == INV
+
+
+def test_linear_argument_checks():
+    f = sq.lib().sq_w8a8_linear
+    base = [A16, A16, A16, A16, 64, 256, 256, A16, sq.SQ_BF16, 256, None, 0, None]
+
+    def call(i, v):
+        a = list(base)
+        a[i] = v
+        return f(*a)
+
+    assert call(4, 0) == sq.SQ_OK          # M == 0: no-op
+    assert call(5, 40) == INV              # N % 16
+    assert call(6, 40) == INV              # K % 16
+    assert call(9, 128) == INV             # ldy < N
+    assert call(8, 9) == INV               # bad output dtype
+    assert call(0, None) == INV
+    assert call(2, None) == INV
+    assert call(3, None) == INV
+    assert call(7, MIS) == INV
+    acc = sq.lib().sq_w8a8_accumulate
+    assert acc(A16, A16, 0, 256, 256, A16, 256, None, 0, None) == sq.SQ_OK
+    assert acc(A16, A16, 4, 256, 256, None, 256, None, 0, None) == INV
+    assert acc(A16, A16, 4, 256, 256, A16, 100, None, 0, None) == INV
+
+
+def test_workspace_size_is_defined_for_all_shapes():
+    for M in (0, 1, 8, 64, 128, 2048):
+        for N, K in ((256, 256), (4096, 4096), (28672, 8192)):
+            assert sq.sq_w8a8_linear_workspace_size(M, N, K) >= 0
+
+
+def test_binding_rejects_host_tensors():
+    import torch
+    with pytest.raises(ValueError):
+        sq.sq_calib_absmax(torch.zeros(4, 16), torch.zeros(16))

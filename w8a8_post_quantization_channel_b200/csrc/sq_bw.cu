@@ -1,0 +1,393 @@
+// sq_bw.cu -- the bandwidth-bound steps of the SmoothQuant path (sm_100a).
+//
+//   calibration maxima  max_t |X_tj|              ("Hyper-parameter alpha":
+//   weight maxima       max_n |W_jn|               the max|X_j|, max|W_j|)
+//   smoothing factor    s_j = a_j^alpha / w_j^(1-alpha), 1/s_j
+//   row quantizer       per-token X~ = X / s and per-output-row W~ = s W
+//   column quantizer    per-output-channel W~ for W stored [K][N]
+// ("SmoothQuant (activation smoothing quantization)", jisaku.com glossary).
+//
+// Every kernel reads its input once with 16-byte vector loads, keeps
+// per-thread partial maxima in registers and merges them with warp
+// shuffles; results are independent of the launch shape (max is exact).
+#include <algorithm>
+
+#include "sq_common.cuh"
+#include "sq_internal.h"
+
+namespace sq {
+
+namespace {
+
+constexpr int kColThreadsX = 32;  // 16-byte column vectors per CTA slab
+constexpr int kColThreadsY = 8;   // row lanes per CTA
+constexpr int kColUnroll = 4;     // independent row loads in flight per thread
+
+// amax[c] = max(amax[c], max_r |v_rc|), v_rc = x[r][c] (* row_scale[r]).
+// CTA (32 x 8): threadIdx.x picks a 16-byte column vector of a 32-vector
+// slab, threadIdx.y a row lane; blockIdx.y splits the rows into chunks.
+template <typename T, bool kScaled>
+__global__ void __launch_bounds__(kColThreadsX *kColThreadsY)
+    absmax_cols_kernel(const T *__restrict__ x, int64_t rows, int64_t nvec, int64_t ld,
+                       const float *__restrict__ row_scale, float *__restrict__ amax) {
+  constexpr int V = Vec<T>::N;
+  __shared__ float red[kColThreadsY][kColThreadsX * V];
+  const int64_t v = (int64_t)blockIdx.x * kColThreadsX + threadIdx.x;
+  const int64_t chunk = (rows + gridDim.y - 1) / gridDim.y;
+  const int64_t r0 = (int64_t)blockIdx.y * chunk;
+  const int64_t r1 = min(rows, r0 + chunk);
+  float m[V];
+#pragma unroll
+  for (int e = 0; e < V; ++e) m[e] = 0.0f;
+  if (v < nvec) {
+    const T *col = x + v * V;
+    int64_t r = r0 + threadIdx.y;
+    for (; r + (kColUnroll - 1) * kColThreadsY < r1; r += kColUnroll * kColThreadsY) {
+      uint4 raw[kColUnroll];
+#pragma unroll
+      for (int u = 0; u < kColUnroll; ++u) raw[u] = ld_stream_v4(col + (r + u * kColThreadsY) * ld);
+#pragma unroll
+      for (int u = 0; u < kColUnroll; ++u) {
+        float f[V];
+        Vec<T>::to_f32(raw[u], f);
+        const float sc = kScaled ? __ldg(row_scale + r + u * kColThreadsY) : 1.0f;
+#pragma unroll
+        for (int e = 0; e < V; ++e) m[e] = fmaxf(m[e], fabsf(kScaled ? __fmul_rn(sc, f[e]) : f[e]));
+      }
+    }
+    for (; r < r1; r += kColThreadsY) {
+      float f[V];
+      Vec<T>::to_f32(ld_stream_v4(col + r * ld), f);
+      const float sc = kScaled ? __ldg(row_scale + r) : 1.0f;
+#pragma unroll
+      for (int e = 0; e < V; ++e) m[e] = fmaxf(m[e], fabsf(kScaled ? __fmul_rn(sc, f[e]) : f[e]));
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < V; ++e) red[threadIdx.y][threadIdx.x * V + e] = m[e];
+  __syncthreads();
+  // Threads of row lane 0 fold the 8 lanes and publish with an integer
+  // atomicMax: for non-negative floats the bit patterns order as integers.
+  if (threadIdx.y == 0 && v < nvec) {
+#pragma unroll
+    for (int e = 0; e < V; ++e) {
+      float mm = red[0][threadIdx.x * V + e];
+#pragma unroll
+      for (int y = 1; y < kColThreadsY; ++y) mm = fmaxf(mm, red[y][threadIdx.x * V + e]);
+      atomicMax(reinterpret_cast<int *>(amax + v * V + e), __float_as_int(mm));
+    }
+  }
+}
+
+// out[r] = max_c |x[r][c]|, one CTA per row.
+template <typename T>
+__global__ void __launch_bounds__(256) absmax_rows_kernel(const T *__restrict__ x, int64_t nvec, int64_t ld,
+                                                          float *__restrict__ out) {
+  constexpr int V = Vec<T>::N;
+  __shared__ float red[32];
+  const T *row = x + (int64_t)blockIdx.x * ld;
+  float m = 0.0f;
+  for (int64_t v = threadIdx.x; v < nvec; v += blockDim.x) {
+    float f[V];
+    Vec<T>::to_f32(ld_stream_v4(row + v * V), f);
+#pragma unroll
+    for (int e = 0; e < V; ++e) m = fmaxf(m, fabsf(f[e]));
+  }
+  m = block_max(m, red);
+  if (threadIdx.x == 0) out[blockIdx.x] = m;
+}
+
+// s_j = a^alpha / w^(1-alpha) with a, w floored at 1e-5; IEEE sqrt for the
+// quarter-step alphas, double pow (rounded once) otherwise.
+__global__ void smooth_factor_kernel(const float *__restrict__ amax, float *__restrict__ s_inout,
+                                     float *__restrict__ inv_s, int64_t K, float alpha) {
+  const int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (j >= K) return;
+  const float a = fmaxf(amax[j], 1e-5f);
+  const float w = fmaxf(s_inout[j], 1e-5f);
+  float s;
+  if (alpha == 1.0f) {
+    s = a;
+  } else if (alpha == 0.0f) {
+    s = __fdiv_rn(1.0f, w);
+  } else if (alpha == 0.5f) {
+    s = __fdiv_rn(__fsqrt_rn(a), __fsqrt_rn(w));
+  } else if (alpha == 0.25f) {
+    const float a14 = __fsqrt_rn(__fsqrt_rn(a));
+    const float w34 = __fmul_rn(__fsqrt_rn(w), __fsqrt_rn(__fsqrt_rn(w)));
+    s = __fdiv_rn(a14, w34);
+  } else if (alpha == 0.75f) {
+    const float a34 = __fmul_rn(__fsqrt_rn(a), __fsqrt_rn(__fsqrt_rn(a)));
+    const float w14 = __fsqrt_rn(__fsqrt_rn(w));
+    s = __fdiv_rn(a34, w14);
+  } else {
+    const double num = pow((double)a, (double)alpha);
+    const double den = pow((double)w, 1.0 - (double)alpha);
+    s = __double2float_rn(__ddiv_rn(num, den));
+  }
+  s_inout[j] = s;
+  inv_s[j] = __fdiv_rn(1.0f, s);
+}
+
+// Row quantizer, one CTA per row, the row held in registers:
+//   v_c = x[r][c] * col_scale[c];  m = max_c |v_c|;
+//   row_scale_out[r] = m / 127;  q[r][c] = clamp(rne(v_c * (127 / m))).
+// Thread t owns the 16-byte vectors t, t + blockDim, ... (kVPT of them).
+template <typename T, int kVPT>
+__global__ void __launch_bounds__(1024) quant_rows_kernel(const T *__restrict__ x, int64_t nvec, int64_t ld,
+                                                          const float *__restrict__ col_scale,
+                                                          int8_t *__restrict__ q, float *__restrict__ row_scale_out) {
+  constexpr int V = Vec<T>::N;
+  __shared__ float red[32];
+  const int64_t r = blockIdx.x;
+  const T *row = x + r * ld;
+  const int64_t K = nvec * V;
+  uint4 raw[kVPT];
+#pragma unroll
+  for (int i = 0; i < kVPT; ++i) {
+    const int64_t v = threadIdx.x + (int64_t)i * blockDim.x;
+    if (v < nvec) raw[i] = ld_stream_v4(row + v * V);
+  }
+  float val[kVPT][V];
+  float m = 0.0f;
+#pragma unroll
+  for (int i = 0; i < kVPT; ++i) {
+    const int64_t v = threadIdx.x + (int64_t)i * blockDim.x;
+    if (v < nvec) {
+      float f[V];
+      Vec<T>::to_f32(raw[i], f);
+      const float4 *sc4 = reinterpret_cast<const float4 *>(col_scale + v * V);
+#pragma unroll
+      for (int e4 = 0; e4 < V / 4; ++e4) {
+        const float4 s = __ldg(sc4 + e4);
+        val[i][4 * e4 + 0] = __fmul_rn(f[4 * e4 + 0], s.x);
+        val[i][4 * e4 + 1] = __fmul_rn(f[4 * e4 + 1], s.y);
+        val[i][4 * e4 + 2] = __fmul_rn(f[4 * e4 + 2], s.z);
+        val[i][4 * e4 + 3] = __fmul_rn(f[4 * e4 + 3], s.w);
+      }
+#pragma unroll
+      for (int e = 0; e < V; ++e) m = fmaxf(m, fabsf(val[i][e]));
+    }
+  }
+  m = block_max(m, red);
+  const bool zero = (m == 0.0f);
+  const float rcp = zero ? 0.0f : __fdiv_rn(127.0f, m);
+  if (threadIdx.x == 0) row_scale_out[r] = zero ? 0.0f : __fdiv_rn(m, 127.0f);
+  int8_t *qrow = q + r * K;
+#pragma unroll
+  for (int i = 0; i < kVPT; ++i) {
+    const int64_t v = threadIdx.x + (int64_t)i * blockDim.x;
+    if (v < nvec) {
+      int c[V];
+#pragma unroll
+      for (int e = 0; e < V; ++e) c[e] = zero ? 0 : quantize(val[i][e], rcp);
+      if constexpr (V == 8) {
+        uint2 o;
+        o.x = pack4_i8(c[0], c[1], c[2], c[3]);
+        o.y = pack4_i8(c[4], c[5], c[6], c[7]);
+        *reinterpret_cast<uint2 *>(qrow + v * V) = o;
+      } else {
+        *reinterpret_cast<uint32_t *>(qrow + v * V) = pack4_i8(c[0], c[1], c[2], c[3]);
+      }
+    }
+  }
+}
+
+// Row quantizer for rows too long to hold in registers: one pass for the
+// maximum, a second for the codes (the row is re-read, mostly from L2).
+template <typename T>
+__global__ void __launch_bounds__(1024) quant_rows_twopass_kernel(const T *__restrict__ x, int64_t nvec, int64_t ld,
+                                                                  const float *__restrict__ col_scale,
+                                                                  int8_t *__restrict__ q,
+                                                                  float *__restrict__ row_scale_out) {
+  constexpr int V = Vec<T>::N;
+  __shared__ float red[32];
+  const int64_t r = blockIdx.x;
+  const T *row = x + r * ld;
+  const int64_t K = nvec * V;
+  float m = 0.0f;
+  for (int64_t v = threadIdx.x; v < nvec; v += blockDim.x) {
+    float f[V];
+    Vec<T>::to_f32(ld_nc_v4(row + v * V), f);
+#pragma unroll
+    for (int e = 0; e < V; ++e) m = fmaxf(m, fabsf(__fmul_rn(f[e], __ldg(col_scale + v * V + e))));
+  }
+  m = block_max(m, red);
+  const bool zero = (m == 0.0f);
+  const float rcp = zero ? 0.0f : __fdiv_rn(127.0f, m);
+  if (threadIdx.x == 0) row_scale_out[r] = zero ? 0.0f : __fdiv_rn(m, 127.0f);
+  int8_t *qrow = q + r * K;
+  for (int64_t v = threadIdx.x; v < nvec; v += blockDim.x) {
+    float f[V];
+    Vec<T>::to_f32(ld_stream_v4(row + v * V), f);
+    int c[V];
+#pragma unroll
+    for (int e = 0; e < V; ++e) c[e] = zero ? 0 : quantize(__fmul_rn(f[e], __ldg(col_scale + v * V + e)), rcp);
+    if constexpr (V == 8) {
+      uint2 o;
+      o.x = pack4_i8(c[0], c[1], c[2], c[3]);
+      o.y = pack4_i8(c[4], c[5], c[6], c[7]);
+      *reinterpret_cast<uint2 *>(qrow + v * V) = o;
+    } else {
+      *reinterpret_cast<uint32_t *>(qrow + v * V) = pack4_i8(c[0], c[1], c[2], c[3]);
+    }
+  }
+}
+
+// W[K][N] (row j = input channel) -> Wq[N][K]: a 64 x 64 tile is read with
+// row-contiguous loads, quantized with its column's maximum, transposed in
+// shared memory and written with row-contiguous stores.
+constexpr int kTT = 64;
+template <typename T>
+__global__ void __launch_bounds__(256) quant_cols_transpose_kernel(const T *__restrict__ w, int64_t K, int64_t N,
+                                                                   int64_t ld, const float *__restrict__ s,
+                                                                   const float *__restrict__ colmax,
+                                                                   int8_t *__restrict__ wq) {
+  __shared__ int8_t tile[kTT][kTT + 4];  // [n][j]
+  const int64_t j0 = (int64_t)blockIdx.y * kTT, n0 = (int64_t)blockIdx.x * kTT;
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;  // 16 x 16 threads
+  // each thread: 4 consecutive n of one j row, rows ty, ty+16, ...
+#pragma unroll
+  for (int jj = ty; jj < kTT; jj += 16) {
+    const int64_t j = j0 + jj;
+    const int64_t n = n0 + tx * 4;
+    int c[4] = {0, 0, 0, 0};
+    if (j < K && n < N) {  // N % 16 == 0: a group of 4 is all in or all out
+      const float sj = __ldg(s + j);
+      const T *p = w + j * ld + n;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float cm = __ldg(colmax + n + e);
+        const float wv = Vec<T>::one(p + e);
+        c[e] = (cm == 0.0f) ? 0 : quantize(__fmul_rn(sj, wv), __fdiv_rn(127.0f, cm));
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) tile[tx * 4 + e][jj] = (int8_t)c[e];
+  }
+  __syncthreads();
+  // write: row n of the tile, 64 bytes of j; each thread 4 bytes
+#pragma unroll
+  for (int nn = ty; nn < kTT; nn += 16) {
+    const int64_t n = n0 + nn;
+    const int64_t j = j0 + tx * 4;
+    if (n < N && j < K) {
+      const uint32_t packed = pack4_i8(tile[nn][tx * 4 + 0], tile[nn][tx * 4 + 1], tile[nn][tx * 4 + 2],
+                                       tile[nn][tx * 4 + 3]);
+      *reinterpret_cast<uint32_t *>(wq + n * K + j) = packed;
+    }
+  }
+}
+
+__global__ void finalize_scale_kernel(float *__restrict__ m_to_scale, int64_t n) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) m_to_scale[i] = __fdiv_rn(m_to_scale[i], 127.0f);
+}
+
+template <typename T>
+cudaError_t absmax_cols_t(const void *x, int64_t rows, int64_t cols, int64_t ld, const float *row_scale,
+                          float *amax, cudaStream_t st) {
+  constexpr int V = Vec<T>::N;
+  const int64_t nvec = cols / V;
+  const int64_t slabs = (nvec + kColThreadsX - 1) / kColThreadsX;
+  const int64_t want = (int64_t)num_sms() * 8;
+  int64_t gy = (want + slabs - 1) / slabs;
+  const int64_t max_gy = (rows + kColUnroll * kColThreadsY - 1) / (kColUnroll * kColThreadsY);
+  gy = std::max<int64_t>(1, std::min<int64_t>(gy, std::min<int64_t>(max_gy, 65535)));
+  dim3 grid((unsigned)slabs, (unsigned)gy), block(kColThreadsX, kColThreadsY);
+  if (row_scale)
+    absmax_cols_kernel<T, true><<<grid, block, 0, st>>>((const T *)x, rows, nvec, ld, row_scale, amax);
+  else
+    absmax_cols_kernel<T, false><<<grid, block, 0, st>>>((const T *)x, rows, nvec, ld, nullptr, amax);
+  return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t absmax_rows_t(const void *x, int64_t rows, int64_t cols, int64_t ld, float *out, cudaStream_t st) {
+  constexpr int V = Vec<T>::N;
+  absmax_rows_kernel<T><<<(unsigned)rows, 256, 0, st>>>((const T *)x, cols / V, ld, out);
+  return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t quant_rows_t(const void *x, int64_t rows, int64_t cols, int64_t ld, const float *col_scale, int8_t *q,
+                         float *row_scale_out, cudaStream_t st) {
+  constexpr int V = Vec<T>::N;
+  const int64_t nvec = cols / V;
+  auto threads_for = [&](int vpt) {
+    int64_t t = (nvec + vpt - 1) / vpt;
+    t = ((t + 31) / 32) * 32;
+    return (int)std::max<int64_t>(32, t);
+  };
+  const T *xp = (const T *)x;
+  const unsigned g = (unsigned)rows;
+  if (threads_for(1) <= 256) {
+    quant_rows_kernel<T, 1><<<g, threads_for(1), 0, st>>>(xp, nvec, ld, col_scale, q, row_scale_out);
+  } else if (threads_for(2) <= 512) {
+    quant_rows_kernel<T, 2><<<g, threads_for(2), 0, st>>>(xp, nvec, ld, col_scale, q, row_scale_out);
+  } else if (threads_for(4) <= 512) {
+    quant_rows_kernel<T, 4><<<g, threads_for(4), 0, st>>>(xp, nvec, ld, col_scale, q, row_scale_out);
+  } else if (threads_for(4) <= 1024) {
+    quant_rows_kernel<T, 4><<<g, threads_for(4), 0, st>>>(xp, nvec, ld, col_scale, q, row_scale_out);
+  } else {
+    quant_rows_twopass_kernel<T><<<g, 1024, 0, st>>>(xp, nvec, ld, col_scale, q, row_scale_out);
+  }
+  return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t quant_cols_t(const void *w, int64_t K, int64_t N, int64_t ld, const float *s, float *colmax, int8_t *wq,
+                         cudaStream_t st) {
+  dim3 grid((unsigned)((N + kTT - 1) / kTT), (unsigned)((K + kTT - 1) / kTT));
+  quant_cols_transpose_kernel<T><<<grid, 256, 0, st>>>((const T *)w, K, N, ld, s, colmax, wq);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  finalize_scale_kernel<<<(unsigned)((N + 255) / 256), 256, 0, st>>>(colmax, N);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_absmax_cols(const void *x, sq_dtype xt, int64_t rows, int64_t cols, int64_t ld,
+                               const float *row_scale, float *amax, cudaStream_t st) {
+  switch (xt) {
+    case SQ_F32: return absmax_cols_t<float>(x, rows, cols, ld, row_scale, amax, st);
+    case SQ_F16: return absmax_cols_t<__half>(x, rows, cols, ld, row_scale, amax, st);
+    default: return absmax_cols_t<__nv_bfloat16>(x, rows, cols, ld, row_scale, amax, st);
+  }
+}
+
+cudaError_t launch_absmax_rows(const void *x, sq_dtype xt, int64_t rows, int64_t cols, int64_t ld, float *out,
+                               cudaStream_t st) {
+  switch (xt) {
+    case SQ_F32: return absmax_rows_t<float>(x, rows, cols, ld, out, st);
+    case SQ_F16: return absmax_rows_t<__half>(x, rows, cols, ld, out, st);
+    default: return absmax_rows_t<__nv_bfloat16>(x, rows, cols, ld, out, st);
+  }
+}
+
+cudaError_t launch_smooth_factor(const float *amax, float *s_inout, float *inv_s, int64_t K, float alpha,
+                                 cudaStream_t st) {
+  smooth_factor_kernel<<<(unsigned)((K + 255) / 256), 256, 0, st>>>(amax, s_inout, inv_s, K, alpha);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quant_rows(const void *x, sq_dtype xt, int64_t rows, int64_t cols, int64_t ld,
+                              const float *col_scale, int8_t *q, float *row_scale_out, cudaStream_t st) {
+  switch (xt) {
+    case SQ_F32: return quant_rows_t<float>(x, rows, cols, ld, col_scale, q, row_scale_out, st);
+    case SQ_F16: return quant_rows_t<__half>(x, rows, cols, ld, col_scale, q, row_scale_out, st);
+    default: return quant_rows_t<__nv_bfloat16>(x, rows, cols, ld, col_scale, q, row_scale_out, st);
+  }
+}
+
+cudaError_t launch_quant_cols_transpose(const void *w, sq_dtype wt, int64_t K, int64_t N, int64_t ld,
+                                        const float *s, float *colmax_to_scale, int8_t *wq, cudaStream_t st) {
+  switch (wt) {
+    case SQ_F32: return quant_cols_t<float>(w, K, N, ld, s, colmax_to_scale, wq, st);
+    case SQ_F16: return quant_cols_t<__half>(w, K, N, ld, s, colmax_to_scale, wq, st);
+    default: return quant_cols_t<__nv_bfloat16>(w, K, N, ld, s, colmax_to_scale, wq, st);
+  }
+}
+
+}  // namespace sq

@@ -1,0 +1,332 @@
+// sq_gemm.cu -- W8A8 linear on the 5th-generation tensor cores (sm_100a).
+//
+// acc_tn = sum_j Xq_tj * Wq_nj (int32, exact), then
+// y_tn = round(((float)acc_tn * dx_t) * dw_n).
+// The page's comparison table puts W8A8's gain in running the product
+// directly on INT8 tensor cores ("SmoothQuant (activation smoothing
+// quantization)", jisaku.com glossary, comparison with GPTQ/AWQ).
+//
+// Kernel structure (one CTA per SM, persistent over output tiles):
+//   warp 0      TMA producer: Xq and Wq tiles (K-major, 128-byte swizzle)
+//               into a STAGES-deep shared-memory ring;
+//   warp 1      allocates TMEM; one thread issues tcgen05.mma kind::i8
+//               (M=128, N=BN, K=32 per instruction) into one of two TMEM
+//               accumulators and signals the ring / epilogue with
+//               tcgen05.commit;
+//   warps 2-5   epilogue: tcgen05.ld of the finished accumulator (one TMEM
+//               lane quarter per warp), fp32 dequant, rounding, stores;
+//               the other accumulator is filled by the MMA meanwhile.
+// Every mbarrier wait is bounded (see mbar_wait); on a timeout the roles
+// stop, in-flight copies and MMAs are drained, TMEM is freed.
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "sq_common.cuh"
+#include "sq_internal.h"
+
+namespace sq {
+
+namespace {
+
+constexpr int kBM = 128;  // rows of Xq per tile (= TMEM lanes)
+constexpr int kBK = 128;  // K bytes per stage (one 128-byte swizzle row)
+constexpr int kThreads = 192;
+
+template <int BN, int STAGES>
+struct GemmSmem {
+  static constexpr uint32_t kA = kBM * kBK;
+  static constexpr uint32_t kB = BN * kBK;
+  static constexpr uint32_t kRing = STAGES * (kA + kB);
+  static constexpr uint32_t kBars = (2 * STAGES + 5) * 8 + 16;
+  static constexpr uint32_t kTotal = kRing + kBars + 1024;  // + alignment slack
+  static constexpr uint32_t kTmemCols = 2 * BN;
+};
+
+template <OutKind KIND>
+__device__ __forceinline__ void store_chunk(const uint32_t (&r)[32], void *y, int64_t ldy, int row, int n0, int N,
+                                            float dx, const float *__restrict__ w_scale) {
+  // N % 16 == 0 and n0 % 32 == 0, so a chunk has 16 or 32 valid columns.
+  const int groups16 = min(2, (N - n0) / 16);
+  if constexpr (KIND == OutKind::I32) {
+    int32_t *yr = reinterpret_cast<int32_t *>(y) + (int64_t)row * ldy + n0;
+#pragma unroll
+    for (int g = 0; g < 8; ++g)
+      if (g / 4 < groups16)
+        reinterpret_cast<uint4 *>(yr)[g] = make_uint4(r[4 * g], r[4 * g + 1], r[4 * g + 2], r[4 * g + 3]);
+  } else {
+    float v[32];
+#pragma unroll
+    for (int g = 0; g < 8; ++g) {
+      if (g / 4 < groups16) {
+        const float4 dw = __ldg(reinterpret_cast<const float4 *>(w_scale + n0) + g);
+        v[4 * g + 0] = __fmul_rn(__fmul_rn(__int2float_rn((int)r[4 * g + 0]), dx), dw.x);
+        v[4 * g + 1] = __fmul_rn(__fmul_rn(__int2float_rn((int)r[4 * g + 1]), dx), dw.y);
+        v[4 * g + 2] = __fmul_rn(__fmul_rn(__int2float_rn((int)r[4 * g + 2]), dx), dw.z);
+        v[4 * g + 3] = __fmul_rn(__fmul_rn(__int2float_rn((int)r[4 * g + 3]), dx), dw.w);
+      } else {
+        v[4 * g + 0] = v[4 * g + 1] = v[4 * g + 2] = v[4 * g + 3] = 0.0f;
+      }
+    }
+    if constexpr (KIND == OutKind::F32) {
+      float *yr = reinterpret_cast<float *>(y) + (int64_t)row * ldy + n0;
+#pragma unroll
+      for (int g = 0; g < 8; ++g)
+        if (g / 4 < groups16)
+          reinterpret_cast<float4 *>(yr)[g] = make_float4(v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]);
+    } else {
+      uint32_t p[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        if constexpr (KIND == OutKind::BF16) {
+          __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+          p[i] = *reinterpret_cast<uint32_t *>(&h);
+        } else {
+          __half2 h = __floats2half2_rn(v[2 * i], v[2 * i + 1]);
+          p[i] = *reinterpret_cast<uint32_t *>(&h);
+        }
+      }
+      uint16_t *yr = reinterpret_cast<uint16_t *>(y) + (int64_t)row * ldy + n0;
+#pragma unroll
+      for (int g = 0; g < 4; ++g)
+        if (g / 2 < groups16)
+          reinterpret_cast<uint4 *>(yr)[g] = make_uint4(p[4 * g], p[4 * g + 1], p[4 * g + 2], p[4 * g + 3]);
+    }
+  }
+}
+
+template <int BN, int STAGES, OutKind KIND>
+__global__ void __launch_bounds__(kThreads, 1)
+    w8a8_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                        const float *__restrict__ x_scale, const float *__restrict__ w_scale, void *__restrict__ y,
+                        int64_t ldy, int M, int N, int K, unsigned *err) {
+  using L = GemmSmem<BN, STAGES>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t *sA = smem;
+  uint8_t *sB = smem + STAGES * L::kA;
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + L::kRing);
+  uint64_t *empty = full + STAGES;
+  uint64_t *tfull = empty + STAGES;
+  uint64_t *tempty = tfull + 2;
+  uint64_t *drain = tempty + 2;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int num_m = (M + kBM - 1) / kBM;
+  const int num_n = (N + BN - 1) / BN;
+  const int tiles = num_m * num_n;
+  const int nk = (K + kBK - 1) / kBK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 4);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, L::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- TMA producer ----------------
+      uint32_t stage = 0, phase = 0;
+      uint32_t armed = 0, armed_parity = 0;  // per-stage bit masks
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
+        const int mb = tile % num_m, nb = tile / num_m;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, err)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&full[stage], L::kA + L::kB);
+          tma_load_2d(&tmA, &full[stage], sA + stage * L::kA, kb * kBK, mb * kBM);
+          tma_load_2d(&tmB, &full[stage], sB + stage * L::kB, kb * kBK, nb * BN);
+          armed |= 1u << stage;
+          armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      if (!ok) {  // let every issued copy land before the CTA may exit
+        for (int s = 0; s < STAGES; ++s)
+          if (armed & (1u << s)) mbar_wait(&full[s], (armed_parity >> s) & 1u, nullptr, err);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------- MMA issuer ----------------
+      constexpr uint32_t idesc = idesc_i8(kBM, BN);
+      uint32_t stage = 0, phase = 0, ab = 0, aphase = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
+        if (!mbar_wait(&tempty[ab], aphase ^ 1, abort_flag, err)) break;
+        tc_fence_after();
+        const uint32_t d = tmem_base + ab * BN;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(&full[stage], phase, abort_flag, err)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t a0 = desc_sw128_kmajor(smem_u32(sA + stage * L::kA));
+          const uint64_t b0 = desc_sw128_kmajor(smem_u32(sB + stage * L::kB));
+#pragma unroll
+          for (int k = 0; k < kBK / 32; ++k)  // 32 int8 = 32 bytes = +2 in the >>4 address field
+            umma_i8(d, a0 + 2 * k, b0 + 2 * k, idesc, (kb | k) != 0 ? 1u : 0u);
+          umma_commit(&empty[stage]);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+        umma_commit(&tfull[ab]);
+        ab ^= 1;
+        if (ab == 0) aphase ^= 1;
+      }
+      // every MMA issued above must finish before TMEM is released
+      umma_commit(drain);
+      mbar_wait(drain, 0, nullptr, err);
+    }
+    __syncwarp();
+  } else {
+    // ---------------- epilogue (warps 2..5) ----------------
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    uint32_t ab = 0, aphase = 0;
+    for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
+      bool ok = mbar_wait(&tfull[ab], aphase, abort_flag, err);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after();
+      const int mb = tile % num_m, nb = tile / num_m;
+      const int row = mb * kBM + q * 32 + lane;
+      const bool row_ok = row < M;
+      const float dx = (KIND != OutKind::I32 && row_ok) ? __ldg(x_scale + row) : 0.0f;
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + ab * BN + c * 32, r);
+        tmem_ld_wait();
+        const int n0 = nb * BN + c * 32;
+        if (row_ok && n0 < N) store_chunk<KIND>(r, y, ldy, row, n0, N, dx, w_scale);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[ab]);
+      ab ^= 1;
+      if (ab == 0) aphase ^= 1;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, L::kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 2-D int8 tensor map over a [rows][cols] row-major matrix (row stride
+// `cols` bytes), box of box_rows x 128 bytes with 128-byte swizzling.
+bool make_tmap_i8(CUtensorMap *m, const int8_t *base, int64_t rows, int64_t cols, int box_rows) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)cols};
+  cuuint32_t box[2] = {(cuuint32_t)kBK, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<int8_t *>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int BN, int STAGES, OutKind KIND>
+cudaError_t launch_tc(const CUtensorMap &tmA, const CUtensorMap &tmB, const float *x_scale, const float *w_scale,
+                      void *y, int64_t ldy, int M, int N, int K, cudaStream_t st) {
+  using L = GemmSmem<BN, STAGES>;
+  auto kern = w8a8_gemm_tc_kernel<BN, STAGES, KIND>;
+  static bool attr_set[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::kTotal);
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  const int tiles = ((M + kBM - 1) / kBM) * ((N + BN - 1) / BN);
+  const int grid = tiles < num_sms() ? tiles : num_sms();
+  kern<<<grid, kThreads, L::kTotal, st>>>(tmA, tmB, x_scale, w_scale, y, ldy, M, N, K, device_error_word());
+  return cudaGetLastError();
+}
+
+template <OutKind KIND>
+cudaError_t gemm_dispatch(const int8_t *xq, const float *x_scale, const int8_t *wq, const float *w_scale, int M,
+                          int N, int K, void *y, int64_t ldy, cudaStream_t st) {
+  const int sms = num_sms();
+  const int tiles256 = ((M + kBM - 1) / kBM) * ((N + 255) / 256);
+  const bool wide = tiles256 >= sms || N % 256 == 0 && tiles256 * 2 > sms;
+  CUtensorMap tmA, tmB;
+  if (!make_tmap_i8(&tmA, xq, M, K, kBM)) return cudaErrorInvalidValue;
+  if (wide) {
+    if (!make_tmap_i8(&tmB, wq, N, K, 256)) return cudaErrorInvalidValue;
+    return launch_tc<256, 4, KIND>(tmA, tmB, x_scale, w_scale, y, ldy, M, N, K, st);
+  }
+  if (!make_tmap_i8(&tmB, wq, N, K, 128)) return cudaErrorInvalidValue;
+  return launch_tc<128, 6, KIND>(tmA, tmB, x_scale, w_scale, y, ldy, M, N, K, st);
+}
+
+}  // namespace
+
+size_t w8a8_workspace_bytes(int64_t, int64_t, int64_t) { return 0; }
+
+cudaError_t launch_w8a8_gemm(const int8_t *xq, const float *x_scale, const int8_t *wq, const float *w_scale,
+                             int64_t M, int64_t N, int64_t K, void *y, OutKind kind, int64_t ldy, void *, size_t,
+                             cudaStream_t st) {
+  switch (kind) {
+    case OutKind::F32: return gemm_dispatch<OutKind::F32>(xq, x_scale, wq, w_scale, (int)M, (int)N, (int)K, y, ldy, st);
+    case OutKind::F16: return gemm_dispatch<OutKind::F16>(xq, x_scale, wq, w_scale, (int)M, (int)N, (int)K, y, ldy, st);
+    case OutKind::BF16:
+      return gemm_dispatch<OutKind::BF16>(xq, x_scale, wq, w_scale, (int)M, (int)N, (int)K, y, ldy, st);
+    default: return gemm_dispatch<OutKind::I32>(xq, nullptr, wq, nullptr, (int)M, (int)N, (int)K, y, ldy, st);
+  }
+}
+
+}  // namespace sq

@@ -1,0 +1,41 @@
+// sq_internal.h -- launchers shared between the ABI shim and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "sq.h"
+
+namespace sq {
+
+// Number of SMs of the current device (cached per device).
+int num_sms();
+// Address of the current device's error word (cached per device).
+unsigned *device_error_word();
+
+// amax[c] = max(amax[c], max_r |x[r][c]| (* row_scale[r] when given)).
+cudaError_t launch_absmax_cols(const void *x, sq_dtype xt, int64_t rows, int64_t cols, int64_t ld,
+                               const float *row_scale, float *amax, cudaStream_t st);
+// out[r] = max_c |x[r][c]|.
+cudaError_t launch_absmax_rows(const void *x, sq_dtype xt, int64_t rows, int64_t cols, int64_t ld, float *out,
+                               cudaStream_t st);
+// s[j] (holding w_j on entry) <- s_j, inv_s[j] <- 1/s_j from amax[j], w_j.
+cudaError_t launch_smooth_factor(const float *amax, float *s_inout, float *inv_s, int64_t K, float alpha,
+                                 cudaStream_t st);
+// Row-wise: v = x[r][c] * col_scale[c]; per row absmax -> scale, codes.
+cudaError_t launch_quant_rows(const void *x, sq_dtype xt, int64_t rows, int64_t cols, int64_t ld,
+                              const float *col_scale, int8_t *q, float *row_scale_out, cudaStream_t st);
+// W[K][N] -> Wq[N][K] with v = s[j] * W[j][n] quantized per column n with
+// the column maxima colmax[n]; then colmax[n] <- colmax[n] / 127.
+cudaError_t launch_quant_cols_transpose(const void *w, sq_dtype wt, int64_t K, int64_t N, int64_t ld,
+                                        const float *s, float *colmax_to_scale, int8_t *wq, cudaStream_t st);
+
+// Output kinds of the tensor-core GEMM epilogue.
+enum class OutKind { F32, F16, BF16, I32 };
+cudaError_t launch_w8a8_gemm(const int8_t *xq, const float *x_scale, const int8_t *wq, const float *w_scale,
+                             int64_t M, int64_t N, int64_t K, void *y, OutKind kind, int64_t ldy, void *workspace,
+                             size_t workspace_bytes, cudaStream_t st);
+size_t w8a8_workspace_bytes(int64_t M, int64_t N, int64_t K);
+
+}  // namespace sq
