@@ -77,12 +77,12 @@ def traffic_for(kernel: str):
 # clocks sampled during the timed region
 # ---------------------------------------------------------------------------
 class ClockSampler:
-    FIELDS = ("uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    FIELDS = ("pci.bus_id,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, uuid: str | None):
-        self.uuid = (uuid or "").lower()
+    def __init__(self, bus_id: str | None):
+        self.bus_id = (bus_id or "").lower()
         self.rows = []
         self.proc = None
         self.thread = None
@@ -90,7 +90,7 @@ class ClockSampler:
     def start(self):
         try:
             self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                                          "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                                          "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except Exception:
             self.proc = None
             return
@@ -100,7 +100,7 @@ class ClockSampler:
     def _read(self):
         for line in self.proc.stdout:
             parts = [p.strip() for p in line.split(",")]
-            if len(parts) >= 9 and (not self.uuid or self.uuid in parts[0].lower()):
+            if len(parts) >= 9:
                 self.rows.append(parts)
 
     def stop(self):
@@ -114,6 +114,8 @@ class ClockSampler:
             self.thread.join(timeout=5)
 
     def summary(self):
+        mine = [r for r in self.rows if self.bus_id and r[0].lower().endswith(self.bus_id)]
+        self.rows = mine or self.rows
         if not self.rows:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no nvidia-smi samples"], "samples": 0}
 
@@ -208,8 +210,8 @@ def bench_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
 
     props = torch.cuda.get_device_properties(local_rank)
-    uuid = str(getattr(props, "uuid", "") or "")
-    clocks = ClockSampler(uuid)
+    bus = f"{props.pci_domain_id:04x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+    clocks = ClockSampler(bus)
     clocks.start()
     for _ in range(args.warmup):
         step(layers, sq, world)
@@ -230,7 +232,6 @@ def bench_ours(args, rank, world, local_rank):
     if world > 1:
         dist.barrier()
     ms_total = t0.elapsed_time(t1)
-    clocks.stop()
     if sq.sq_check_device_error() != sq.SQ_OK:
         raise RuntimeError("device-side timeout during the timed region")
     row_ms = {r: sum(a.elapsed_time(b) for a, b in v) / args.steps for r, v in ev.items()}
@@ -279,11 +280,12 @@ def bench_ours(args, rank, world, local_rank):
                       "parallelism": f"dp{world}",
                       "l2": "inputs larger than L2: each step streams 3.8 GB of calibration tokens and 0.4 GB of "
                             "weights per rank"},
-           "roofline": roof, "rows": rows, "gpu_launches": LAUNCHES_PER_LINEAR * nlin * args.steps,
-           "clocks": clocks.summary()}
+           "roofline": roof, "rows": rows, "gpu_launches": LAUNCHES_PER_LINEAR * nlin * args.steps}
 
     if not args.no_e2e:
         out["e2e"] = bench_e2e(args, layers, sq, world, work)
+    clocks.stop()
+    out["clocks"] = clocks.summary()
     if world > 1:
         dist.barrier()
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -434,7 +436,7 @@ def bench_reference(args, rank, world):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=300)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-e2e", action="store_true")

@@ -174,6 +174,34 @@ def test_accumulate_exact(M, N, K):
     no_device_error()
 
 
+# Shapes with >= 128 tiles of 256 x 256, which the library runs on CTA pairs
+# (tcgen05 cta_group::2): tails in M, N and K, including tiles whose second
+# CTA's half of Xq or Wq lies entirely past the matrix edge.
+PAIR_SHAPES = [(1000, 8464, 272), (2304, 4160, 144), (300, 16384, 256)]
+
+
+@pytest.mark.parametrize("M,N,K", PAIR_SHAPES)
+def test_accumulate_exact_cta_pairs(M, N, K):
+    xq = _rand_codes((M, K), M * 13 + K)
+    wq = _rand_codes((N, K), N * 7 + K)
+    acc = sq.sq_w8a8_accumulate(xq.to(DEV), wq.to(DEV))
+    np.testing.assert_array_equal(acc.cpu().numpy(), oracle.gemm_i8(xq.numpy(), wq.numpy()))
+    no_device_error()
+
+
+@pytest.mark.parametrize("dt", ["f32", "bf16"])
+def test_linear_epilogue_cta_pairs(dt):
+    M, N, K = 300, 16384, 256
+    xq = _rand_codes((M, K), 21)
+    wq = _rand_codes((N, K), 22)
+    xs = torch.rand(M, generator=synth.gen(23)) * 1e-2
+    ws = torch.rand(N, generator=synth.gen(24)) * 1e-2
+    y = sq.sq_w8a8_linear(xq.to(DEV), xs.to(DEV), wq.to(DEV), ws.to(DEV), TORCH_DT[dt])
+    y_ref = oracle_y(oracle.dequant(oracle.gemm_i8(xq.numpy(), wq.numpy()), xs.numpy(), ws.numpy()), dt)
+    assert_y(y, y_ref, dt)
+    no_device_error()
+
+
 def test_accumulate_int32_extremes():
     M, N, K = 130, 272, 28672  # 127*127*28672 is the largest sum these layers reach
     xq = torch.full((M, K), 127, dtype=torch.int8)

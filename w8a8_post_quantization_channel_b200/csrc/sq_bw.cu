@@ -129,67 +129,92 @@ __global__ void smooth_factor_kernel(const float *__restrict__ amax, float *__re
   inv_s[j] = __fdiv_rn(1.0f, s);
 }
 
-// Row quantizer, one CTA per row, the row held in registers:
+// Row quantizer (persistent): each CTA walks rows r = blockIdx.x,
+// blockIdx.x + gridDim.x, ...; per row
 //   v_c = x[r][c] * col_scale[c];  m = max_c |v_c|;
-//   row_scale_out[r] = m / 127;  q[r][c] = clamp(rne(v_c * (127 / m))).
-// Thread t owns the 16-byte vectors t, t + blockDim, ... (kVPT of them).
+//   row_scale_out[r] = m / 127;  q[r][c] = rne(v_c * (127 / m)).
+// Thread t owns the 16-byte vectors t + i*blockDim (i < kVPT) of every row:
+// their column scales stay in registers for the CTA's lifetime, the next
+// row's vectors are loaded before the current row is reduced, and the row
+// maximum needs one barrier (two alternating reduction slots).
+constexpr int kRowMaxThreads = 512;
 template <typename T, int kVPT>
-__global__ void __launch_bounds__(1024) quant_rows_kernel(const T *__restrict__ x, int64_t nvec, int64_t ld,
-                                                          const float *__restrict__ col_scale,
-                                                          int8_t *__restrict__ q, float *__restrict__ row_scale_out) {
+__global__ void __launch_bounds__(kRowMaxThreads)
+    quant_rows_kernel(const T *__restrict__ x, int64_t rows, int64_t nvec, int64_t ld,
+                      const float *__restrict__ col_scale, int8_t *__restrict__ q, float *__restrict__ row_scale_out) {
   constexpr int V = Vec<T>::N;
-  __shared__ float red[32];
-  const int64_t r = blockIdx.x;
-  const T *row = x + r * ld;
+  __shared__ float red[2][kRowMaxThreads / 32];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int nwarps = blockDim.x >> 5;
   const int64_t K = nvec * V;
-  uint4 raw[kVPT];
+
+  float sc[kVPT][V];
 #pragma unroll
   for (int i = 0; i < kVPT; ++i) {
-    const int64_t v = threadIdx.x + (int64_t)i * blockDim.x;
-    if (v < nvec) raw[i] = ld_stream_v4(row + v * V);
+    const int64_t v = tid + (int64_t)i * blockDim.x;
+#pragma unroll
+    for (int e = 0; e < V; ++e) sc[i][e] = v < nvec ? __ldg(col_scale + v * V + e) : 0.0f;
   }
-  float val[kVPT][V];
-  float m = 0.0f;
+  uint4 cur[kVPT], nxt[kVPT];
+  int64_t r = blockIdx.x;
 #pragma unroll
   for (int i = 0; i < kVPT; ++i) {
-    const int64_t v = threadIdx.x + (int64_t)i * blockDim.x;
-    if (v < nvec) {
-      float f[V];
-      Vec<T>::to_f32(raw[i], f);
-      const float4 *sc4 = reinterpret_cast<const float4 *>(col_scale + v * V);
+    const int64_t v = tid + (int64_t)i * blockDim.x;
+    cur[i] = (r < rows && v < nvec) ? ld_stream_v4(x + r * ld + v * V) : make_uint4(0, 0, 0, 0);
+  }
+  int slot = 0;
+  for (; r < rows; r += gridDim.x) {
+    const int64_t rn = r + gridDim.x;
 #pragma unroll
-      for (int e4 = 0; e4 < V / 4; ++e4) {
-        const float4 s = __ldg(sc4 + e4);
-        val[i][4 * e4 + 0] = __fmul_rn(f[4 * e4 + 0], s.x);
-        val[i][4 * e4 + 1] = __fmul_rn(f[4 * e4 + 1], s.y);
-        val[i][4 * e4 + 2] = __fmul_rn(f[4 * e4 + 2], s.z);
-        val[i][4 * e4 + 3] = __fmul_rn(f[4 * e4 + 3], s.w);
+    for (int i = 0; i < kVPT; ++i) {
+      const int64_t v = tid + (int64_t)i * blockDim.x;
+      nxt[i] = (rn < rows && v < nvec) ? ld_stream_v4(x + rn * ld + v * V) : make_uint4(0, 0, 0, 0);
+    }
+    float val[kVPT][V];
+    float m = 0.0f;
+#pragma unroll
+    for (int i = 0; i < kVPT; ++i) {
+      float f[V];
+      Vec<T>::to_f32(cur[i], f);
+#pragma unroll
+      for (int e = 0; e < V; e += 2) {
+        const float2 p = fmul2_rn(make_float2(f[e], f[e + 1]), make_float2(sc[i][e], sc[i][e + 1]));
+        val[i][e] = p.x;
+        val[i][e + 1] = p.y;
       }
 #pragma unroll
       for (int e = 0; e < V; ++e) m = fmaxf(m, fabsf(val[i][e]));
     }
-  }
-  m = block_max(m, red);
-  const bool zero = (m == 0.0f);
-  const float rcp = zero ? 0.0f : __fdiv_rn(127.0f, m);
-  if (threadIdx.x == 0) row_scale_out[r] = zero ? 0.0f : __fdiv_rn(m, 127.0f);
-  int8_t *qrow = q + r * K;
+    m = warp_max(m);
+    if (lane == 0) red[slot][warp] = m;
+    __syncthreads();
+    m = 0.0f;
+    for (int w = 0; w < nwarps; ++w) m = fmaxf(m, red[slot][w]);
+    slot ^= 1;
+    // m == 0 (all-zero row): rcp = 0 gives codes 0 and scale 0
+    const float rcp = m > 0.0f ? __fdiv_rn(127.0f, m) : 0.0f;
+    if (tid == 0) row_scale_out[r] = __fdiv_rn(m, 127.0f);
+    int8_t *qrow = q + r * K;
 #pragma unroll
-  for (int i = 0; i < kVPT; ++i) {
-    const int64_t v = threadIdx.x + (int64_t)i * blockDim.x;
-    if (v < nvec) {
-      int c[V];
-#pragma unroll
-      for (int e = 0; e < V; ++e) c[e] = zero ? 0 : quantize(val[i][e], rcp);
-      if constexpr (V == 8) {
-        uint2 o;
-        o.x = pack4_i8(c[0], c[1], c[2], c[3]);
-        o.y = pack4_i8(c[4], c[5], c[6], c[7]);
-        *reinterpret_cast<uint2 *>(qrow + v * V) = o;
-      } else {
-        *reinterpret_cast<uint32_t *>(qrow + v * V) = pack4_i8(c[0], c[1], c[2], c[3]);
+    for (int i = 0; i < kVPT; ++i) {
+      const int64_t v = tid + (int64_t)i * blockDim.x;
+      if (v < nvec) {
+        if constexpr (V == 8) {
+          uint2 o;
+          o.x = pack4_codes(quantize_dynamic(val[i][0], rcp), quantize_dynamic(val[i][1], rcp),
+                            quantize_dynamic(val[i][2], rcp), quantize_dynamic(val[i][3], rcp));
+          o.y = pack4_codes(quantize_dynamic(val[i][4], rcp), quantize_dynamic(val[i][5], rcp),
+                            quantize_dynamic(val[i][6], rcp), quantize_dynamic(val[i][7], rcp));
+          *reinterpret_cast<uint2 *>(qrow + v * V) = o;
+        } else {
+          *reinterpret_cast<uint32_t *>(qrow + v * V) =
+              pack4_codes(quantize_dynamic(val[i][0], rcp), quantize_dynamic(val[i][1], rcp),
+                          quantize_dynamic(val[i][2], rcp), quantize_dynamic(val[i][3], rcp));
+        }
       }
     }
+#pragma unroll
+    for (int i = 0; i < kVPT; ++i) cur[i] = nxt[i];
   }
 }
 
@@ -213,23 +238,22 @@ __global__ void __launch_bounds__(1024) quant_rows_twopass_kernel(const T *__res
     for (int e = 0; e < V; ++e) m = fmaxf(m, fabsf(__fmul_rn(f[e], __ldg(col_scale + v * V + e))));
   }
   m = block_max(m, red);
-  const bool zero = (m == 0.0f);
-  const float rcp = zero ? 0.0f : __fdiv_rn(127.0f, m);
-  if (threadIdx.x == 0) row_scale_out[r] = zero ? 0.0f : __fdiv_rn(m, 127.0f);
+  const float rcp = m > 0.0f ? __fdiv_rn(127.0f, m) : 0.0f;
+  if (threadIdx.x == 0) row_scale_out[r] = __fdiv_rn(m, 127.0f);
   int8_t *qrow = q + r * K;
   for (int64_t v = threadIdx.x; v < nvec; v += blockDim.x) {
     float f[V];
     Vec<T>::to_f32(ld_stream_v4(row + v * V), f);
     int c[V];
 #pragma unroll
-    for (int e = 0; e < V; ++e) c[e] = zero ? 0 : quantize(__fmul_rn(f[e], __ldg(col_scale + v * V + e)), rcp);
+    for (int e = 0; e < V; ++e) c[e] = quantize_dynamic(__fmul_rn(f[e], __ldg(col_scale + v * V + e)), rcp);
     if constexpr (V == 8) {
       uint2 o;
-      o.x = pack4_i8(c[0], c[1], c[2], c[3]);
-      o.y = pack4_i8(c[4], c[5], c[6], c[7]);
+      o.x = pack4_codes(c[0], c[1], c[2], c[3]);
+      o.y = pack4_codes(c[4], c[5], c[6], c[7]);
       *reinterpret_cast<uint2 *>(qrow + v * V) = o;
     } else {
-      *reinterpret_cast<uint32_t *>(qrow + v * V) = pack4_i8(c[0], c[1], c[2], c[3]);
+      *reinterpret_cast<uint32_t *>(qrow + v * V) = pack4_codes(c[0], c[1], c[2], c[3]);
     }
   }
 }
@@ -244,8 +268,15 @@ __global__ void __launch_bounds__(256) quant_cols_transpose_kernel(const T *__re
                                                                    const float *__restrict__ colmax,
                                                                    int8_t *__restrict__ wq) {
   __shared__ int8_t tile[kTT][kTT + 4];  // [n][j]
+  __shared__ float rcp[kTT];
   const int64_t j0 = (int64_t)blockIdx.y * kTT, n0 = (int64_t)blockIdx.x * kTT;
   const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;  // 16 x 16 threads
+  if (threadIdx.x < kTT) {
+    const int64_t n = n0 + threadIdx.x;
+    const float cm = n < N ? __ldg(colmax + n) : 0.0f;
+    rcp[threadIdx.x] = cm > 0.0f ? __fdiv_rn(127.0f, cm) : 0.0f;
+  }
+  __syncthreads();
   // each thread: 4 consecutive n of one j row, rows ty, ty+16, ...
 #pragma unroll
   for (int jj = ty; jj < kTT; jj += 16) {
@@ -256,11 +287,7 @@ __global__ void __launch_bounds__(256) quant_cols_transpose_kernel(const T *__re
       const float sj = __ldg(s + j);
       const T *p = w + j * ld + n;
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float cm = __ldg(colmax + n + e);
-        const float wv = Vec<T>::one(p + e);
-        c[e] = (cm == 0.0f) ? 0 : quantize(__fmul_rn(sj, wv), __fdiv_rn(127.0f, cm));
-      }
+      for (int e = 0; e < 4; ++e) c[e] = quantize(__fmul_rn(sj, Vec<T>::one(p + e)), rcp[tx * 4 + e]);
     }
 #pragma unroll
     for (int e = 0; e < 4; ++e) tile[tx * 4 + e][jj] = (int8_t)c[e];
@@ -309,29 +336,41 @@ cudaError_t absmax_rows_t(const void *x, int64_t rows, int64_t cols, int64_t ld,
   return cudaGetLastError();
 }
 
+template <typename T, int kVPT>
+cudaError_t launch_quant_rows_persistent(const T *x, int64_t rows, int64_t nvec, int64_t ld, const float *col_scale,
+                                         int8_t *q, float *row_scale_out, int threads, cudaStream_t st) {
+  static int per_sm[64][5] = {};  // [device][threads / 128]
+  int dev = 0;
+  cudaGetDevice(&dev);
+  int &cached = per_sm[dev & 63][(threads - 1) / 128];
+  if (cached == 0) {
+    int n = 0;
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, quant_rows_kernel<T, kVPT>, threads, 0);
+    if (e != cudaSuccess) return e;
+    cached = n > 0 ? n : 1;
+  }
+  const int64_t grid = std::min<int64_t>(rows, (int64_t)cached * num_sms());
+  quant_rows_kernel<T, kVPT><<<(unsigned)grid, threads, 0, st>>>(x, rows, nvec, ld, col_scale, q, row_scale_out);
+  return cudaGetLastError();
+}
+
 template <typename T>
 cudaError_t quant_rows_t(const void *x, int64_t rows, int64_t cols, int64_t ld, const float *col_scale, int8_t *q,
                          float *row_scale_out, cudaStream_t st) {
   constexpr int V = Vec<T>::N;
   const int64_t nvec = cols / V;
+  const T *xp = (const T *)x;
   auto threads_for = [&](int vpt) {
     int64_t t = (nvec + vpt - 1) / vpt;
-    t = ((t + 31) / 32) * 32;
-    return (int)std::max<int64_t>(32, t);
+    return (int)std::max<int64_t>(32, ((t + 31) / 32) * 32);
   };
-  const T *xp = (const T *)x;
-  const unsigned g = (unsigned)rows;
-  if (threads_for(1) <= 256) {
-    quant_rows_kernel<T, 1><<<g, threads_for(1), 0, st>>>(xp, nvec, ld, col_scale, q, row_scale_out);
-  } else if (threads_for(2) <= 512) {
-    quant_rows_kernel<T, 2><<<g, threads_for(2), 0, st>>>(xp, nvec, ld, col_scale, q, row_scale_out);
-  } else if (threads_for(4) <= 512) {
-    quant_rows_kernel<T, 4><<<g, threads_for(4), 0, st>>>(xp, nvec, ld, col_scale, q, row_scale_out);
-  } else if (threads_for(4) <= 1024) {
-    quant_rows_kernel<T, 4><<<g, threads_for(4), 0, st>>>(xp, nvec, ld, col_scale, q, row_scale_out);
-  } else {
-    quant_rows_twopass_kernel<T><<<g, 1024, 0, st>>>(xp, nvec, ld, col_scale, q, row_scale_out);
+  if (nvec <= 4 * 32) {
+    return launch_quant_rows_persistent<T, 1>(xp, rows, nvec, ld, col_scale, q, row_scale_out, threads_for(1), st);
   }
+  if (nvec <= 4 * kRowMaxThreads) {
+    return launch_quant_rows_persistent<T, 4>(xp, rows, nvec, ld, col_scale, q, row_scale_out, threads_for(4), st);
+  }
+  quant_rows_twopass_kernel<T><<<(unsigned)rows, 1024, 0, st>>>(xp, nvec, ld, col_scale, q, row_scale_out);
   return cudaGetLastError();
 }
 

@@ -248,6 +248,194 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ---------------------------------------------------------------------------
+// CTA-pair kernel: a cluster of two CTAs computes a 256 x 256 tile with
+// tcgen05.mma.cta_group::2 (M = 256, N = 256, K = 32 per instruction).
+// CTA r of the pair loads rows [128 r, 128 r + 128) of the tile's Xq block
+// and of its Wq block into its own shared memory; both loads count bytes on
+// the leader CTA's (rank 0) full barrier.  The leader's single MMA thread
+// drives the pair; its commits arrive on the matching barriers of both
+// CTAs.  Each CTA's epilogue reads its own TMEM: 128 rows x 256 columns.
+// Per CTA and k-block this moves 32 KB for 128 x 256 x 128 MACs, a third
+// less operand traffic than the single-CTA 128 x 256 tile.
+// ---------------------------------------------------------------------------
+constexpr int kPairBN = 256;
+
+template <int STAGES>
+struct PairSmem {
+  static constexpr uint32_t kA = kBM * kBK;           // 16 KB: this CTA's 128 rows of Xq
+  static constexpr uint32_t kB = (kPairBN / 2) * kBK;  // 16 KB: this CTA's 128 rows of Wq
+  static constexpr uint32_t kRing = STAGES * (kA + kB);
+  static constexpr uint32_t kBars = (2 * STAGES + 5) * 8 + 16;
+  static constexpr uint32_t kTotal = kRing + kBars + 1024;
+  static constexpr uint32_t kTmemCols = 2 * kPairBN;  // two 256-column accumulators
+};
+
+template <int STAGES, OutKind KIND>
+__global__ void __launch_bounds__(kThreads, 1)
+    w8a8_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                          const float *__restrict__ x_scale, const float *__restrict__ w_scale,
+                          void *__restrict__ y, int64_t ldy, int M, int N, int K, unsigned *err) {
+  using L = PairSmem<STAGES>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t *sA = smem;
+  uint8_t *sB = smem + STAGES * L::kA;
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + L::kRing);
+  uint64_t *empty = full + STAGES;
+  uint64_t *tfull = empty + STAGES;
+  uint64_t *tempty = tfull + 2;
+  uint64_t *drain = tempty + 2;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const uint32_t peer = rank ^ 1u;
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  const int num_m = (M + 2 * kBM - 1) / (2 * kBM);
+  const int num_n = (N + kPairBN - 1) / kPairBN;
+  const int tiles = num_m * num_n;
+  const int nk = (K + kBK - 1) / kBK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 8);  // 4 epilogue warps in each CTA of the pair
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, L::kTmemCols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync();  // barriers of both CTAs initialised, TMEM allocated
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- TMA producer (both CTAs) ----------------
+      uint32_t stage = 0, phase = 0;
+      uint32_t armed = 0, armed_parity = 0;
+      bool ok = true;
+      for (int tile = pair; tile < tiles && ok; tile += npairs) {
+        const int mb = tile % num_m, nb = tile / num_m;
+        const int row_a = mb * 2 * kBM + (int)rank * kBM;
+        const int row_b = nb * kPairBN + (int)rank * (kPairBN / 2);
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, err)) {
+            ok = false;
+            break;
+          }
+          if (leader) {
+            mbar_arrive_expect_tx(&full[stage], 2 * (L::kA + L::kB));
+            armed |= 1u << stage;
+            armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
+          }
+          const uint32_t bar = mapa_shared(smem_u32(&full[stage]), 0);
+          tma_load_2d_pair(&tmA, bar, sA + stage * L::kA, kb * kBK, row_a);
+          tma_load_2d_pair(&tmB, bar, sB + stage * L::kB, kb * kBK, row_b);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      if (!ok && leader) {  // the leader's barriers count both CTAs' copies
+        for (int s = 0; s < STAGES; ++s)
+          if (armed & (1u << s)) mbar_wait(&full[s], (armed_parity >> s) & 1u, nullptr, err);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && leader) {
+      // ---------------- MMA issuer (leader CTA) ----------------
+      constexpr uint32_t idesc = idesc_i8(2 * kBM, kPairBN);
+      uint32_t stage = 0, phase = 0, ab = 0, aphase = 0;
+      bool ok = true;
+      for (int tile = pair; tile < tiles && ok; tile += npairs) {
+        if (!mbar_wait(&tempty[ab], aphase ^ 1, abort_flag, err)) break;
+        tc_fence_after();
+        const uint32_t d = tmem_base + ab * kPairBN;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(&full[stage], phase, abort_flag, err)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t a0 = desc_sw128_kmajor(smem_u32(sA + stage * L::kA));
+          const uint64_t b0 = desc_sw128_kmajor(smem_u32(sB + stage * L::kB));
+#pragma unroll
+          for (int k = 0; k < kBK / 32; ++k) umma_i8_pair(d, a0 + 2 * k, b0 + 2 * k, idesc, (kb | k) != 0 ? 1u : 0u);
+          const uint32_t e = smem_u32(&empty[stage]);
+          umma_commit_pair(mapa_shared(e, 0));
+          umma_commit_pair(mapa_shared(e, 1));
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+        const uint32_t t = smem_u32(&tfull[ab]);
+        umma_commit_pair(mapa_shared(t, 0));
+        umma_commit_pair(mapa_shared(t, 1));
+        ab ^= 1;
+        if (ab == 0) aphase ^= 1;
+      }
+      umma_commit_pair(mapa_shared(smem_u32(drain), 0));
+      mbar_wait(drain, 0, nullptr, err);
+    }
+    __syncwarp();
+  } else {
+    // ---------------- epilogue (warps 2..5 of both CTAs) ----------------
+    const int q = warp & 3;
+    const uint32_t tempty_leader = mapa_shared(smem_u32(&tempty[0]), 0);
+    uint32_t ab = 0, aphase = 0;
+    for (int tile = pair; tile < tiles; tile += npairs) {
+      bool ok = mbar_wait(&tfull[ab], aphase, abort_flag, err);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after();
+      const int mb = tile % num_m, nb = tile / num_m;
+      const int row = mb * 2 * kBM + (int)rank * kBM + q * 32 + lane;
+      const bool row_ok = row < M;
+      const float dx = (KIND != OutKind::I32 && row_ok) ? __ldg(x_scale + row) : 0.0f;
+#pragma unroll 1
+      for (int c = 0; c < kPairBN / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + ab * kPairBN + c * 32, r);
+        tmem_ld_wait();
+        const int n0 = nb * kPairBN + c * 32;
+        if (row_ok && n0 < N) store_chunk<KIND>(r, y, ldy, row, n0, N, dx, w_scale);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(tempty_leader + ab * 8);
+      ab ^= 1;
+      if (ab == 0) aphase ^= 1;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // the peer's shared memory and TMEM stay live until the leader is done
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, L::kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -297,13 +485,77 @@ cudaError_t launch_tc(const CUtensorMap &tmA, const CUtensorMap &tmB, const floa
   return cudaGetLastError();
 }
 
+template <int STAGES, OutKind KIND>
+cudaError_t launch_pair(const CUtensorMap &tmA, const CUtensorMap &tmB, const float *x_scale, const float *w_scale,
+                        void *y, int64_t ldy, int M, int N, int K, int max_clusters, cudaStream_t st) {
+  using L = PairSmem<STAGES>;
+  auto kern = w8a8_gemm_pair_kernel<STAGES, KIND>;
+  const int tiles = ((M + 2 * kBM - 1) / (2 * kBM)) * ((N + kPairBN - 1) / kPairBN);
+  const int clusters = tiles < max_clusters ? tiles : max_clusters;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * clusters, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = L::kTotal;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tmA, tmB, x_scale, w_scale, y, ldy, M, N, K, device_error_word());
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+// Clusters of two 1-CTA-per-SM blocks that fit on the device at once.
+template <int STAGES, OutKind KIND>
+int pair_capacity() {
+  using L = PairSmem<STAGES>;
+  static int cache[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  int &c = cache[dev & 63];
+  if (c == 0) {
+    auto kern = w8a8_gemm_pair_kernel<STAGES, KIND>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::kTotal) != cudaSuccess)
+      return -1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2, 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = L::kTotal;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) return -1;
+    c = n;
+  }
+  return c;
+}
+
+constexpr int kPairStages = 6;
+
 template <OutKind KIND>
 cudaError_t gemm_dispatch(const int8_t *xq, const float *x_scale, const int8_t *wq, const float *w_scale, int M,
                           int N, int K, void *y, int64_t ldy, cudaStream_t st) {
   const int sms = num_sms();
-  const int tiles256 = ((M + kBM - 1) / kBM) * ((N + 255) / 256);
-  const bool wide = tiles256 >= sms || N % 256 == 0 && tiles256 * 2 > sms;
   CUtensorMap tmA, tmB;
+  // CTA pairs once there are enough 256 x 256 tiles to occupy every pair
+  const int tiles_pair = ((M + 255) / 256) * ((N + 255) / 256);
+  const int cap = pair_capacity<kPairStages, KIND>();
+  if (cap > 0 && tiles_pair >= cap) {
+    if (!make_tmap_i8(&tmA, xq, M, K, kBM)) return cudaErrorInvalidValue;
+    if (!make_tmap_i8(&tmB, wq, N, K, kPairBN / 2)) return cudaErrorInvalidValue;
+    return launch_pair<kPairStages, KIND>(tmA, tmB, x_scale, w_scale, y, ldy, M, N, K, cap, st);
+  }
+  const int tiles256 = ((M + kBM - 1) / kBM) * ((N + 255) / 256);
+  const bool wide = tiles256 >= sms || (N % 256 == 0 && tiles256 * 2 > sms);
   if (!make_tmap_i8(&tmA, xq, M, K, kBM)) return cudaErrorInvalidValue;
   if (wide) {
     if (!make_tmap_i8(&tmB, wq, N, K, 256)) return cudaErrorInvalidValue;
