@@ -109,7 +109,20 @@ def test_linear_argument_checks():
 def test_workspace_size_is_defined_for_all_shapes():
     for M in (0, 1, 8, 64, 128, 2048):
         for N, K in ((256, 256), (4096, 4096), (28672, 8192)):
-            assert sq.sq_w8a8_linear_workspace_size(M, N, K) >= 0
+            need = sq.sq_w8a8_linear_workspace_size(M, N, K)
+            if 1 <= M <= 64:   # decode-shaped: int32 partial sums + tile counters
+                assert need >= M * N * 4 + 4 * ((N + 127) // 128)
+                assert need % 256 == 0
+            else:
+                assert need == 0
+
+
+def test_linear_requires_workspace_when_needed():
+    f = sq.lib().sq_w8a8_linear
+    need = sq.sq_w8a8_linear_workspace_size(8, 256, 256)
+    assert f(A16, A16, A16, A16, 8, 256, 256, A16, sq.SQ_BF16, 256, None, 0, None) == INV
+    assert f(A16, A16, A16, A16, 8, 256, 256, A16, sq.SQ_BF16, 256, A16, need - 1, None) == INV
+    assert f(A16, A16, A16, A16, 8, 256, 256, A16, sq.SQ_BF16, 256, MIS, need, None) == INV
 
 
 def test_binding_rejects_host_tensors():

@@ -202,6 +202,34 @@ def test_linear_epilogue_cta_pairs(dt):
     no_device_error()
 
 
+# Decode-shaped products (M <= 64 tokens): the weight-streaming kernel,
+# whose CTAs combine partial tiles through the caller's workspace.
+DECODE_SHAPES = [(1, 4096, 4096), (2, 272, 1040), (16, 1024, 8192), (17, 4096, 272), (33, 528, 4096),
+                 (48, 16, 16), (64, 12288, 1040), (64, 1040, 11008), (8, 28672, 8192), (1, 8192, 8192)]
+
+
+@pytest.mark.parametrize("M,N,K", DECODE_SHAPES)
+def test_decode_shapes_exact_and_workspace_clean(M, N, K):
+    xq = _rand_codes((M, K), M * 3 + K)
+    wq = _rand_codes((N, K), N * 5 + K)
+    xs = torch.rand(M, generator=synth.gen(M + 1)) * 1e-2
+    ws = torch.rand(N, generator=synth.gen(N + 1)) * 1e-2
+    need = sq.sq_w8a8_linear_workspace_size(M, N, K)
+    assert need >= M * N * 4
+    work = torch.zeros(need, dtype=torch.uint8, device=DEV)
+    acc_ref = oracle.gemm_i8(xq.numpy(), wq.numpy())
+    xq_d, wq_d = xq.to(DEV), wq.to(DEV)
+    for _ in range(2):  # two calls in a row on one workspace
+        acc = sq.sq_w8a8_accumulate(xq_d, wq_d, workspace=work)
+        np.testing.assert_array_equal(acc.cpu().numpy(), acc_ref)
+        assert int(work.count_nonzero()) == 0  # left zero for the next call
+    y_ref = oracle_y(oracle.dequant(acc_ref, xs.numpy(), ws.numpy()), "bf16")
+    y = sq.sq_w8a8_linear(xq_d, xs.to(DEV), wq_d, ws.to(DEV), torch.bfloat16, workspace=work)
+    assert_y(y, y_ref, "bf16")
+    assert int(work.count_nonzero()) == 0
+    no_device_error()
+
+
 def test_accumulate_int32_extremes():
     M, N, K = 130, 272, 28672  # 127*127*28672 is the largest sum these layers reach
     xq = torch.full((M, K), 127, dtype=torch.int8)

@@ -32,6 +32,12 @@ namespace {
 constexpr int kBM = 128;  // rows of Xq per tile (= TMEM lanes)
 constexpr int kBK = 128;  // K bytes per stage (one 128-byte swizzle row)
 constexpr int kThreads = 192;
+constexpr int kDecodeMaxM = 64;  // token counts served by the weight-streaming kernel
+
+// Workspace of the decode kernel: int32 partial sums [M][N], then one
+// arrival counter per 128-row tile of Wq (each region 256-byte aligned).
+inline int64_t decode_ws_elems(int64_t M, int64_t N) { return ((M * N * 4 + 255) / 256) * 64; }
+inline int64_t decode_counter_bytes(int64_t N) { return (((N + 127) / 128) * 4 + 255) / 256 * 256; }
 
 template <int BN, int STAGES>
 struct GemmSmem {
@@ -436,6 +442,243 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ---------------------------------------------------------------------------
+// Decode-shaped linear (M <= 64 tokens): bound by streaming Wq from HBM.
+// The roles of the operands swap: 128 rows of Wq sit on the MMA's M side
+// and the (padded) MP tokens on its N side, so D^T[n][t] accumulates in
+// TMEM lanes n, columns t.  The N/128 x K/128 (tile, k-block) items are
+// split evenly over the CTAs (each streams the same number of Wq bytes);
+// a CTA's share may cover parts of two tiles.  A CTA that covers a whole
+// tile dequantizes it straight from TMEM.  Otherwise it adds its int32
+// partial sums into the workspace (exact, order-free), counts the k-blocks
+// it contributed on the tile's counter, and the CTA whose count completes
+// the tile dequantizes it from the workspace and leaves the workspace and
+// the counter zero again.  No CTA waits for another.
+// ---------------------------------------------------------------------------
+constexpr int kDecRows = 128;  // Wq rows per tile (MMA M)
+constexpr int kDecStages = 8;
+
+template <int MP>
+struct DecSmem {
+  static constexpr uint32_t kW = kDecRows * kBK;  // 16 KB of Wq per stage
+  static constexpr uint32_t kX = MP * kBK;        // MP token rows of Xq per stage
+  static constexpr uint32_t kStage = kW + kX;
+  static constexpr uint32_t kRing = kDecStages * kStage;
+  static constexpr uint32_t kBars = (2 * kDecStages + 5) * 8 + 32;
+  static constexpr uint32_t kTotal = kRing + kBars + 1024;
+  static constexpr uint32_t kTmemCols = (2 * MP <= 32) ? 32 : (2 * MP <= 64) ? 64 : 128;
+};
+
+template <OutKind KIND>
+__device__ __forceinline__ void store_one(void *y, int64_t ldy, int t, int n, int32_t acc, float dx, float dw) {
+  if constexpr (KIND == OutKind::I32) {
+    reinterpret_cast<int32_t *>(y)[(int64_t)t * ldy + n] = acc;
+  } else {
+    const float v = __fmul_rn(__fmul_rn(__int2float_rn(acc), dx), dw);
+    if constexpr (KIND == OutKind::F32) {
+      reinterpret_cast<float *>(y)[(int64_t)t * ldy + n] = v;
+    } else if constexpr (KIND == OutKind::BF16) {
+      reinterpret_cast<__nv_bfloat16 *>(y)[(int64_t)t * ldy + n] = __float2bfloat16_rn(v);
+    } else {
+      reinterpret_cast<__half *>(y)[(int64_t)t * ldy + n] = __float2half_rn(v);
+    }
+  }
+}
+
+template <int MP, OutKind KIND>
+__global__ void __launch_bounds__(kThreads, 1)
+    w8a8_gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
+                            const float *__restrict__ x_scale, const float *__restrict__ w_scale,
+                            void *__restrict__ y, int64_t ldy, int M, int N, int K, int32_t *__restrict__ ws,
+                            unsigned *__restrict__ tile_count, unsigned *err) {
+  using L = DecSmem<MP>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + L::kRing);
+  uint64_t *empty = full + kDecStages;
+  uint64_t *tfull = empty + kDecStages;
+  uint64_t *tempty = tfull + 2;
+  uint64_t *drain = tempty + 2;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+  volatile int *last_flag = reinterpret_cast<volatile int *>(tmem_slot + 2);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int ntiles = (N + kDecRows - 1) / kDecRows;
+  const int nk = (K + kBK - 1) / kBK;
+  const int64_t items = (int64_t)ntiles * nk;
+  const int64_t w0 = items * blockIdx.x / gridDim.x;
+  const int64_t w1 = items * (blockIdx.x + 1) / gridDim.x;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kDecStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 4);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmW);
+    prefetch_tmap(&tmX);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, L::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- TMA producer ----------------
+      uint32_t stage = 0, phase = 0, armed = 0, armed_parity = 0;
+      bool ok = true;
+      for (int64_t w = w0; w < w1 && ok; ++w) {
+        const int tile = (int)(w / nk), kb = (int)(w % nk);
+        if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, err)) {
+          ok = false;
+          break;
+        }
+        uint8_t *st = smem + stage * L::kStage;
+        mbar_arrive_expect_tx(&full[stage], L::kStage);
+        tma_load_2d(&tmW, &full[stage], st, kb * kBK, tile * kDecRows);
+        tma_load_2d(&tmX, &full[stage], st + L::kW, kb * kBK, 0);
+        armed |= 1u << stage;
+        armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
+        if (++stage == kDecStages) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+      if (!ok) {
+        for (int s = 0; s < kDecStages; ++s)
+          if (armed & (1u << s)) mbar_wait(&full[s], (armed_parity >> s) & 1u, nullptr, err);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------- MMA issuer: one accumulation per segment ----------------
+      constexpr uint32_t idesc = idesc_i8(kDecRows, MP);
+      uint32_t stage = 0, phase = 0, ab = 0, aphase = 0;
+      bool ok = true;
+      for (int64_t w = w0; w < w1 && ok;) {
+        const int tile = (int)(w / nk);
+        const int64_t seg_end = w1 < (int64_t)(tile + 1) * nk ? w1 : (int64_t)(tile + 1) * nk;
+        if (!mbar_wait(&tempty[ab], aphase ^ 1, abort_flag, err)) break;
+        tc_fence_after();
+        const uint32_t d = tmem_base + ab * MP;
+        for (int64_t i = w; i < seg_end; ++i) {
+          if (!mbar_wait(&full[stage], phase, abort_flag, err)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          uint8_t *st = smem + stage * L::kStage;
+          const uint64_t a0 = desc_sw128_kmajor(smem_u32(st));
+          const uint64_t b0 = desc_sw128_kmajor(smem_u32(st + L::kW));
+#pragma unroll
+          for (int k = 0; k < kBK / 32; ++k)
+            umma_i8(d, a0 + 2 * k, b0 + 2 * k, idesc, (i != w || k != 0) ? 1u : 0u);
+          umma_commit(&empty[stage]);
+          if (++stage == kDecStages) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+        umma_commit(&tfull[ab]);
+        ab ^= 1;
+        if (ab == 0) aphase ^= 1;
+        w = seg_end;
+      }
+      umma_commit(drain);
+      mbar_wait(drain, 0, nullptr, err);
+    }
+    __syncwarp();
+  } else {
+    // ---------------- epilogue (warps 2..5: 128 threads, one Wq row each) ----------------
+    const int q = warp & 3;
+    const int et = threadIdx.x - 64;  // 0..127
+    uint32_t ab = 0, aphase = 0;
+    for (int64_t w = w0; w < w1;) {
+      const int tile = (int)(w / nk);
+      const int64_t seg_end = w1 < (int64_t)(tile + 1) * nk ? w1 : (int64_t)(tile + 1) * nk;
+      const int seg_len = (int)(seg_end - w);
+      // one decision for all four warps: they share named barriers below
+      const bool ok = mbar_wait(&tfull[ab], aphase, abort_flag, err);
+      if (!named_barrier_and(1, 128, ok)) break;
+      tc_fence_after();
+      const int n = tile * kDecRows + q * 32 + lane;
+      const bool n_ok = n < N;
+      const float dw = (KIND != OutKind::I32 && n_ok) ? __ldg(w_scale + n) : 0.0f;
+      const bool whole = seg_len == nk;
+#pragma unroll
+      for (int c = 0; c < MP / 16; ++c) {
+        uint32_t r[16];
+        tmem_ld16(tmem_base + ((uint32_t)(q * 32) << 16) + ab * MP + c * 16, r);
+        tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const int t = c * 16 + j;
+          if (t < M && n_ok) {
+            if (whole) {
+              const float dx = KIND != OutKind::I32 ? __ldg(x_scale + t) : 0.0f;
+              store_one<KIND>(y, ldy, t, n, (int32_t)r[j], dx, dw);
+            } else if (r[j] != 0u) {
+              atomicAdd(ws + (int64_t)t * N + n, (int32_t)r[j]);
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[ab]);
+      if (!whole) {
+        // publish this CTA's partial sums, then count its k-blocks
+        __threadfence();
+        named_barrier(1, 128);
+        if (et == 0) {
+          const unsigned before = atomicAdd(tile_count + tile, (unsigned)seg_len);
+          *last_flag = (before + (unsigned)seg_len == (unsigned)nk) ? 1 : 0;
+        }
+        named_barrier(1, 128);
+        if (*last_flag) {
+          __threadfence();
+          if (n_ok) {
+            for (int t = 0; t < M; ++t) {
+              int32_t *p = ws + (int64_t)t * N + n;
+              const int32_t acc = __ldcg(p);
+              const float dx = KIND != OutKind::I32 ? __ldg(x_scale + t) : 0.0f;
+              store_one<KIND>(y, ldy, t, n, acc, dx, dw);
+              *p = 0;
+            }
+          }
+          if (et == 0) tile_count[tile] = 0u;
+        }
+        named_barrier(1, 128);
+      }
+      ab ^= 1;
+      if (ab == 0) aphase ^= 1;
+      w = seg_end;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, L::kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -541,9 +784,40 @@ int pair_capacity() {
 
 constexpr int kPairStages = 6;
 
+template <int MP, OutKind KIND>
+cudaError_t launch_decode(const int8_t *xq, const float *x_scale, const int8_t *wq, const float *w_scale, int M,
+                          int N, int K, void *y, int64_t ldy, void *workspace, cudaStream_t st) {
+  using L = DecSmem<MP>;
+  auto kern = w8a8_gemm_decode_kernel<MP, KIND>;
+  static bool attr_set[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (!attr_set[dev & 63]) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::kTotal);
+    if (e != cudaSuccess) return e;
+    attr_set[dev & 63] = true;
+  }
+  CUtensorMap tmW, tmX;
+  if (!make_tmap_i8(&tmW, wq, N, K, kDecRows)) return cudaErrorInvalidValue;
+  if (!make_tmap_i8(&tmX, xq, M, K, MP)) return cudaErrorInvalidValue;
+  const int64_t items = (int64_t)((N + kDecRows - 1) / kDecRows) * ((K + kBK - 1) / kBK);
+  const int grid = (int)(items < num_sms() ? items : num_sms());
+  int32_t *ws = static_cast<int32_t *>(workspace);
+  unsigned *counts = reinterpret_cast<unsigned *>(static_cast<uint8_t *>(workspace) + decode_ws_elems(M, N) * 4);
+  kern<<<grid, kThreads, L::kTotal, st>>>(tmW, tmX, x_scale, w_scale, y, ldy, M, N, K, ws, counts,
+                                          device_error_word());
+  return cudaGetLastError();
+}
+
 template <OutKind KIND>
 cudaError_t gemm_dispatch(const int8_t *xq, const float *x_scale, const int8_t *wq, const float *w_scale, int M,
-                          int N, int K, void *y, int64_t ldy, cudaStream_t st) {
+                          int N, int K, void *y, int64_t ldy, void *workspace, cudaStream_t st) {
+  if (M <= kDecodeMaxM) {  // weight-streaming regime
+    if (M <= 16) return launch_decode<16, KIND>(xq, x_scale, wq, w_scale, M, N, K, y, ldy, workspace, st);
+    if (M <= 32) return launch_decode<32, KIND>(xq, x_scale, wq, w_scale, M, N, K, y, ldy, workspace, st);
+    if (M <= 48) return launch_decode<48, KIND>(xq, x_scale, wq, w_scale, M, N, K, y, ldy, workspace, st);
+    return launch_decode<64, KIND>(xq, x_scale, wq, w_scale, M, N, K, y, ldy, workspace, st);
+  }
   const int sms = num_sms();
   CUtensorMap tmA, tmB;
   // CTA pairs once there are enough 256 x 256 tiles to occupy every pair
@@ -567,17 +841,20 @@ cudaError_t gemm_dispatch(const int8_t *xq, const float *x_scale, const int8_t *
 
 }  // namespace
 
-size_t w8a8_workspace_bytes(int64_t, int64_t, int64_t) { return 0; }
+size_t w8a8_workspace_bytes(int64_t M, int64_t N, int64_t) {
+  if (M <= 0 || M > kDecodeMaxM) return 0;
+  return decode_ws_elems(M, N) * 4 + decode_counter_bytes(N);
+}
 
 cudaError_t launch_w8a8_gemm(const int8_t *xq, const float *x_scale, const int8_t *wq, const float *w_scale,
-                             int64_t M, int64_t N, int64_t K, void *y, OutKind kind, int64_t ldy, void *, size_t,
+                             int64_t M, int64_t N, int64_t K, void *y, OutKind kind, int64_t ldy, void *ws, size_t,
                              cudaStream_t st) {
+  const int m = (int)M, n = (int)N, k = (int)K;
   switch (kind) {
-    case OutKind::F32: return gemm_dispatch<OutKind::F32>(xq, x_scale, wq, w_scale, (int)M, (int)N, (int)K, y, ldy, st);
-    case OutKind::F16: return gemm_dispatch<OutKind::F16>(xq, x_scale, wq, w_scale, (int)M, (int)N, (int)K, y, ldy, st);
-    case OutKind::BF16:
-      return gemm_dispatch<OutKind::BF16>(xq, x_scale, wq, w_scale, (int)M, (int)N, (int)K, y, ldy, st);
-    default: return gemm_dispatch<OutKind::I32>(xq, nullptr, wq, nullptr, (int)M, (int)N, (int)K, y, ldy, st);
+    case OutKind::F32: return gemm_dispatch<OutKind::F32>(xq, x_scale, wq, w_scale, m, n, k, y, ldy, ws, st);
+    case OutKind::F16: return gemm_dispatch<OutKind::F16>(xq, x_scale, wq, w_scale, m, n, k, y, ldy, ws, st);
+    case OutKind::BF16: return gemm_dispatch<OutKind::BF16>(xq, x_scale, wq, w_scale, m, n, k, y, ldy, ws, st);
+    default: return gemm_dispatch<OutKind::I32>(xq, nullptr, wq, nullptr, m, n, k, y, ldy, ws, st);
   }
 }
 

@@ -1,14 +1,25 @@
-"""Runs one libsq operation on one shape a few times, for profilers.
+"""Runs (and optionally times) one libsq operation on one shape, or a sweep
+of the workloads' shapes, for profilers and roofline measurements.
 
   python -m w8a8_post_quantization_channel_b200.profile_case --op linear \
       --M 2048 --K 4096 --N 16384 --dtype f16 --iters 3
+  python -m w8a8_post_quantization_channel_b200.profile_case --sweep decode
 
-Inputs are seeded device-side draws of the benchmark's distributions;
---op is calib (T=M tokens), weight (W [N,K]), act or linear.
+--op is calib (T = M tokens), weight (W [N, K]), act or linear.  With
+--time (implied by --sweep) every iteration is timed with CUDA events on
+the launching stream, a 512 MB buffer is rewritten between iterations so
+that L2 (126 MB) holds none of the operands, and the median is reported
+against the measured peaks: algorithmic bytes / time against HBM for calib,
+act, weight and decode-shaped linears (M <= 64: streaming Wq dominates),
+2MNK / time against the INT8 tensor peak (2 x measured bf16) otherwise.
+Inputs are seeded device-side draws of the benchmark's distributions.
 """
 from __future__ import annotations
 
 import argparse
+import json
+import os
+import statistics
 
 import torch
 
@@ -16,42 +27,124 @@ import w8a8_post_quantization_channel_b200 as sq
 from w8a8_post_quantization_channel_b200 import synth
 
 DT = {"f32": torch.float32, "f16": torch.float16, "bf16": torch.bfloat16}
+ESZ = {"f32": 4, "f16": 2, "bf16": 2}
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+SWEEPS = {
+    # decode-shaped linears: Llama-2-70B and -7B layers at M in {1, 8, 32, 64}
+    "decode": [("linear", M, K, N, "bf16") for (K, N) in ((8192, 8192), (8192, 1024), (8192, 28672),
+                                                             (28672, 8192), (4096, 4096), (4096, 11008),
+                                                             (11008, 4096))
+               for M in (1, 8, 32, 64)],
+    # activation quantization on 16384-token batches
+    "act": [("act", 16384, K, 0, "bf16") for K in (4096, 7168, 8192, 28672)] + [("act", 2048, 4096, 0, "f16"),
+                                                                                   ("act", 2048, 16384, 0, "f16")],
+    # calibration chunks of the token stream
+    "calib": [("calib", 131072, K, 0, "bf16") for K in (4096, 7168, 8192)] + [("calib", 32768, 28672, 0, "bf16"),
+                                                                                 ("calib", 65536, 4096, 0, "f16"),
+                                                                                 ("calib", 65536, 16384, 0, "f16")],
+    # smoothing + weight quantization, [K, K] and the OPT shapes
+    "weight": [("weight", 0, K, K, "bf16") for K in (4096, 7168, 8192, 28672)] + [("weight", 0, 4096, 12288, "f16"),
+                                                                                     ("weight", 0, 16384, 4096, "f16")],
+    # prefill-shaped linears
+    "prefill": [("linear", 2048, K, N, "f16") for _, K, N in synth.OPT_6_7B]
+               + [("linear", 4096, K, N, "bf16") for _, K, N in synth.LLAMA2_70B[1:]]
+               + [("linear", M, 4096, 11008, "bf16") for M in (128, 1024, 4096)],
+}
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), 2.0 * float(d["bf16_tflops"]), "measured"
+    return 6650.0, 2.0 * 1590.0, "fallback"
+
+
+def make_case(op, M, K, N, dtype, dev="cuda"):
+    dt = DT[dtype]
+    o = synth.outliers(K, frac=0.01, mult=100.0, seed=1)
+    if op in ("calib", "act"):
+        x = synth.activations(M, K, o, 2, dt, device=dev)
+        amax = torch.zeros(K, device=dev)
+        inv = torch.rand(K, device=dev) + 0.5
+        xq = torch.empty(M, K, dtype=torch.int8, device=dev)
+        xs = torch.empty(M, device=dev)
+        if op == "calib":
+            return (lambda: sq.sq_calib_absmax(x, amax)), M * K * ESZ[dtype] + 8 * K, None
+        return (lambda: sq.sq_quant_act(x, inv, xq=xq, x_scale=xs)), M * K * (ESZ[dtype] + 1) + 4 * (M + K), None
+    if op == "weight":
+        w = synth.weights(K, N, 3, dt, "nk", device=dev)
+        amax = torch.rand(K, device=dev) * 10
+        outs = dict(wq=torch.empty(N, K, dtype=torch.int8, device=dev), w_scale=torch.empty(N, device=dev),
+                    smooth=torch.empty(K, device=dev), inv_smooth=torch.empty(K, device=dev))
+        fn = lambda: sq.sq_smooth_quant_weight(w, sq.SQ_W_NK, amax, 0.5, **outs)  # noqa: E731
+        return fn, 2 * N * K * ESZ[dtype] + N * K + 4 * N + 16 * K, None
+    g = synth.gen(4, dev)
+    xq = torch.randint(-127, 128, (M, K), generator=g, dtype=torch.int8, device=dev)
+    wq = torch.randint(-127, 128, (N, K), generator=g, dtype=torch.int8, device=dev)
+    xs = torch.rand(M, device=dev) * 1e-2
+    ws = torch.rand(N, device=dev) * 1e-2
+    y = torch.empty(M, N, dtype=dt, device=dev)
+    need = sq.sq_w8a8_linear_workspace_size(M, N, K)
+    work = torch.zeros(max(need, 1), dtype=torch.uint8, device=dev) if need else None
+    fn = lambda: sq.sq_w8a8_linear(xq, xs, wq, ws, dt, y=y, workspace=work)  # noqa: E731
+    return fn, M * K + N * K + M * N * ESZ[dtype] + 4 * (M + N), 2 * M * N * K
+
+
+def time_case(op, M, K, N, dtype, iters):
+    fn, nbytes, ops = make_case(op, M, K, N, dtype)
+    flush = torch.empty(512 * 2 ** 20, dtype=torch.uint8, device="cuda")
+    fn()
+    torch.cuda.synchronize()
+    times = []
+    for i in range(iters):
+        flush.fill_(i & 0xFF)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        fn()
+        b.record()
+        torch.cuda.synchronize()
+        times.append(a.elapsed_time(b) * 1e-3)
+    if sq.sq_check_device_error() != sq.SQ_OK:
+        raise SystemExit("device-side timeout")
+    t = statistics.median(times)
+    hbm, int8_peak, src = peaks()
+    out = {"op": op, "M": M, "K": K, "N": N, "dtype": dtype, "us": round(t * 1e6, 2),
+           "GB/s": round(nbytes / t / 1e9, 1), "frac_hbm": round(nbytes / t / 1e9 / hbm, 3)}
+    if ops is not None:
+        out["TOPS"] = round(ops / t / 1e12, 1)
+        out["frac_int8_peak"] = round(ops / t / 1e12 / int8_peak, 3)
+        out["bound"] = "hbm" if M <= 64 else "tensor"
+    else:
+        out["bound"] = "hbm"
+    out["peaks"] = src
+    return out
 
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--op", choices=["calib", "weight", "act", "linear"], required=True)
+    ap.add_argument("--op", choices=["calib", "weight", "act", "linear"])
+    ap.add_argument("--sweep", choices=sorted(SWEEPS))
     ap.add_argument("--M", type=int, default=2048)
     ap.add_argument("--K", type=int, default=4096)
     ap.add_argument("--N", type=int, default=4096)
     ap.add_argument("--dtype", choices=list(DT), default="f16")
     ap.add_argument("--iters", type=int, default=3)
+    ap.add_argument("--time", action="store_true")
     a = ap.parse_args()
-    dev = "cuda"
-    dt = DT[a.dtype]
-    o = synth.outliers(a.K, frac=0.01, mult=100.0, seed=1)
-    if a.op in ("calib", "act"):
-        x = synth.activations(a.M, a.K, o, 2, dt, device=dev)
-        amax = torch.zeros(a.K, device=dev)
-        inv = torch.rand(a.K, device=dev) + 0.5
-        xq = torch.empty(a.M, a.K, dtype=torch.int8, device=dev)
-        xs = torch.empty(a.M, device=dev)
-        fn = (lambda: sq.sq_calib_absmax(x, amax)) if a.op == "calib" else \
-            (lambda: sq.sq_quant_act(x, inv, xq=xq, x_scale=xs))
-    elif a.op == "weight":
-        w = synth.weights(a.K, a.N, 3, dt, "nk", device=dev)
-        amax = torch.rand(a.K, device=dev) * 10
-        outs = dict(wq=torch.empty(a.N, a.K, dtype=torch.int8, device=dev), w_scale=torch.empty(a.N, device=dev),
-                    smooth=torch.empty(a.K, device=dev), inv_smooth=torch.empty(a.K, device=dev))
-        fn = lambda: sq.sq_smooth_quant_weight(w, sq.SQ_W_NK, amax, 0.5, **outs)  # noqa: E731
-    else:
-        g = synth.gen(4, dev)
-        xq = torch.randint(-127, 128, (a.M, a.K), generator=g, dtype=torch.int8, device=dev)
-        wq = torch.randint(-127, 128, (a.N, a.K), generator=g, dtype=torch.int8, device=dev)
-        xs = torch.rand(a.M, device=dev) * 1e-2
-        ws = torch.rand(a.N, device=dev) * 1e-2
-        y = torch.empty(a.M, a.N, dtype=dt, device=dev)
-        fn = lambda: sq.sq_w8a8_linear(xq, xs, wq, ws, dt, y=y)  # noqa: E731
+    if a.sweep:
+        for case in SWEEPS[a.sweep]:
+            print(json.dumps(time_case(*case, iters=max(a.iters, 5))), flush=True)
+            torch.cuda.empty_cache()
+        return
+    if a.op is None:
+        raise SystemExit("--op or --sweep is required")
+    if a.time:
+        print(json.dumps(time_case(a.op, a.M, a.K, a.N, a.dtype, a.iters)))
+        return
+    fn, _, _ = make_case(a.op, a.M, a.K, a.N, a.dtype)
     for _ in range(a.iters):
         fn()
     torch.cuda.synchronize()
