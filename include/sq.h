@@ -149,6 +149,41 @@ sq_status sq_w8a8_accumulate(const int8_t *xq, const int8_t *wq, int64_t M,
                              sq_stream_t stream);
 
 /*
+ * Allocation-free variant of sq_w8a8_linear for decode-shaped calls.
+ * (This has no counterpart in the SmoothQuant page; it is a deployment
+ * convenience of this library.)
+ *
+ * Some callers cannot allocate device memory at the point of the call:
+ * plugins whose host framework owns all device memory through its own pool
+ * and forbids side allocations, latency-critical loops that cannot accept
+ * cudaMalloc's implicit device-wide synchronisation, and code running inside
+ * an allocator's own callbacks.  sq_w8a8_linear needs a caller-provided
+ * workspace for 1 <= M <= 64; this entry point instead uses a scratch array
+ * of SQ_DECODE_STATIC_SCRATCH_BYTES compiled into the library (a static
+ * device array that every GPU which loads the library holds until the
+ * process exits).  It allocates nothing and calls no allocating routine.
+ *
+ * Arguments, layouts and results are those of sq_w8a8_linear (minus the
+ * workspace); the results are identical.
+ *   - 1 <= M <= 64 and sq_w8a8_linear_workspace_size(M, N, K) <=
+ *     SQ_DECODE_STATIC_SCRATCH_BYTES, else SQ_ERR_UNSUPPORTED (nothing is
+ *     enqueued).  M == 0 is a no-op.
+ *   - The first call on a device looks up the scratch array's device
+ *     address (once per device, with that device current); make that first
+ *     call outside any stream capture.
+ *   - Every call on a device shares the one scratch array and clears the
+ *     part it uses on `stream` before using it.  Calls whose work overlaps
+ *     on the GPU (different streams without ordering, or several host
+ *     threads) race on the scratch and give wrong results: serialise them.
+ */
+#define SQ_DECODE_STATIC_SCRATCH_BYTES ((size_t)8 << 20) /* 8 MiB */
+sq_status sq_w8a8_linear_decode_noalloc(const int8_t *xq, const float *x_scale,
+                                        const int8_t *wq, const float *w_scale,
+                                        int64_t M, int64_t N, int64_t K,
+                                        void *y, sq_dtype yt, int64_t ldy,
+                                        sq_stream_t stream);
+
+/*
  * Synchronises `stream`, then reports (and clears) a timeout that any
  * kernel of this library recorded on the current device since the last
  * check: SQ_ERR_TIMEOUT, else SQ_OK (or SQ_ERR_CUDA if the sync failed).

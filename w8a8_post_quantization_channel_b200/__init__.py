@@ -33,6 +33,7 @@ __all__ = [
     "lib", "library_path", "header_functions",
     "sq_calib_absmax", "sq_smooth_quant_weight", "sq_quant_act", "sq_w8a8_linear",
     "sq_w8a8_linear_workspace_size", "sq_w8a8_accumulate", "sq_check_device_error", "sq_status_string",
+    "sq_w8a8_linear_decode_noalloc", "SQ_DECODE_STATIC_SCRATCH_BYTES",
 ]
 
 SQ_OK, SQ_ERR_INVALID_ARG, SQ_ERR_UNSUPPORTED, SQ_ERR_CUDA, SQ_ERR_TIMEOUT = 0, 1, 2, 3, 4
@@ -77,6 +78,7 @@ def lib() -> ctypes.CDLL:
             "sq_w8a8_linear": [vp, vp, vp, vp, i64, i64, i64, vp, i32, i64, vp, sz, vp],
             "sq_w8a8_accumulate": [vp, vp, i64, i64, i64, vp, i64, vp, sz, vp],
             "sq_check_device_error": [vp],
+            "sq_w8a8_linear_decode_noalloc": [vp, vp, vp, vp, i64, i64, i64, vp, i32, i64, vp],
         }
         for name, args in sigs.items():
             fn = getattr(L, name)
@@ -197,6 +199,29 @@ def sq_w8a8_accumulate(xq: torch.Tensor, wq: torch.Tensor, acc=None, workspace=N
     _check(lib().sq_w8a8_accumulate(_ptr(xq), _ptr(wq), M, N, K, _ptr(acc), acc.stride(0), _ptr(workspace),
                                     wbytes, _stream(stream)), "sq_w8a8_accumulate")
     return acc
+
+
+# Size of the scratch array compiled into libsq.so for the allocation-free
+# decode entry point (SQ_DECODE_STATIC_SCRATCH_BYTES in include/sq.h).
+SQ_DECODE_STATIC_SCRATCH_BYTES = 8 << 20
+
+
+def sq_w8a8_linear_decode_noalloc(xq: torch.Tensor, x_scale: torch.Tensor, wq: torch.Tensor,
+                                  w_scale: torch.Tensor, out_dtype=torch.bfloat16, y=None,
+                                  stream=None) -> torch.Tensor:
+    """sq_w8a8_linear for 1 <= M <= 64 without a caller workspace: for callers
+    that must not allocate device memory at call time, the library uses a
+    scratch array of its own (shared by all calls on a device, so calls must
+    not overlap on the GPU).  y may be preallocated to avoid any allocation
+    here as well."""
+    M, K = xq.shape
+    N = wq.shape[0]
+    y = torch.empty((M, N), dtype=out_dtype, device=xq.device) if y is None else y
+    _rowmajor(y, "y")
+    _check(lib().sq_w8a8_linear_decode_noalloc(_ptr(xq), _ptr(x_scale), _ptr(wq), _ptr(w_scale), M, N, K,
+                                               _ptr(y), _dtype(y, "y"), y.stride(0), _stream(stream)),
+           "sq_w8a8_linear_decode_noalloc")
+    return y
 
 
 def sq_check_device_error(stream=None) -> int:

@@ -859,3 +859,63 @@ cudaError_t launch_w8a8_gemm(const int8_t *xq, const float *x_scale, const int8_
 }
 
 }  // namespace sq
+
+// ---------------------------------------------------------------------------
+// Allocation-free decode entry point: the decode kernel's workspace comes
+// from a scratch array compiled into this library instead of from the
+// caller.  Its host-side name is not a device address, so the address is
+// looked up once per device (cudaGetSymbolAddress, that device current).
+// ---------------------------------------------------------------------------
+static __device__ __align__(256) uint8_t sq_decode_scratch[SQ_DECODE_STATIC_SCRATCH_BYTES];
+
+namespace {
+
+// Device address of sq_decode_scratch on the current device, looked up on
+// the first call per device; nullptr (and *err set) if the lookup fails.
+void *decode_scratch_address(cudaError_t *err) {
+  static void *addr[64] = {};
+  static std::mutex mu;
+  int dev = 0;
+  *err = cudaGetDevice(&dev);
+  if (*err != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (addr[dev] == nullptr) {
+    void *p = nullptr;
+    *err = cudaGetSymbolAddress(&p, sq_decode_scratch);
+    if (*err != cudaSuccess) return nullptr;
+    addr[dev] = p;
+  }
+  return addr[dev];
+}
+
+bool is_aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+
+extern "C" sq_status sq_w8a8_linear_decode_noalloc(const int8_t *xq, const float *x_scale, const int8_t *wq,
+                                                   const float *w_scale, int64_t M, int64_t N, int64_t K, void *y,
+                                                   sq_dtype yt, int64_t ldy, sq_stream_t stream) {
+  if (yt != SQ_F32 && yt != SQ_F16 && yt != SQ_BF16) return SQ_ERR_INVALID_ARG;
+  const int64_t ysize = yt == SQ_F32 ? 4 : 2;
+  if (M < 0 || N <= 0 || K <= 0 || N % 16 != 0 || K % 16 != 0 || N >= ((int64_t)1 << 31) ||
+      K >= ((int64_t)1 << 31))
+    return SQ_ERR_INVALID_ARG;
+  if (ldy < N || (ldy * ysize) % 16 != 0) return SQ_ERR_INVALID_ARG;
+  if (wq == nullptr || w_scale == nullptr || !is_aligned16(wq) || !is_aligned16(w_scale)) return SQ_ERR_INVALID_ARG;
+  if (M == 0) return SQ_OK;
+  if (xq == nullptr || x_scale == nullptr || y == nullptr || !is_aligned16(xq) || !is_aligned16(x_scale) ||
+      !is_aligned16(y))
+    return SQ_ERR_INVALID_ARG;
+  if (M > sq::kDecodeMaxM) return SQ_ERR_UNSUPPORTED;
+  const size_t need = sq::w8a8_workspace_bytes(M, N, K);
+  if (need == 0 || need > SQ_DECODE_STATIC_SCRATCH_BYTES) return SQ_ERR_UNSUPPORTED;
+  cudaError_t e = cudaSuccess;
+  void *scratch = decode_scratch_address(&e);
+  if (scratch == nullptr) return SQ_ERR_CUDA;
+  cudaStream_t st = (cudaStream_t)stream;
+  // the decode kernel expects zero partial sums and zero tile counters
+  if (cudaMemsetAsync(scratch, 0, need, st) != cudaSuccess) return SQ_ERR_CUDA;
+  const sq::OutKind kind = yt == SQ_F32 ? sq::OutKind::F32 : yt == SQ_F16 ? sq::OutKind::F16 : sq::OutKind::BF16;
+  e = sq::launch_w8a8_gemm(xq, x_scale, wq, w_scale, M, N, K, y, kind, ldy, scratch, need, st);
+  return e == cudaSuccess ? SQ_OK : SQ_ERR_CUDA;
+}
