@@ -40,9 +40,11 @@ WORKLOAD = ("OPT-6.7B linears qkv 4096x12288, out 4096x4096, fc1 4096x16384, fc2
             "M=2048 tokens; calibration 128x512 tokens per linear; alpha=0.5; W [N,K]")
 METRIC = "W8A8 smoothed linear TOPS & % INT8 tensor peak; act-quant GB/s % of HBM"
 INT8_PER_BF16 = 2.0  # nominal dense INT8 / dense bf16 tensor throughput (4.5 / 2.25 PFLOP/s)
-# Kernel launches of libsq per linear per step: calib 1, weight 3
-# (column max, smoothing factor, row quantizer), act-quant 1, linear 1.
-LAUNCHES_PER_LINEAR = 6
+# Kernel launches of libsq per linear per step: calib 1, weight 4
+# (zero fill, column max, smoothing factor, row quantizer), act-quant 1,
+# linear 1.
+LAUNCHES_PER_LINEAR = 7
+WEIGHT_LAUNCHES = 4
 
 # Per-launch DRAM traffic (read + write bytes) from ncu captures of the
 # benchmark's own command; each entry is tied to the hash of the kernel
@@ -250,7 +252,7 @@ def bench_ours(args, rank, world, local_rank):
     rows = {}
     for r, key in (("calib", "calib"), ("weight", "weight"), ("act", "act")):
         gbs = work[key] / (row_ms[r] * 1e-3) / 1e9
-        rows[r] = {"ms_per_step": round(row_ms[r], 4), "launches_per_step": nlin * (3 if r == "weight" else 1),
+        rows[r] = {"ms_per_step": round(row_ms[r], 4), "launches_per_step": nlin * (WEIGHT_LAUNCHES if r == "weight" else 1),
                    "algorithmic_bytes_per_step": work[key], "GB/s": round(gbs, 1),
                    "frac_of_hbm": round(gbs / pk["hbm"], 4)}
     tops = work["linear_ops"] / (row_ms["linear"] * 1e-3) / 1e12
@@ -265,8 +267,8 @@ def bench_ours(args, rank, world, local_rank):
                 "traffic": traffic_for("w8a8_gemm_tc_kernel"),
                 "peak_note": "INT8 = 2 x measured sustained bf16 (nominal dense ratio 4.5/2.25)"}
     else:
-        per_launch_bytes = work[dominant] / (nlin * (3 if dominant == "weight" else 1))
-        per_launch_ms = row_ms[dominant] / (nlin * (3 if dominant == "weight" else 1))
+        per_launch_bytes = work[dominant] / (nlin * (WEIGHT_LAUNCHES if dominant == "weight" else 1))
+        per_launch_ms = row_ms[dominant] / (nlin * (WEIGHT_LAUNCHES if dominant == "weight" else 1))
         kname = {"calib": "absmax_cols_kernel", "act": "quant_rows_kernel", "weight": "weight path"}[dominant]
         ach = per_launch_bytes / (per_launch_ms * 1e-3) / 1e9
         roof = {"kernel": kname, "bound": "hbm", "achieved": round(ach, 1), "peak": pk["hbm"], "unit": "GB/s",

@@ -119,12 +119,14 @@ def test_smooth_quant_weight(layout, dt, alpha, K, N):
 
 
 # ---------------------------------------------------------------------------
-# activation quantization (every register-tiling variant and the two-pass one)
+# activation quantization: every register-tiling variant, the shared-memory
+# staged kernel for long rows (K > 16384 at 16 bits, > 8192 at 32 bits) and
+# the two-pass kernel beyond it
 # ---------------------------------------------------------------------------
 
 @pytest.mark.parametrize("dt,K", [("bf16", 16), ("bf16", 2048), ("bf16", 4096), ("f16", 11008), ("bf16", 16384),
-                                  ("bf16", 28672), ("bf16", 40960), ("f32", 256), ("f32", 4096), ("f32", 20000),
-                                  ("f16", 1040)])
+                                  ("bf16", 28672), ("f16", 20480), ("bf16", 40960), ("f32", 256), ("f32", 4096),
+                                  ("f32", 12288), ("f32", 20000), ("f16", 1040)])
 @pytest.mark.parametrize("M", [1, 5, 33])
 def test_quant_act(dt, K, M):
     o = synth.outliers(K, frac=0.01, mult=100.0, seed=K)

@@ -93,7 +93,7 @@ sq_status sq_calib_absmax(const void *x, sq_dtype xt, int64_t T, int64_t K, int6
   if (ldx < K || (ldx * dsize(xt)) % 16 != 0) return SQ_ERR_INVALID_ARG;
   if (T == 0) return SQ_OK;
   if (!valid_matrix(x, xt, T, K, ldx)) return SQ_ERR_INVALID_ARG;
-  return from_cuda(sq::launch_absmax_cols(x, xt, T, K, ldx, nullptr, amax, (cudaStream_t)stream));
+  return from_cuda(sq::launch_absmax_cols(x, xt, T, K, ldx, nullptr, amax, false, (cudaStream_t)stream));
 }
 
 sq_status sq_smooth_quant_weight(const void *w, sq_dtype wt, sq_wlayout layout, int64_t K, int64_t N, int64_t ldw,
@@ -112,8 +112,8 @@ sq_status sq_smooth_quant_weight(const void *w, sq_dtype wt, sq_wlayout layout, 
   if (kn) {
     e = sq::launch_absmax_rows(w, wt, K, N, ldw, smooth, st);
   } else {
-    e = cudaMemsetAsync(smooth, 0, K * sizeof(float), st);
-    if (e == cudaSuccess) e = sq::launch_absmax_cols(w, wt, N, K, ldw, nullptr, smooth, st);
+    e = sq::launch_zero_fill(smooth, K, st);
+    if (e == cudaSuccess) e = sq::launch_absmax_cols(w, wt, N, K, ldw, nullptr, smooth, true, st);
   }
   if (e != cudaSuccess) return SQ_ERR_CUDA;
   // s_j, 1/s_j
@@ -121,8 +121,8 @@ sq_status sq_smooth_quant_weight(const void *w, sq_dtype wt, sq_wlayout layout, 
   if (e != cudaSuccess) return SQ_ERR_CUDA;
   // W~ = diag(s) W, per-output-channel INT8
   if (kn) {
-    e = cudaMemsetAsync(w_scale, 0, N * sizeof(float), st);
-    if (e == cudaSuccess) e = sq::launch_absmax_cols(w, wt, K, N, ldw, smooth, w_scale, st);
+    e = sq::launch_zero_fill(w_scale, N, st);
+    if (e == cudaSuccess) e = sq::launch_absmax_cols(w, wt, K, N, ldw, smooth, w_scale, true, st);
     if (e == cudaSuccess) e = sq::launch_quant_cols_transpose(w, wt, K, N, ldw, smooth, w_scale, wq, st);
   } else {
     e = sq::launch_quant_rows(w, wt, N, K, ldw, smooth, wq, w_scale, st);

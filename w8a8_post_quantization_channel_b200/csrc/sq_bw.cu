@@ -29,9 +29,14 @@ constexpr int kColUnroll = 4;     // independent row loads in flight per thread
 template <typename T, bool kScaled>
 __global__ void __launch_bounds__(kColThreadsX *kColThreadsY)
     absmax_cols_kernel(const T *__restrict__ x, int64_t rows, int64_t nvec, int64_t ld,
-                       const float *__restrict__ row_scale, float *__restrict__ amax) {
+                       const float *__restrict__ row_scale, float *__restrict__ amax, bool keep_in_l2) {
+  pdl_wait();  // the previous kernel's results are visible from here on
+  pdl_trigger();
   constexpr int V = Vec<T>::N;
   __shared__ float red[kColThreadsY][kColThreadsX * V];
+  // data read again right after this kernel (the weights) is kept in L2,
+  // read-once data (a calibration stream) is marked first to go
+  const uint64_t policy = keep_in_l2 ? policy_evict_last() : policy_evict_first();
   const int64_t v = (int64_t)blockIdx.x * kColThreadsX + threadIdx.x;
   const int64_t chunk = (rows + gridDim.y - 1) / gridDim.y;
   const int64_t r0 = (int64_t)blockIdx.y * chunk;
@@ -45,7 +50,7 @@ __global__ void __launch_bounds__(kColThreadsX *kColThreadsY)
     for (; r + (kColUnroll - 1) * kColThreadsY < r1; r += kColUnroll * kColThreadsY) {
       uint4 raw[kColUnroll];
 #pragma unroll
-      for (int u = 0; u < kColUnroll; ++u) raw[u] = ld_stream_v4(col + (r + u * kColThreadsY) * ld);
+      for (int u = 0; u < kColUnroll; ++u) raw[u] = ld_policy_v4(col + (r + u * kColThreadsY) * ld, policy);
 #pragma unroll
       for (int u = 0; u < kColUnroll; ++u) {
         float f[V];
@@ -57,7 +62,7 @@ __global__ void __launch_bounds__(kColThreadsX *kColThreadsY)
     }
     for (; r < r1; r += kColThreadsY) {
       float f[V];
-      Vec<T>::to_f32(ld_stream_v4(col + r * ld), f);
+      Vec<T>::to_f32(ld_policy_v4(col + r * ld, policy), f);
       const float sc = kScaled ? __ldg(row_scale + r) : 1.0f;
 #pragma unroll
       for (int e = 0; e < V; ++e) m[e] = fmaxf(m[e], fabsf(kScaled ? __fmul_rn(sc, f[e]) : f[e]));
@@ -83,6 +88,8 @@ __global__ void __launch_bounds__(kColThreadsX *kColThreadsY)
 template <typename T>
 __global__ void __launch_bounds__(256) absmax_rows_kernel(const T *__restrict__ x, int64_t nvec, int64_t ld,
                                                           float *__restrict__ out) {
+  pdl_wait();  // the previous kernel's results are visible from here on
+  pdl_trigger();
   constexpr int V = Vec<T>::N;
   __shared__ float red[32];
   const T *row = x + (int64_t)blockIdx.x * ld;
@@ -101,6 +108,8 @@ __global__ void __launch_bounds__(256) absmax_rows_kernel(const T *__restrict__ 
 // quarter-step alphas, double pow (rounded once) otherwise.
 __global__ void smooth_factor_kernel(const float *__restrict__ amax, float *__restrict__ s_inout,
                                      float *__restrict__ inv_s, int64_t K, float alpha) {
+  pdl_wait();  // the previous kernel's results are visible from here on
+  pdl_trigger();
   const int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (j >= K) return;
   const float a = fmaxf(amax[j], 1e-5f);
@@ -142,6 +151,8 @@ template <typename T, int kVPT>
 __global__ void __launch_bounds__(kRowMaxThreads)
     quant_rows_kernel(const T *__restrict__ x, int64_t rows, int64_t nvec, int64_t ld,
                       const float *__restrict__ col_scale, int8_t *__restrict__ q, float *__restrict__ row_scale_out) {
+  pdl_wait();  // the previous kernel's results are visible from here on
+  pdl_trigger();
   constexpr int V = Vec<T>::N;
   __shared__ float red[2][kRowMaxThreads / 32];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -155,12 +166,13 @@ __global__ void __launch_bounds__(kRowMaxThreads)
 #pragma unroll
     for (int e = 0; e < V; ++e) sc[i][e] = v < nvec ? __ldg(col_scale + v * V + e) : 0.0f;
   }
+  const uint64_t policy = policy_evict_first();  // every row is read exactly once
   uint4 cur[kVPT], nxt[kVPT];
   int64_t r = blockIdx.x;
 #pragma unroll
   for (int i = 0; i < kVPT; ++i) {
     const int64_t v = tid + (int64_t)i * blockDim.x;
-    cur[i] = (r < rows && v < nvec) ? ld_stream_v4(x + r * ld + v * V) : make_uint4(0, 0, 0, 0);
+    cur[i] = (r < rows && v < nvec) ? ld_policy_v4(x + r * ld + v * V, policy) : make_uint4(0, 0, 0, 0);
   }
   int slot = 0;
   for (; r < rows; r += gridDim.x) {
@@ -168,7 +180,7 @@ __global__ void __launch_bounds__(kRowMaxThreads)
 #pragma unroll
     for (int i = 0; i < kVPT; ++i) {
       const int64_t v = tid + (int64_t)i * blockDim.x;
-      nxt[i] = (rn < rows && v < nvec) ? ld_stream_v4(x + rn * ld + v * V) : make_uint4(0, 0, 0, 0);
+      nxt[i] = (rn < rows && v < nvec) ? ld_policy_v4(x + rn * ld + v * V, policy) : make_uint4(0, 0, 0, 0);
     }
     float val[kVPT][V];
     float m = 0.0f;
@@ -218,6 +230,127 @@ __global__ void __launch_bounds__(kRowMaxThreads)
   }
 }
 
+// Row quantizer for long rows (persistent, one CTA of 512 threads per SM):
+// whole rows are staged in shared memory by bulk async copies into
+// kStages buffers (one mbarrier each), issued kStages rows ahead; the
+// column scales stay in registers; each row is read from shared memory
+// twice (maximum, then codes), so HBM sees every byte once.
+constexpr int kSmemRowThreads = 512;
+template <typename T, int kVPT, int kStages>
+__global__ void __launch_bounds__(kSmemRowThreads, 1)
+    quant_rows_smem_kernel(const T *__restrict__ x, int64_t rows, int64_t nvec, int64_t ld,
+                           const float *__restrict__ col_scale, int8_t *__restrict__ q,
+                           float *__restrict__ row_scale_out, uint32_t row_bytes, unsigned *err) {
+  pdl_wait();  // the previous kernel's results are visible from here on
+  pdl_trigger();
+  constexpr int V = Vec<T>::N;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+  const uint32_t buf_bytes = (row_bytes + 127u) & ~127u;
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + kStages * buf_bytes);
+  float *red = reinterpret_cast<float *>(full + kStages);  // [2][16]
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(red + 32);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int64_t K = nvec * V;
+
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s) mbar_init(&full[s], 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      const int64_t r = blockIdx.x + (int64_t)s * gridDim.x;
+      if (r < rows) {
+        mbar_arrive_expect_tx(&full[s], row_bytes);
+        bulk_load(smem + s * buf_bytes, x + r * ld, row_bytes, &full[s]);
+      }
+    }
+  }
+  float sc[kVPT][V];
+#pragma unroll
+  for (int i = 0; i < kVPT; ++i) {
+    const int64_t v = tid + (int64_t)i * kSmemRowThreads;
+#pragma unroll
+    for (int e = 0; e < V; ++e) sc[i][e] = v < nvec ? __ldg(col_scale + v * V + e) : 0.0f;
+  }
+  int slot = 0;
+  int64_t it = 0;
+  for (int64_t r = blockIdx.x; r < rows; r += gridDim.x, ++it) {
+    const int s = (int)(it % kStages);
+    const uint32_t parity = (uint32_t)((it / kStages) & 1);
+    const bool ok = mbar_wait(&full[s], parity, abort_flag, err);
+    if (!__syncthreads_and(ok)) break;
+    const uint4 *row = reinterpret_cast<const uint4 *>(smem + s * buf_bytes);
+    float m = 0.0f;
+#pragma unroll
+    for (int i = 0; i < kVPT; ++i) {
+      const int64_t v = tid + (int64_t)i * kSmemRowThreads;
+      if (v < nvec) {
+        float f[V];
+        Vec<T>::to_f32(row[v], f);
+#pragma unroll
+        for (int e = 0; e < V; e += 2) {
+          const float2 p = fmul2_rn(make_float2(f[e], f[e + 1]), make_float2(sc[i][e], sc[i][e + 1]));
+          m = fmaxf(m, fmaxf(fabsf(p.x), fabsf(p.y)));
+        }
+      }
+    }
+    m = warp_max(m);
+    if (lane == 0) red[slot * 16 + warp] = m;
+    __syncthreads();
+    m = 0.0f;
+#pragma unroll
+    for (int w = 0; w < kSmemRowThreads / 32; ++w) m = fmaxf(m, red[slot * 16 + w]);
+    slot ^= 1;
+    const float rcp = m > 0.0f ? __fdiv_rn(127.0f, m) : 0.0f;
+    if (tid == 0) row_scale_out[r] = __fdiv_rn(m, 127.0f);
+    int8_t *qrow = q + r * K;
+#pragma unroll
+    for (int i = 0; i < kVPT; ++i) {
+      const int64_t v = tid + (int64_t)i * kSmemRowThreads;
+      if (v < nvec) {
+        float f[V];
+        Vec<T>::to_f32(row[v], f);
+        float val[V];
+#pragma unroll
+        for (int e = 0; e < V; e += 2) {
+          const float2 p = fmul2_rn(make_float2(f[e], f[e + 1]), make_float2(sc[i][e], sc[i][e + 1]));
+          val[e] = p.x;
+          val[e + 1] = p.y;
+        }
+        if constexpr (V == 8) {
+          uint2 o;
+          o.x = pack4_codes(quantize_dynamic(val[0], rcp), quantize_dynamic(val[1], rcp),
+                            quantize_dynamic(val[2], rcp), quantize_dynamic(val[3], rcp));
+          o.y = pack4_codes(quantize_dynamic(val[4], rcp), quantize_dynamic(val[5], rcp),
+                            quantize_dynamic(val[6], rcp), quantize_dynamic(val[7], rcp));
+          *reinterpret_cast<uint2 *>(qrow + v * V) = o;
+        } else {
+          *reinterpret_cast<uint32_t *>(qrow + v * V) =
+              pack4_codes(quantize_dynamic(val[0], rcp), quantize_dynamic(val[1], rcp),
+                          quantize_dynamic(val[2], rcp), quantize_dynamic(val[3], rcp));
+        }
+      }
+    }
+    __syncthreads();  // every thread is done with buffer s
+    if (tid == 0) {
+      const int64_t rn = r + (int64_t)kStages * gridDim.x;
+      if (rn < rows) {
+        mbar_arrive_expect_tx(&full[s], row_bytes);
+        bulk_load(smem + s * buf_bytes, x + rn * ld, row_bytes, &full[s]);
+      }
+    }
+  }
+  // on an abort, copies already issued must land before the CTA exits
+  if (tid == 0 && *abort_flag) {
+    int64_t r = blockIdx.x + it * gridDim.x;
+    for (int k = 0; k < kStages && r < rows; ++k, ++it, r += gridDim.x)
+      mbar_wait(&full[it % kStages], (uint32_t)((it / kStages) & 1), nullptr, err);
+  }
+}
+
 // Row quantizer for rows too long to hold in registers: one pass for the
 // maximum, a second for the codes (the row is re-read, mostly from L2).
 template <typename T>
@@ -225,6 +358,8 @@ __global__ void __launch_bounds__(1024) quant_rows_twopass_kernel(const T *__res
                                                                   const float *__restrict__ col_scale,
                                                                   int8_t *__restrict__ q,
                                                                   float *__restrict__ row_scale_out) {
+  pdl_wait();  // the previous kernel's results are visible from here on
+  pdl_trigger();
   constexpr int V = Vec<T>::N;
   __shared__ float red[32];
   const int64_t r = blockIdx.x;
@@ -267,6 +402,8 @@ __global__ void __launch_bounds__(256) quant_cols_transpose_kernel(const T *__re
                                                                    int64_t ld, const float *__restrict__ s,
                                                                    const float *__restrict__ colmax,
                                                                    int8_t *__restrict__ wq) {
+  pdl_wait();  // the previous kernel's results are visible from here on
+  pdl_trigger();
   __shared__ int8_t tile[kTT][kTT + 4];  // [n][j]
   __shared__ float rcp[kTT];
   const int64_t j0 = (int64_t)blockIdx.y * kTT, n0 = (int64_t)blockIdx.x * kTT;
@@ -307,13 +444,22 @@ __global__ void __launch_bounds__(256) quant_cols_transpose_kernel(const T *__re
 }
 
 __global__ void finalize_scale_kernel(float *__restrict__ m_to_scale, int64_t n) {
+  pdl_wait();  // the previous kernel's results are visible from here on
+  pdl_trigger();
   const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (i < n) m_to_scale[i] = __fdiv_rn(m_to_scale[i], 127.0f);
 }
 
+__global__ void zero_fill_kernel(float *__restrict__ p, int64_t n) {
+  pdl_wait();  // the previous kernel's results are visible from here on
+  pdl_trigger();
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
+    p[i] = 0.0f;
+}
+
 template <typename T>
 cudaError_t absmax_cols_t(const void *x, int64_t rows, int64_t cols, int64_t ld, const float *row_scale,
-                          float *amax, cudaStream_t st) {
+                          float *amax, bool keep_in_l2, cudaStream_t st) {
   constexpr int V = Vec<T>::N;
   const int64_t nvec = cols / V;
   const int64_t slabs = (nvec + kColThreadsX - 1) / kColThreadsX;
@@ -323,17 +469,16 @@ cudaError_t absmax_cols_t(const void *x, int64_t rows, int64_t cols, int64_t ld,
   gy = std::max<int64_t>(1, std::min<int64_t>(gy, std::min<int64_t>(max_gy, 65535)));
   dim3 grid((unsigned)slabs, (unsigned)gy), block(kColThreadsX, kColThreadsY);
   if (row_scale)
-    absmax_cols_kernel<T, true><<<grid, block, 0, st>>>((const T *)x, rows, nvec, ld, row_scale, amax);
-  else
-    absmax_cols_kernel<T, false><<<grid, block, 0, st>>>((const T *)x, rows, nvec, ld, nullptr, amax);
-  return cudaGetLastError();
+    return launch_pdl(absmax_cols_kernel<T, true>, grid, block, 0, st, 1, (const T *)x, rows, nvec, ld, row_scale,
+                      amax, keep_in_l2);
+  return launch_pdl(absmax_cols_kernel<T, false>, grid, block, 0, st, 1, (const T *)x, rows, nvec, ld,
+                    (const float *)nullptr, amax, keep_in_l2);
 }
 
 template <typename T>
 cudaError_t absmax_rows_t(const void *x, int64_t rows, int64_t cols, int64_t ld, float *out, cudaStream_t st) {
   constexpr int V = Vec<T>::N;
-  absmax_rows_kernel<T><<<(unsigned)rows, 256, 0, st>>>((const T *)x, cols / V, ld, out);
-  return cudaGetLastError();
+  return launch_pdl(absmax_rows_kernel<T>, dim3((unsigned)rows), dim3(256), 0, st, 1, (const T *)x, cols / V, ld, out);
 }
 
 template <typename T, int kVPT>
@@ -350,8 +495,26 @@ cudaError_t launch_quant_rows_persistent(const T *x, int64_t rows, int64_t nvec,
     cached = n > 0 ? n : 1;
   }
   const int64_t grid = std::min<int64_t>(rows, (int64_t)cached * num_sms());
-  quant_rows_kernel<T, kVPT><<<(unsigned)grid, threads, 0, st>>>(x, rows, nvec, ld, col_scale, q, row_scale_out);
-  return cudaGetLastError();
+  return launch_pdl(quant_rows_kernel<T, kVPT>, dim3((unsigned)grid), dim3(threads), 0, st, 1, x, rows, nvec, ld,
+                    col_scale, q, row_scale_out);
+}
+
+template <typename T, int kVPT, int kStages>
+cudaError_t launch_quant_rows_smem(const T *x, int64_t rows, int64_t nvec, int64_t ld, const float *col_scale,
+                                   int8_t *q, float *row_scale_out, uint32_t row_bytes, uint32_t smem_bytes,
+                                   cudaStream_t st) {
+  auto kern = quant_rows_smem_kernel<T, kVPT, kStages>;
+  static int attr_bytes[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (attr_bytes[dev & 63] < (int)smem_bytes) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_bytes);
+    if (e != cudaSuccess) return e;
+    attr_bytes[dev & 63] = (int)smem_bytes;
+  }
+  const int64_t grid = std::min<int64_t>(rows, (int64_t)num_sms());
+  return launch_pdl(kern, dim3((unsigned)grid), dim3(kSmemRowThreads), smem_bytes, st, 1, x, rows, nvec, ld, col_scale,
+                    q, row_scale_out, row_bytes, device_error_word());
 }
 
 template <typename T>
@@ -370,29 +533,39 @@ cudaError_t quant_rows_t(const void *x, int64_t rows, int64_t cols, int64_t ld, 
   if (nvec <= 4 * kRowMaxThreads) {
     return launch_quant_rows_persistent<T, 4>(xp, rows, nvec, ld, col_scale, q, row_scale_out, threads_for(4), st);
   }
-  quant_rows_twopass_kernel<T><<<(unsigned)rows, 1024, 0, st>>>(xp, nvec, ld, col_scale, q, row_scale_out);
-  return cudaGetLastError();
+  const uint32_t row_bytes = (uint32_t)(cols * sizeof(T));
+  const uint32_t buf = (row_bytes + 127u) & ~127u;
+  const uint32_t extra = 128 + 8 * 3 + 2 * 16 * 4 + 16;
+  if (nvec <= 8 * kSmemRowThreads && 3 * buf + extra <= 200 * 1024) {
+    return launch_quant_rows_smem<T, 8, 3>(xp, rows, nvec, ld, col_scale, q, row_scale_out, row_bytes,
+                                           3 * buf + extra, st);
+  }
+  if (nvec <= 8 * kSmemRowThreads && 2 * buf + extra <= 220 * 1024) {
+    return launch_quant_rows_smem<T, 8, 2>(xp, rows, nvec, ld, col_scale, q, row_scale_out, row_bytes,
+                                           2 * buf + extra, st);
+  }
+  return launch_pdl(quant_rows_twopass_kernel<T>, dim3((unsigned)rows), dim3(1024), 0, st, 1, xp, nvec, ld, col_scale,
+                    q, row_scale_out);
 }
 
 template <typename T>
 cudaError_t quant_cols_t(const void *w, int64_t K, int64_t N, int64_t ld, const float *s, float *colmax, int8_t *wq,
                          cudaStream_t st) {
   dim3 grid((unsigned)((N + kTT - 1) / kTT), (unsigned)((K + kTT - 1) / kTT));
-  quant_cols_transpose_kernel<T><<<grid, 256, 0, st>>>((const T *)w, K, N, ld, s, colmax, wq);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pdl(quant_cols_transpose_kernel<T>, grid, dim3(256), 0, st, 1, (const T *)w, K, N, ld, s,
+                             (const float *)colmax, wq);
   if (e != cudaSuccess) return e;
-  finalize_scale_kernel<<<(unsigned)((N + 255) / 256), 256, 0, st>>>(colmax, N);
-  return cudaGetLastError();
+  return launch_pdl(finalize_scale_kernel, dim3((unsigned)((N + 255) / 256)), dim3(256), 0, st, 1, colmax, N);
 }
 
 }  // namespace
 
 cudaError_t launch_absmax_cols(const void *x, sq_dtype xt, int64_t rows, int64_t cols, int64_t ld,
-                               const float *row_scale, float *amax, cudaStream_t st) {
+                               const float *row_scale, float *amax, bool keep_in_l2, cudaStream_t st) {
   switch (xt) {
-    case SQ_F32: return absmax_cols_t<float>(x, rows, cols, ld, row_scale, amax, st);
-    case SQ_F16: return absmax_cols_t<__half>(x, rows, cols, ld, row_scale, amax, st);
-    default: return absmax_cols_t<__nv_bfloat16>(x, rows, cols, ld, row_scale, amax, st);
+    case SQ_F32: return absmax_cols_t<float>(x, rows, cols, ld, row_scale, amax, keep_in_l2, st);
+    case SQ_F16: return absmax_cols_t<__half>(x, rows, cols, ld, row_scale, amax, keep_in_l2, st);
+    default: return absmax_cols_t<__nv_bfloat16>(x, rows, cols, ld, row_scale, amax, keep_in_l2, st);
   }
 }
 
@@ -405,10 +578,15 @@ cudaError_t launch_absmax_rows(const void *x, sq_dtype xt, int64_t rows, int64_t
   }
 }
 
+cudaError_t launch_zero_fill(float *p, int64_t n, cudaStream_t st) {
+  const int64_t blocks = std::min<int64_t>((n + 255) / 256, 4 * (int64_t)num_sms());
+  return launch_pdl(zero_fill_kernel, dim3((unsigned)std::max<int64_t>(1, blocks)), dim3(256), 0, st, 1, p, n);
+}
+
 cudaError_t launch_smooth_factor(const float *amax, float *s_inout, float *inv_s, int64_t K, float alpha,
                                  cudaStream_t st) {
-  smooth_factor_kernel<<<(unsigned)((K + 255) / 256), 256, 0, st>>>(amax, s_inout, inv_s, K, alpha);
-  return cudaGetLastError();
+  return launch_pdl(smooth_factor_kernel, dim3((unsigned)((K + 255) / 256)), dim3(256), 0, st, 1, amax, s_inout, inv_s,
+                    K, alpha);
 }
 
 cudaError_t launch_quant_rows(const void *x, sq_dtype xt, int64_t rows, int64_t cols, int64_t ld,

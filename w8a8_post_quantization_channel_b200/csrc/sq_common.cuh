@@ -10,12 +10,53 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 namespace sq {
 
 // Device error word bits (see sq_check_device_error).
 constexpr unsigned kDevErrTimeout = 1u;
 // Every in-kernel wait gives up after this long.
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s
+
+// ---------------------------------------------------------------------------
+// Programmatic dependent launch.  Every libsq kernel is launched so that it
+// may start while the previous kernel on the stream is still finishing; it
+// runs only its prologue (shared-memory barriers, TMEM allocation, tensor
+// map prefetch) before pdl_wait(), which returns once the previous grid has
+// completed and its memory is visible, and it touches global memory only
+// after that.  pdl_trigger() lets the next kernel's blocks be scheduled as
+// soon as this grid's blocks have all started.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                              unsigned cluster_x, Args &&...args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  unsigned n = 0;
+  attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[n].val.programmaticStreamSerializationAllowed = 1;
+  ++n;
+  if (cluster_x > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = cluster_x;
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
 
 // ---------------------------------------------------------------------------
 // Element types: 16-byte vectors converted exactly to fp32.
@@ -73,6 +114,15 @@ __device__ __forceinline__ uint4 ld_nc_v4(const void *p) {
 
 // Read-once data: same load; kept as a separate name for streaming inputs.
 __device__ __forceinline__ uint4 ld_stream_v4(const void *p) { return ld_nc_v4(p); }
+
+// 16-byte load with an L2 eviction policy (from createpolicy below).
+__device__ __forceinline__ uint4 ld_policy_v4(const void *p, uint64_t policy) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.u32 {%0, %1, %2, %3}, [%4], %5;"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p), "l"(policy));
+  return r;
+}
 
 // ---------------------------------------------------------------------------
 // The quantizer: clamp(rne(v * r), -127, 127), r = 127 / absmax of the row.
@@ -201,6 +251,15 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
 
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap *m) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
+}
+
+// Contiguous bulk copy global -> this CTA's shared memory (both addresses
+// 16-byte aligned, bytes a multiple of 16); completion counted on `bar`.
+__device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
 }
 
 // 2-D tiled TMA load into this CTA's shared memory; completion is counted
@@ -333,6 +392,12 @@ __device__ __forceinline__ void cluster_sync() {
 // Arrive on an mbarrier given by its shared::cluster address (any CTA).
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+// 32-bit load from shared memory of any CTA of the cluster.
+__device__ __forceinline__ uint32_t ld_shared_cluster_u32(uint32_t cluster_addr) {
+  uint32_t v;
+  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(cluster_addr) : "memory");
+  return v;
 }
 // TMA load into this CTA's shared memory whose byte count completes on an
 // mbarrier that may live in the peer CTA of the pair.

@@ -150,6 +150,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_wait();  // prologue done; the previous kernel's results are visible from here on
+  pdl_trigger();
 
   if (warp == 0) {
     if (lane == 0) {
@@ -296,7 +298,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
-  const uint32_t peer = rank ^ 1u;
   const bool leader = rank == 0;
   const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
   const int num_m = (M + 2 * kBM - 1) / (2 * kBM);
@@ -329,6 +330,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   cluster_sync();  // barriers of both CTAs initialised, TMEM allocated
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_wait();  // prologue done; the previous kernel's results are visible from here on
+  pdl_trigger();
 
   if (warp == 0) {
     if (lane == 0) {
@@ -455,15 +458,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 // the counter zero again.  No CTA waits for another.
 // ---------------------------------------------------------------------------
 constexpr int kDecRows = 128;  // Wq rows per tile (MMA M)
-constexpr int kDecStages = 8;
 
 template <int MP>
 struct DecSmem {
   static constexpr uint32_t kW = kDecRows * kBK;  // 16 KB of Wq per stage
   static constexpr uint32_t kX = MP * kBK;        // MP token rows of Xq per stage
   static constexpr uint32_t kStage = kW + kX;
-  static constexpr uint32_t kRing = kDecStages * kStage;
-  static constexpr uint32_t kBars = (2 * kDecStages + 5) * 8 + 32;
+  // Under full HBM load a request takes ~3-4 us to return, so each SM keeps
+  // as many stages in flight as ~216 KB of shared memory holds.
+  static constexpr int kStages = (216 * 1024) / kStage;
+  static constexpr uint32_t kRing = kStages * kStage;
+  static constexpr uint32_t kBars = (2 * kStages + 5) * 8 + 32;
   static constexpr uint32_t kTotal = kRing + kBars + 1024;
   static constexpr uint32_t kTmemCols = (2 * MP <= 32) ? 32 : (2 * MP <= 64) ? 64 : 128;
 };
@@ -494,8 +499,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + L::kRing);
-  uint64_t *empty = full + kDecStages;
-  uint64_t *tfull = empty + kDecStages;
+  uint64_t *empty = full + L::kStages;
+  uint64_t *tfull = empty + L::kStages;
   uint64_t *tempty = tfull + 2;
   uint64_t *drain = tempty + 2;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
@@ -510,7 +515,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int64_t w1 = items * (blockIdx.x + 1) / gridDim.x;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kDecStages; ++s) {
+    for (int s = 0; s < L::kStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
@@ -534,6 +539,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_wait();  // prologue done; the previous kernel's results are visible from here on
+  pdl_trigger();
 
   if (warp == 0) {
     if (lane == 0) {
@@ -552,13 +559,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_2d(&tmX, &full[stage], st + L::kW, kb * kBK, 0);
         armed |= 1u << stage;
         armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
-        if (++stage == kDecStages) {
+        if (++stage == L::kStages) {
           stage = 0;
           phase ^= 1;
         }
       }
       if (!ok) {
-        for (int s = 0; s < kDecStages; ++s)
+        for (int s = 0; s < L::kStages; ++s)
           if (armed & (1u << s)) mbar_wait(&full[s], (armed_parity >> s) & 1u, nullptr, err);
       }
     }
@@ -587,7 +594,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int k = 0; k < kBK / 32; ++k)
             umma_i8(d, a0 + 2 * k, b0 + 2 * k, idesc, (i != w || k != 0) ? 1u : 0u);
           umma_commit(&empty[stage]);
-          if (++stage == kDecStages) {
+          if (++stage == L::kStages) {
             stage = 0;
             phase ^= 1;
           }
@@ -652,12 +659,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (*last_flag) {
           __threadfence();
           if (n_ok) {
-            for (int t = 0; t < M; ++t) {
-              int32_t *p = ws + (int64_t)t * N + n;
-              const int32_t acc = __ldcg(p);
-              const float dx = KIND != OutKind::I32 ? __ldg(x_scale + t) : 0.0f;
-              store_one<KIND>(y, ldy, t, n, acc, dx, dw);
-              *p = 0;
+            // 16 tokens at a time: their partial sums as independent L2
+            // loads, then dequantize, store, and leave the workspace zero
+#pragma unroll 1
+            for (int t0 = 0; t0 < M; t0 += 16) {
+              int32_t acc[16];
+#pragma unroll
+              for (int j = 0; j < 16; ++j) acc[j] = t0 + j < M ? __ldcg(ws + (int64_t)(t0 + j) * N + n) : 0;
+#pragma unroll
+              for (int j = 0; j < 16; ++j) {
+                const int t = t0 + j;
+                if (t < M) {
+                  const float dx = KIND != OutKind::I32 ? __ldg(x_scale + t) : 0.0f;
+                  store_one<KIND>(y, ldy, t, n, acc[j], dx, dw);
+                  __stcg(ws + (int64_t)t * N + n, 0);
+                }
+              }
             }
           }
           if (et == 0) tile_count[tile] = 0u;
@@ -670,6 +687,205 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
 
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, L::kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Decode-shaped linear, cluster split: for at most one wave of 128-row Wq
+// tiles.  A cluster of S CTAs owns one tile; CTA c of the cluster streams
+// k-blocks [c nk / S, (c+1) nk / S) into its TMEM accumulator (Wq rows on
+// the MMA's M side, tokens on N, as in the stream-K kernel).  The S int32
+// partials are then exchanged through distributed shared memory: each CTA
+// parks its partial in its own shared memory, the cluster synchronises,
+// and CTA c sums rows [c 128 / S, (c+1) 128 / S) over all S partials and
+// dequantizes them.  No workspace, no global atomics, no fences.
+// ---------------------------------------------------------------------------
+template <int MP, OutKind KIND>
+__global__ void __launch_bounds__(kThreads, 1)
+    w8a8_gemm_decode_cluster_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
+                                    const float *__restrict__ x_scale, const float *__restrict__ w_scale,
+                                    void *__restrict__ y, int64_t ldy, int M, int N, int K, int S, unsigned *err) {
+  using L = DecSmem<MP>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + L::kRing);
+  uint64_t *empty = full + L::kStages;
+  uint64_t *tfull = empty + L::kStages;
+  uint64_t *drain = tfull + 1;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+  // after the MMAs have drained the ring, it holds this CTA's partial sums
+  // as part[t][row] (t < MP, row < 128)
+  int32_t *part = reinterpret_cast<int32_t *>(smem);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const int tile = blockIdx.x / S;
+  const int nk = (K + kBK - 1) / kBK;
+  const int kb0 = (int)((int64_t)nk * rank / S), kb1 = (int)((int64_t)nk * (rank + 1) / S);
+  // Tiles start their k-walk at different k-blocks so that the CTAs of the
+  // grid do not all fetch the same Xq tile from L2 at the same moment (the
+  // int32 sum does not depend on the order).
+  const int cnt = kb1 - kb0;
+  const int rot = cnt > 0 ? tile % cnt : 0;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < L::kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(tfull, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmW);
+    prefetch_tmap(&tmX);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, L::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  pdl_wait();  // prologue done; the previous kernel's results are visible from here on
+  pdl_trigger();
+
+  if (warp == 0) {
+    if (lane == 0) {
+      uint32_t stage = 0, phase = 0, armed = 0, armed_parity = 0;
+      bool ok = true;
+      for (int i = 0; i < cnt; ++i) {
+        const int kb = kb0 + (i + rot) % cnt;
+        if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, err)) {
+          ok = false;
+          break;
+        }
+        uint8_t *st = smem + stage * L::kStage;
+        mbar_arrive_expect_tx(&full[stage], L::kStage);
+        tma_load_2d(&tmW, &full[stage], st, kb * kBK, tile * kDecRows);
+        tma_load_2d(&tmX, &full[stage], st + L::kW, kb * kBK, 0);
+        armed |= 1u << stage;
+        armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
+        if (++stage == L::kStages) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+      if (!ok) {
+        for (int s = 0; s < L::kStages; ++s)
+          if (armed & (1u << s)) mbar_wait(&full[s], (armed_parity >> s) & 1u, nullptr, err);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_i8(kDecRows, MP);
+      uint32_t stage = 0, phase = 0;
+      for (int i = 0; i < cnt; ++i) {
+        if (!mbar_wait(&full[stage], phase, abort_flag, err)) break;
+        tc_fence_after();
+        uint8_t *st = smem + stage * L::kStage;
+        const uint64_t a0 = desc_sw128_kmajor(smem_u32(st));
+        const uint64_t b0 = desc_sw128_kmajor(smem_u32(st + L::kW));
+#pragma unroll
+        for (int k = 0; k < kBK / 32; ++k)
+          umma_i8(tmem_base, a0 + 2 * k, b0 + 2 * k, idesc, (i != 0 || k != 0) ? 1u : 0u);
+        umma_commit(&empty[stage]);
+        if (++stage == L::kStages) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+      umma_commit(tfull);  // also arrives when no MMA was issued
+      umma_commit(drain);
+      mbar_wait(drain, 0, nullptr, err);
+    }
+    __syncwarp();
+  }
+
+  // ---- epilogue: accumulator -> registers -> (shared memory) ----
+  const bool epi = warp >= 2;
+  const int q = warp & 3;
+  const int row = q * 32 + lane;  // 0..127 for the epilogue warps
+  bool ok = true;
+  if (epi) ok = mbar_wait(tfull, 0, abort_flag, err);
+  ok = __syncthreads_and(ok);  // every thread of the CTA takes the same path
+  const bool whole = S == 1;
+  if (ok && epi) {
+    tc_fence_after();
+    const int n = tile * kDecRows + row;
+    const bool n_ok = n < N;
+    const float dw = (KIND != OutKind::I32 && n_ok) ? __ldg(w_scale + n) : 0.0f;
+    const bool have = kb1 > kb0;  // a CTA without k-blocks contributes zeros
+#pragma unroll
+    for (int c = 0; c < MP / 16; ++c) {
+      uint32_t r[16];
+      tmem_ld16(tmem_base + ((uint32_t)(q * 32) << 16) + c * 16, r);
+      tmem_ld_wait();
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const int t = c * 16 + j;
+        const int32_t v = have ? (int32_t)r[j] : 0;
+        if (whole) {
+          if (t < M && n_ok) {
+            const float dx = KIND != OutKind::I32 ? __ldg(x_scale + t) : 0.0f;
+            store_one<KIND>(y, ldy, t, n, v, dx, dw);
+          }
+        } else {
+          part[t * kDecRows + row] = v;
+        }
+      }
+    }
+  }
+  if (!whole) {
+    // partials of all S CTAs in place (and visible cluster-wide)
+    cluster_sync();
+    if (ok && epi) {
+      const int rows_per = kDecRows / S;
+      const int items = rows_per * M;
+      const uint32_t part_addr = smem_u32(part);
+      // 4 (token, row) items per round: their remote loads for each peer are
+      // issued together, so a round costs about one latency per peer
+      for (int base = threadIdx.x - 64; base < items; base += 4 * 128) {
+        uint32_t off[4];
+        int32_t sum[4] = {0, 0, 0, 0};
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+          const int idx = base + b * 128;
+          const int t = idx / rows_per, rr = (int)rank * rows_per + idx % rows_per;
+          off[b] = part_addr + (uint32_t)(t * kDecRows + rr) * 4u;
+        }
+#pragma unroll 1
+        for (int p = 0; p < S; ++p) {
+#pragma unroll
+          for (int b = 0; b < 4; ++b)
+            if (base + b * 128 < items) sum[b] += (int32_t)ld_shared_cluster_u32(mapa_shared(off[b], (uint32_t)p));
+        }
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+          const int idx = base + b * 128;
+          if (idx < items) {
+            const int t = idx / rows_per, rr = (int)rank * rows_per + idx % rows_per;
+            const int n = tile * kDecRows + rr;
+            if (n < N) {
+              const float dx = KIND != OutKind::I32 ? __ldg(x_scale + t) : 0.0f;
+              const float dw = KIND != OutKind::I32 ? __ldg(w_scale + n) : 0.0f;
+              store_one<KIND>(y, ldy, t, n, sum[b], dx, dw);
+            }
+          }
+        }
+      }
+    }
+    cluster_sync();  // no CTA leaves while a peer still reads its partial
+  }
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -724,8 +940,8 @@ cudaError_t launch_tc(const CUtensorMap &tmA, const CUtensorMap &tmB, const floa
   }
   const int tiles = ((M + kBM - 1) / kBM) * ((N + BN - 1) / BN);
   const int grid = tiles < num_sms() ? tiles : num_sms();
-  kern<<<grid, kThreads, L::kTotal, st>>>(tmA, tmB, x_scale, w_scale, y, ldy, M, N, K, device_error_word());
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3(grid), dim3(kThreads), L::kTotal, st, 1, tmA, tmB, x_scale, w_scale, y, ldy, M, N, K,
+                    device_error_word());
 }
 
 template <int STAGES, OutKind KIND>
@@ -735,21 +951,8 @@ cudaError_t launch_pair(const CUtensorMap &tmA, const CUtensorMap &tmB, const fl
   auto kern = w8a8_gemm_pair_kernel<STAGES, KIND>;
   const int tiles = ((M + 2 * kBM - 1) / (2 * kBM)) * ((N + kPairBN - 1) / kPairBN);
   const int clusters = tiles < max_clusters ? tiles : max_clusters;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(2 * clusters, 1, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = L::kTotal;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tmA, tmB, x_scale, w_scale, y, ldy, M, N, K, device_error_word());
-  if (e != cudaSuccess) return e;
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3(2 * clusters), dim3(kThreads), L::kTotal, st, 2, tmA, tmB, x_scale, w_scale, y, ldy, M,
+                    N, K, device_error_word());
 }
 
 // Clusters of two 1-CTA-per-SM blocks that fit on the device at once.
@@ -782,7 +985,65 @@ int pair_capacity() {
   return c;
 }
 
-constexpr int kPairStages = 6;
+constexpr int kPairStages = 7;
+
+template <int MP, OutKind KIND>
+void prepare_decode_cluster_kernel() {
+  using L = DecSmem<MP>;
+  static bool done[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (!done[dev & 63]) {
+    auto kern = w8a8_gemm_decode_cluster_kernel<MP, KIND>;
+    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::kTotal);
+    cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    done[dev & 63] = true;
+  }
+}
+
+// Clusters of S one-CTA-per-SM blocks of the decode cluster kernel that can
+// be resident at once (0 if none or the query fails).
+template <int MP, OutKind KIND>
+int cluster_capacity(int S) {
+  using L = DecSmem<MP>;
+  static int cache[64][5] = {};  // [device][log2 S]
+  int dev = 0;
+  cudaGetDevice(&dev);
+  int lg = 0;
+  while ((1 << lg) < S) ++lg;
+  int &c = cache[dev & 63][lg];
+  if (c == 0) {
+    prepare_decode_cluster_kernel<MP, KIND>();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(S, 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = L::kTotal;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = S;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, w8a8_gemm_decode_cluster_kernel<MP, KIND>, &cfg) != cudaSuccess) {
+      cudaGetLastError();  // clear the query's error
+      n = -1;
+    }
+    c = n > 0 ? n : -1;
+  }
+  return c > 0 ? c : 0;
+}
+
+template <int MP, OutKind KIND>
+cudaError_t launch_decode_cluster(const CUtensorMap &tmW, const CUtensorMap &tmX, const float *x_scale,
+                                  const float *w_scale, int M, int N, int K, void *y, int64_t ldy, int nt, int S,
+                                  cudaStream_t st) {
+  using L = DecSmem<MP>;
+  prepare_decode_cluster_kernel<MP, KIND>();
+  return launch_pdl(w8a8_gemm_decode_cluster_kernel<MP, KIND>, dim3(nt * S), dim3(kThreads), L::kTotal, st,
+                    (unsigned)S, tmW, tmX, x_scale, w_scale, y, ldy, M, N, K, S, device_error_word());
+}
 
 template <int MP, OutKind KIND>
 cudaError_t launch_decode(const int8_t *xq, const float *x_scale, const int8_t *wq, const float *w_scale, int M,
@@ -800,13 +1061,20 @@ cudaError_t launch_decode(const int8_t *xq, const float *x_scale, const int8_t *
   CUtensorMap tmW, tmX;
   if (!make_tmap_i8(&tmW, wq, N, K, kDecRows)) return cudaErrorInvalidValue;
   if (!make_tmap_i8(&tmX, xq, M, K, MP)) return cudaErrorInvalidValue;
-  const int64_t items = (int64_t)((N + kDecRows - 1) / kDecRows) * ((K + kBK - 1) / kBK);
+  const int nt = (N + kDecRows - 1) / kDecRows, nk = (K + kBK - 1) / kBK;
+  if (nt <= num_sms()) {
+    // one wave of tiles: split K across a cluster of S CTAs per tile
+    int S = 1;
+    for (int cand = 2; cand <= 16; cand *= 2)
+      if (cand <= nk && (int64_t)nt * cand <= num_sms() && cluster_capacity<MP, KIND>(cand) >= nt) S = cand;
+    return launch_decode_cluster<MP, KIND>(tmW, tmX, x_scale, w_scale, M, N, K, y, ldy, nt, S, st);
+  }
+  const int64_t items = (int64_t)nt * nk;
   const int grid = (int)(items < num_sms() ? items : num_sms());
   int32_t *ws = static_cast<int32_t *>(workspace);
   unsigned *counts = reinterpret_cast<unsigned *>(static_cast<uint8_t *>(workspace) + decode_ws_elems(M, N) * 4);
-  kern<<<grid, kThreads, L::kTotal, st>>>(tmW, tmX, x_scale, w_scale, y, ldy, M, N, K, ws, counts,
-                                          device_error_word());
-  return cudaGetLastError();
+return launch_pdl(kern, dim3(grid), dim3(kThreads), L::kTotal, st, 1, tmW, tmX, x_scale, w_scale, y, ldy, M, N, K,
+                    ws, counts, device_error_word());
 }
 
 template <OutKind KIND>

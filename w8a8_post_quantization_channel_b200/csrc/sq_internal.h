@@ -14,12 +14,17 @@ int num_sms();
 // Address of the current device's error word (cached per device).
 unsigned *device_error_word();
 
+
 // amax[c] = max(amax[c], max_r |x[r][c]| (* row_scale[r] when given)).
+// keep_in_l2: x is read again by the next kernel (weights), so its lines
+// are loaded with evict-last priority; otherwise evict-first.
 cudaError_t launch_absmax_cols(const void *x, sq_dtype xt, int64_t rows, int64_t cols, int64_t ld,
-                               const float *row_scale, float *amax, cudaStream_t st);
+                               const float *row_scale, float *amax, bool keep_in_l2, cudaStream_t st);
 // out[r] = max_c |x[r][c]|.
 cudaError_t launch_absmax_rows(const void *x, sq_dtype xt, int64_t rows, int64_t cols, int64_t ld, float *out,
                                cudaStream_t st);
+// p[0..n) = 0 (a kernel, so that it chains with its neighbours).
+cudaError_t launch_zero_fill(float *p, int64_t n, cudaStream_t st);
 // s[j] (holding w_j on entry) <- s_j, inv_s[j] <- 1/s_j from amax[j], w_j.
 cudaError_t launch_smooth_factor(const float *amax, float *s_inout, float *inv_s, int64_t K, float alpha,
                                  cudaStream_t st);

@@ -7,8 +7,10 @@ of the workloads' shapes, for profilers and roofline measurements.
 
 --op is calib (T = M tokens), weight (W [N, K]), act or linear.  With
 --time (implied by --sweep) every iteration is timed with CUDA events on
-the launching stream, a 512 MB buffer is rewritten between iterations so
-that L2 (126 MB) holds none of the operands, and the median is reported
+the launching stream, a 512 MB buffer is read between iterations so that
+L2 (126 MB) holds none of the operands (a read leaves clean lines behind, so
+the timed kernel pays no write-back of someone else's dirty data), and the
+median is reported
 against the measured peaks: algorithmic bytes / time against HBM for calib,
 act, weight and decode-shaped linears (M <= 64: streaming Wq dominates),
 2MNK / time against the INT8 tensor peak (2 x measured bf16) otherwise.
@@ -95,12 +97,12 @@ def make_case(op, M, K, N, dtype, dev="cuda"):
 
 def time_case(op, M, K, N, dtype, iters):
     fn, nbytes, ops = make_case(op, M, K, N, dtype)
-    flush = torch.empty(512 * 2 ** 20, dtype=torch.uint8, device="cuda")
+    flush = torch.ones(128 * 2 ** 20, dtype=torch.float32, device="cuda")  # 512 MB
     fn()
     torch.cuda.synchronize()
     times = []
     for i in range(iters):
-        flush.fill_(i & 0xFF)
+        flush.sum()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record()
         fn()
