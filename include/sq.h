@@ -184,6 +184,17 @@ sq_status sq_w8a8_linear_decode_noalloc(const int8_t *xq, const float *x_scale,
                                         sq_stream_t stream);
 
 /*
+ * Self-test of the failure path.  Launches one block whose thread waits on a
+ * shared-memory barrier that nothing ever arrives at; the wait gives up
+ * after `limit_ms` milliseconds (1..5000), records SQ_ERR_TIMEOUT in the
+ * device error word, and the kernel returns normally, so the device stays
+ * usable.  The next sq_check_device_error(stream) then reports
+ * SQ_ERR_TIMEOUT.  Every wait in the other kernels uses the same mechanism
+ * (with a 2 s limit).  Returns SQ_ERR_INVALID_ARG for a limit out of range.
+ */
+sq_status sq_selftest_wait_timeout(int limit_ms, sq_stream_t stream);
+
+/*
  * Synchronises `stream`, then reports (and clears) a timeout that any
  * kernel of this library recorded on the current device since the last
  * check: SQ_ERR_TIMEOUT, else SQ_OK (or SQ_ERR_CUDA if the sync failed).

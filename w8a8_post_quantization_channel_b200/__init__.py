@@ -33,7 +33,7 @@ __all__ = [
     "lib", "library_path", "header_functions",
     "sq_calib_absmax", "sq_smooth_quant_weight", "sq_quant_act", "sq_w8a8_linear",
     "sq_w8a8_linear_workspace_size", "sq_w8a8_accumulate", "sq_check_device_error", "sq_status_string",
-    "sq_w8a8_linear_decode_noalloc", "SQ_DECODE_STATIC_SCRATCH_BYTES",
+    "sq_w8a8_linear_decode_noalloc", "SQ_DECODE_STATIC_SCRATCH_BYTES", "sq_selftest_wait_timeout",
 ]
 
 SQ_OK, SQ_ERR_INVALID_ARG, SQ_ERR_UNSUPPORTED, SQ_ERR_CUDA, SQ_ERR_TIMEOUT = 0, 1, 2, 3, 4
@@ -79,6 +79,7 @@ def lib() -> ctypes.CDLL:
             "sq_w8a8_accumulate": [vp, vp, i64, i64, i64, vp, i64, vp, sz, vp],
             "sq_check_device_error": [vp],
             "sq_w8a8_linear_decode_noalloc": [vp, vp, vp, vp, i64, i64, i64, vp, i32, i64, vp],
+            "sq_selftest_wait_timeout": [i32, vp],
         }
         for name, args in sigs.items():
             fn = getattr(L, name)
@@ -222,6 +223,12 @@ def sq_w8a8_linear_decode_noalloc(xq: torch.Tensor, x_scale: torch.Tensor, wq: t
                                                _ptr(y), _dtype(y, "y"), y.stride(0), _stream(stream)),
            "sq_w8a8_linear_decode_noalloc")
     return y
+
+
+def sq_selftest_wait_timeout(limit_ms: int = 100, stream=None) -> int:
+    """Runs the bounded-wait self-test kernel (see include/sq.h); returns the
+    launch status.  Follow with sq_check_device_error()."""
+    return int(lib().sq_selftest_wait_timeout(int(limit_ms), _stream(stream)))
 
 
 def sq_check_device_error(stream=None) -> int:

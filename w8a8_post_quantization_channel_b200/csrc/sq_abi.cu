@@ -180,6 +180,11 @@ sq_status sq_w8a8_accumulate(const int8_t *xq, const int8_t *wq, int64_t M, int6
                                         workspace_bytes, (cudaStream_t)stream));
 }
 
+sq_status sq_selftest_wait_timeout(int limit_ms, sq_stream_t stream) {
+  if (limit_ms < 1 || limit_ms > 5000) return SQ_ERR_INVALID_ARG;
+  return from_cuda(sq::launch_wait_timeout_selftest((unsigned long long)limit_ms * 1000000ull, (cudaStream_t)stream));
+}
+
 sq_status sq_check_device_error(sq_stream_t stream) {
   if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return SQ_ERR_CUDA;
   unsigned *word = sq::device_error_word();

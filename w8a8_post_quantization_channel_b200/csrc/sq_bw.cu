@@ -457,6 +457,18 @@ __global__ void zero_fill_kernel(float *__restrict__ p, int64_t n) {
     p[i] = 0.0f;
 }
 
+// One thread waits on a barrier that nothing arrives at: the bounded wait
+// gives up after limit_ns and records the timeout (self-test of the path
+// every other kernel takes when a wait runs out).
+__global__ void wait_timeout_selftest_kernel(unsigned long long limit_ns, unsigned *err) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+    mbar_wait(&bar, 0, nullptr, err, limit_ns);
+  }
+}
+
 template <typename T>
 cudaError_t absmax_cols_t(const void *x, int64_t rows, int64_t cols, int64_t ld, const float *row_scale,
                           float *amax, bool keep_in_l2, cudaStream_t st) {
@@ -576,6 +588,11 @@ cudaError_t launch_absmax_rows(const void *x, sq_dtype xt, int64_t rows, int64_t
     case SQ_F16: return absmax_rows_t<__half>(x, rows, cols, ld, out, st);
     default: return absmax_rows_t<__nv_bfloat16>(x, rows, cols, ld, out, st);
   }
+}
+
+cudaError_t launch_wait_timeout_selftest(unsigned long long limit_ns, cudaStream_t st) {
+  wait_timeout_selftest_kernel<<<1, 32, 0, st>>>(limit_ns, device_error_word());
+  return cudaGetLastError();
 }
 
 cudaError_t launch_zero_fill(float *p, int64_t n, cudaStream_t st) {

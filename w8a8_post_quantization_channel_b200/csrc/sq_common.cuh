@@ -232,7 +232,8 @@ __device__ __forceinline__ unsigned long long globaltimer_ns() {
 // false, without waiting further, once *abort is set by another role or
 // after kWaitLimitNs; on the timeout it records kDevErrTimeout in *err and
 // raises *abort for the rest of the block.  `abort` may be null.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort, unsigned *err) {
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort, unsigned *err,
+                                          unsigned long long limit_ns = kWaitLimitNs) {
   const uint32_t a = smem_u32(bar);
   if (mbar_try_wait(a, parity)) return true;
   const unsigned long long t0 = globaltimer_ns();
@@ -240,7 +241,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
     if (mbar_try_wait(a, parity)) return true;
     if ((it & 15u) == 0) {
       if (abort != nullptr && *abort) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      if (globaltimer_ns() - t0 > limit_ns) {
         atomicOr(err, kDevErrTimeout);
         if (abort != nullptr) *abort = 1;
         return false;

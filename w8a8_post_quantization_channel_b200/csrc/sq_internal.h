@@ -23,6 +23,8 @@ cudaError_t launch_absmax_cols(const void *x, sq_dtype xt, int64_t rows, int64_t
 // out[r] = max_c |x[r][c]|.
 cudaError_t launch_absmax_rows(const void *x, sq_dtype xt, int64_t rows, int64_t cols, int64_t ld, float *out,
                                cudaStream_t st);
+// One block waits on a barrier nobody arrives at, up to limit_ns.
+cudaError_t launch_wait_timeout_selftest(unsigned long long limit_ns, cudaStream_t st);
 // p[0..n) = 0 (a kernel, so that it chains with its neighbours).
 cudaError_t launch_zero_fill(float *p, int64_t n, cudaStream_t st);
 // s[j] (holding w_j on entry) <- s_j, inv_s[j] <- 1/s_j from amax[j], w_j.
