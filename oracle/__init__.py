@@ -68,6 +68,10 @@ def _load():
             "or_dequant": ([i32p, f32p, f32p, i64, i64, f32p], None),
             "or_round_bf16": ([f32p, i64, u16p], None),
             "or_round_f16": ([f32p, i64, u16p], None),
+            "or_rmsnorm_quant_act": ([f32p, i64, i64, f32p, ctypes.c_float, f32p, i8p, f32p], None),
+            "or_rmsnorm_factor": ([f32p, i64, i64, ctypes.c_float, f32p], None),
+            "or_static_act_scale": ([f32p, f32p, i64], ctypes.c_float),
+            "or_quant_act_static": ([f32p, i64, i64, f32p, ctypes.c_float, i8p, f32p], None),
         }
         for name, (args, res) in sig.items():
             fn = getattr(lib, name)
@@ -206,6 +210,49 @@ def round_to(y, dtype: str) -> np.ndarray:
         raise ValueError(dtype)
     fn(_ptr(y, ctypes.c_float), y.size, _ptr(out, ctypes.c_uint16))
     return out
+
+
+def rmsnorm_quant_act(x, gamma, eps: float, inv_s):
+    """(Xq, dx): RMSNorm (weight gamma, epsilon eps) folded with X diag(s)^-1,
+    then per-token quantization."""
+    x = _f32(x)
+    gamma = _f32(gamma)
+    inv_s = _f32(inv_s)
+    M, K = x.shape
+    xq = np.zeros((M, K), np.int8)
+    dx = np.zeros(M, np.float32)
+    _load().or_rmsnorm_quant_act(_ptr(x, ctypes.c_float), M, K, _ptr(gamma, ctypes.c_float), ctypes.c_float(eps),
+                                 _ptr(inv_s, ctypes.c_float), _ptr(xq, ctypes.c_int8), _ptr(dx, ctypes.c_float))
+    return xq, dx
+
+
+def rmsnorm_factor(x, eps: float) -> np.ndarray:
+    """Per-token r_t = 1 / sqrt(mean_j x_tj^2 + eps), rounded once to fp32."""
+    x = _f32(x)
+    M, K = x.shape
+    r = np.zeros(M, np.float32)
+    _load().or_rmsnorm_factor(_ptr(x, ctypes.c_float), M, K, ctypes.c_float(eps), _ptr(r, ctypes.c_float))
+    return r
+
+
+def static_act_scale(amax, inv_s) -> float:
+    """Per-tensor scale max_j(a_j * inv_s_j) / 127 from calibration maxima."""
+    amax = _f32(amax)
+    inv_s = _f32(inv_s)
+    return float(_load().or_static_act_scale(_ptr(amax, ctypes.c_float), _ptr(inv_s, ctypes.c_float),
+                                             amax.shape[0]))
+
+
+def quant_act_static(x, inv_s, delta: float):
+    """(Xq, dx): smoothing then quantization with one fixed scale delta."""
+    x = _f32(x)
+    inv_s = _f32(inv_s)
+    M, K = x.shape
+    xq = np.zeros((M, K), np.int8)
+    dx = np.zeros(M, np.float32)
+    _load().or_quant_act_static(_ptr(x, ctypes.c_float), M, K, _ptr(inv_s, ctypes.c_float), ctypes.c_float(delta),
+                                _ptr(xq, ctypes.c_int8), _ptr(dx, ctypes.c_float))
+    return xq, dx
 
 
 def linear(x, inv_s, wq, dw, out_dtype: str = "f32"):

@@ -229,3 +229,69 @@ void or_round_f16(const float *y, int64_t count, uint16_t *out) {
     memcpy(&out[i], &h, 2);
   }
 }
+
+/* ---- upstream producer: RMSNorm, smoothing and per-token quantization ----
+ * The usage example's smooth_lm(alpha) folds diag(s)^-1 into the layer that
+ * produces X, in transformer blocks an RMS normalisation.  For token t:
+ *   ss_t = sum_j x_tj^2            (double precision, sequential)
+ *   r_t  = (float)(1 / sqrt(ss_t / K + eps))   (double, rounded once)
+ *   v_tj = ((x_tj * r_t) * gamma_j) * inv_s_j  (fp32, in that order)
+ * then v is quantized per token as in or_quant_act. */
+void or_rmsnorm_quant_act(const float *x, int64_t M, int64_t K, const float *gamma, float eps,
+                          const float *inv_s, int8_t *xq, float *dx) {
+  for (int64_t t = 0; t < M; ++t) {
+    double ss = 0.0;
+    for (int64_t j = 0; j < K; ++j) ss += (double)x[t * K + j] * (double)x[t * K + j];
+    const float r = (float)(1.0 / sqrt(ss / (double)K + (double)eps));
+    float m = 0.0f;
+    for (int64_t j = 0; j < K; ++j) {
+      float v = fabsf(((x[t * K + j] * r) * gamma[j]) * inv_s[j]);
+      if (v > m) m = v;
+    }
+    if (m == 0.0f) {
+      dx[t] = 0.0f;
+      for (int64_t j = 0; j < K; ++j) xq[t * K + j] = 0;
+      continue;
+    }
+    dx[t] = m / 127.0f;
+    float rq = 127.0f / m;
+    for (int64_t j = 0; j < K; ++j)
+      xq[t * K + j] = or_quantize_value(((x[t * K + j] * r) * gamma[j]) * inv_s[j], rq);
+  }
+}
+
+/* Per-token normalisation factor r_t of or_rmsnorm_quant_act (exposed so
+ * tests can see how close a product lies to a rounding boundary). */
+void or_rmsnorm_factor(const float *x, int64_t M, int64_t K, float eps, float *r) {
+  for (int64_t t = 0; t < M; ++t) {
+    double ss = 0.0;
+    for (int64_t j = 0; j < K; ++j) ss += (double)x[t * K + j] * (double)x[t * K + j];
+    r[t] = (float)(1.0 / sqrt(ss / (double)K + (double)eps));
+  }
+}
+
+/* ---- static per-tensor activation scale --------------------------------
+ * The page notes activations change per prompt, which is why the main path
+ * quantizes per token at run time; the static alternative fixes one scale
+ * from calibration.  After smoothing, channel j's calibrated maximum is
+ * a_j * inv_s_j, so the tensor scale is delta = max_j(a_j * inv_s_j) / 127. */
+float or_static_act_scale(const float *amax, const float *inv_s, int64_t K) {
+  float m = 0.0f;
+  for (int64_t j = 0; j < K; ++j) {
+    float v = amax[j] * inv_s[j];
+    if (v > m) m = v;
+  }
+  return m / 127.0f;
+}
+
+/* Static quantization with a fixed scale delta > 0: every token is scaled
+ * by r = 1 / delta (one IEEE division) and rounded; values beyond the
+ * calibrated range saturate at +-127.  dx_t = delta for every token. */
+void or_quant_act_static(const float *x, int64_t M, int64_t K, const float *inv_s, float delta,
+                         int8_t *xq, float *dx) {
+  const float r = 1.0f / delta;
+  for (int64_t t = 0; t < M; ++t) {
+    dx[t] = delta;
+    for (int64_t j = 0; j < K; ++j) xq[t * K + j] = or_quantize_value(x[t * K + j] * inv_s[j], r);
+  }
+}

@@ -319,3 +319,65 @@ def test_output_rounding_matches_library_conversions():
     np.testing.assert_array_equal(bf, ref_bf)
     h = oracle.round_to(y, "f16")
     np.testing.assert_array_equal(h, y.astype(np.float16).view(np.uint16))
+
+
+# ---------------------------------------------------------------------------
+# upstream producer: RMSNorm folded with X diag(s)^-1, and the static scale
+# ---------------------------------------------------------------------------
+
+def test_rmsnorm_factor_matches_library_rms_norm():
+    rng = np.random.default_rng(21)
+    x = rng.standard_normal((9, 320)).astype(np.float32)
+    x[:, 5] *= 80
+    eps = 1e-5
+    r = oracle.rmsnorm_factor(x, eps)
+    xt = torch.from_numpy(x.astype(np.float64))
+    normed = torch.nn.functional.rms_norm(xt, (320,), eps=eps)  # x / sqrt(mean(x^2) + eps)
+    r_lib = (normed / xt)[:, 0].numpy()
+    assert _ulps(r, r_lib).max() <= 1
+
+
+@pytest.mark.parametrize("dt", [np.float32, np.float16])
+def test_rmsnorm_quant_power_of_two_identity(dt):
+    # rows with mean(x^2) = 4 exactly (and eps = 0) have r = 1/2 exactly, so
+    # ((x r) gamma) inv_s = ((x gamma) inv_s) / 2 with no extra rounding:
+    # the codes equal plain per-token quantization of x * gamma, and the
+    # scale halves.  This fixes that gamma and inv_s act per column and r
+    # per row.
+    rng = np.random.default_rng(22)
+    base = np.array([7, 3, 1, 1, 1, 1, 1, 1] + [0] * 8, np.float32)  # sum of squares 64, K = 16
+    rows = []
+    for _ in range(6):
+        rows.append(base[rng.permutation(16)] * rng.choice([-1.0, 1.0], 16).astype(np.float32))
+    x = np.stack(rows).astype(dt).astype(np.float32)
+    gamma = np.exp(rng.uniform(-1, 1, 16)).astype(np.float32)
+    inv_s = np.exp(rng.uniform(-2, 2, 16)).astype(np.float32)
+    np.testing.assert_array_equal(oracle.rmsnorm_factor(x, 0.0), 0.5)
+    xq, dx = oracle.rmsnorm_quant_act(x, gamma, 0.0, inv_s)
+    xg = (x * gamma).astype(np.float32)
+    xq_plain, dx_plain = oracle.quant_act(xg, inv_s)
+    np.testing.assert_array_equal(xq, xq_plain)
+    np.testing.assert_array_equal(dx, dx_plain * np.float32(0.5))
+
+
+def test_rmsnorm_quant_scale_invariance():
+    # per-token quantization after RMSNorm ignores a power-of-two rescaling
+    # of the token (eps = 0): r absorbs it exactly
+    rng = np.random.default_rng(23)
+    x = rng.standard_normal((5, 96)).astype(np.float32)
+    gamma = rng.uniform(0.5, 2, 96).astype(np.float32)
+    inv_s = rng.uniform(0.1, 3, 96).astype(np.float32)
+    a = oracle.rmsnorm_quant_act(x, gamma, 0.0, inv_s)
+    b = oracle.rmsnorm_quant_act(x * np.float32(8.0), gamma, 0.0, inv_s)
+    np.testing.assert_array_equal(a[0], b[0])
+    np.testing.assert_array_equal(a[1], b[1])
+
+
+def test_p7_static_scale_and_saturation():
+    g = load("p7_static_scale.txt")
+    delta = oracle.static_act_scale(_fl(g["amax"]), _fl(g["inv_s_scale"]))
+    assert delta == np.float32(np.float32(float(g["delta_num"][0])) / np.float32(127))
+    x = _fl(g["x"]).astype(np.float32)[None, :]
+    xq, dx = oracle.quant_act_static(x, np.ones(x.shape[1], np.float32), float(g["delta"][0]))
+    np.testing.assert_array_equal(xq[0], _int(g["xq"]))
+    assert dx[0] == np.float32(float(g["delta"][0]))
