@@ -68,7 +68,8 @@ def _load():
             "or_dequant": ([i32p, f32p, f32p, i64, i64, f32p], None),
             "or_round_bf16": ([f32p, i64, u16p], None),
             "or_round_f16": ([f32p, i64, u16p], None),
-            "or_rmsnorm_quant_act": ([f32p, i64, i64, f32p, ctypes.c_float, f32p, i8p, f32p], None),
+            "or_fold_norm_weight": ([f32p, f32p, i64, f32p], None),
+            "or_rmsnorm_quant_act": ([f32p, i64, i64, f32p, ctypes.c_float, i8p, f32p], None),
             "or_rmsnorm_factor": ([f32p, i64, i64, ctypes.c_float, f32p], None),
             "or_static_act_scale": ([f32p, f32p, i64], ctypes.c_float),
             "or_quant_act_static": ([f32p, i64, i64, f32p, ctypes.c_float, i8p, f32p], None),
@@ -212,17 +213,26 @@ def round_to(y, dtype: str) -> np.ndarray:
     return out
 
 
-def rmsnorm_quant_act(x, gamma, eps: float, inv_s):
-    """(Xq, dx): RMSNorm (weight gamma, epsilon eps) folded with X diag(s)^-1,
-    then per-token quantization."""
-    x = _f32(x)
+def fold_norm_weight(gamma, inv_s) -> np.ndarray:
+    """gs_j = gamma_j * inv_s_j: diag(s)^-1 folded into the norm's weight."""
     gamma = _f32(gamma)
     inv_s = _f32(inv_s)
+    gs = np.zeros(gamma.shape[0], np.float32)
+    _load().or_fold_norm_weight(_ptr(gamma, ctypes.c_float), _ptr(inv_s, ctypes.c_float), gamma.shape[0],
+                                _ptr(gs, ctypes.c_float))
+    return gs
+
+
+def rmsnorm_quant_act(x, gs, eps: float):
+    """(Xq, dx): RMSNorm (epsilon eps) with the folded weight gs, then
+    per-token quantization."""
+    x = _f32(x)
+    gs = _f32(gs)
     M, K = x.shape
     xq = np.zeros((M, K), np.int8)
     dx = np.zeros(M, np.float32)
-    _load().or_rmsnorm_quant_act(_ptr(x, ctypes.c_float), M, K, _ptr(gamma, ctypes.c_float), ctypes.c_float(eps),
-                                 _ptr(inv_s, ctypes.c_float), _ptr(xq, ctypes.c_int8), _ptr(dx, ctypes.c_float))
+    _load().or_rmsnorm_quant_act(_ptr(x, ctypes.c_float), M, K, _ptr(gs, ctypes.c_float), ctypes.c_float(eps),
+                                 _ptr(xq, ctypes.c_int8), _ptr(dx, ctypes.c_float))
     return xq, dx
 
 

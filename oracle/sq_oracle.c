@@ -232,20 +232,27 @@ void or_round_f16(const float *y, int64_t count, uint16_t *out) {
 
 /* ---- upstream producer: RMSNorm, smoothing and per-token quantization ----
  * The usage example's smooth_lm(alpha) folds diag(s)^-1 into the layer that
- * produces X, in transformer blocks an RMS normalisation.  For token t:
+ * produces X -- in transformer blocks an RMS normalisation -- offline, the
+ * same way diag(s) is folded into W.  The norm's weight becomes
+ *   gs_j = gamma_j * inv_s_j                     (fp32, once per layer)
+ * and for token t the producer computes
  *   ss_t = sum_j x_tj^2            (double precision, sequential)
  *   r_t  = (float)(1 / sqrt(ss_t / K + eps))   (double, rounded once)
- *   v_tj = ((x_tj * r_t) * gamma_j) * inv_s_j  (fp32, in that order)
- * then v is quantized per token as in or_quant_act. */
-void or_rmsnorm_quant_act(const float *x, int64_t M, int64_t K, const float *gamma, float eps,
-                          const float *inv_s, int8_t *xq, float *dx) {
+ *   v_tj = (x_tj * r_t) * gs_j                 (fp32, in that order)
+ * then quantizes v per token as in or_quant_act. */
+void or_fold_norm_weight(const float *gamma, const float *inv_s, int64_t K, float *gs) {
+  for (int64_t j = 0; j < K; ++j) gs[j] = gamma[j] * inv_s[j];
+}
+
+void or_rmsnorm_quant_act(const float *x, int64_t M, int64_t K, const float *gs, float eps, int8_t *xq,
+                          float *dx) {
   for (int64_t t = 0; t < M; ++t) {
     double ss = 0.0;
     for (int64_t j = 0; j < K; ++j) ss += (double)x[t * K + j] * (double)x[t * K + j];
     const float r = (float)(1.0 / sqrt(ss / (double)K + (double)eps));
     float m = 0.0f;
     for (int64_t j = 0; j < K; ++j) {
-      float v = fabsf(((x[t * K + j] * r) * gamma[j]) * inv_s[j]);
+      float v = fabsf((x[t * K + j] * r) * gs[j]);
       if (v > m) m = v;
     }
     if (m == 0.0f) {
@@ -255,8 +262,7 @@ void or_rmsnorm_quant_act(const float *x, int64_t M, int64_t K, const float *gam
     }
     dx[t] = m / 127.0f;
     float rq = 127.0f / m;
-    for (int64_t j = 0; j < K; ++j)
-      xq[t * K + j] = or_quantize_value(((x[t * K + j] * r) * gamma[j]) * inv_s[j], rq);
+    for (int64_t j = 0; j < K; ++j) xq[t * K + j] = or_quantize_value((x[t * K + j] * r) * gs[j], rq);
   }
 }
 

@@ -340,10 +340,9 @@ def test_rmsnorm_factor_matches_library_rms_norm():
 @pytest.mark.parametrize("dt", [np.float32, np.float16])
 def test_rmsnorm_quant_power_of_two_identity(dt):
     # rows with mean(x^2) = 4 exactly (and eps = 0) have r = 1/2 exactly, so
-    # ((x r) gamma) inv_s = ((x gamma) inv_s) / 2 with no extra rounding:
-    # the codes equal plain per-token quantization of x * gamma, and the
-    # scale halves.  This fixes that gamma and inv_s act per column and r
-    # per row.
+    # (x r) gs = (x gs) / 2 with no extra rounding: the codes equal plain
+    # per-token quantization of x with column scales gs, and the scale
+    # halves.  This fixes that gs acts per column and r per row.
     rng = np.random.default_rng(22)
     base = np.array([7, 3, 1, 1, 1, 1, 1, 1] + [0] * 8, np.float32)  # sum of squares 64, K = 16
     rows = []
@@ -352,12 +351,35 @@ def test_rmsnorm_quant_power_of_two_identity(dt):
     x = np.stack(rows).astype(dt).astype(np.float32)
     gamma = np.exp(rng.uniform(-1, 1, 16)).astype(np.float32)
     inv_s = np.exp(rng.uniform(-2, 2, 16)).astype(np.float32)
+    gs = oracle.fold_norm_weight(gamma, inv_s)
     np.testing.assert_array_equal(oracle.rmsnorm_factor(x, 0.0), 0.5)
-    xq, dx = oracle.rmsnorm_quant_act(x, gamma, 0.0, inv_s)
-    xg = (x * gamma).astype(np.float32)
-    xq_plain, dx_plain = oracle.quant_act(xg, inv_s)
+    xq, dx = oracle.rmsnorm_quant_act(x, gs, 0.0)
+    xq_plain, dx_plain = oracle.quant_act(x, gs)
     np.testing.assert_array_equal(xq, xq_plain)
     np.testing.assert_array_equal(dx, dx_plain * np.float32(0.5))
+
+
+def test_folded_norm_equals_norm_then_smoothing():
+    # with inv_s a power of two per channel, folding it into the norm weight
+    # changes no rounding: ((x r) gamma) inv_s == (x r)(gamma inv_s) exactly.
+    # So the folded producer must equal the unfolded sequence -- normalise,
+    # apply gamma, then X diag(s)^-1 and per-token quantization.  A fold that
+    # used s instead of 1/s, or dropped gamma, fails here.
+    rng = np.random.default_rng(24)
+    K = 64
+    x = rng.standard_normal((7, K)).astype(np.float32)
+    x[:, 3] *= 40
+    gamma = rng.uniform(0.2, 3.0, K).astype(np.float32)
+    inv_s = np.float32(2.0) ** rng.integers(-6, 7, K).astype(np.float32)
+    eps = 1e-5
+    gs = oracle.fold_norm_weight(gamma, inv_s)
+    xq, dx = oracle.rmsnorm_quant_act(x, gs, eps)
+    r = oracle.rmsnorm_factor(x, eps)
+    normed = ((x * r[:, None]).astype(np.float32) * gamma).astype(np.float32)
+    xq_u, dx_u = oracle.quant_act(normed, inv_s)
+    np.testing.assert_array_equal(xq, xq_u)
+    np.testing.assert_array_equal(dx, dx_u)
+    assert not np.array_equal(xq, oracle.rmsnorm_quant_act(x, oracle.fold_norm_weight(gamma, 1 / inv_s), eps)[0])
 
 
 def test_rmsnorm_quant_scale_invariance():
@@ -365,10 +387,9 @@ def test_rmsnorm_quant_scale_invariance():
     # of the token (eps = 0): r absorbs it exactly
     rng = np.random.default_rng(23)
     x = rng.standard_normal((5, 96)).astype(np.float32)
-    gamma = rng.uniform(0.5, 2, 96).astype(np.float32)
-    inv_s = rng.uniform(0.1, 3, 96).astype(np.float32)
-    a = oracle.rmsnorm_quant_act(x, gamma, 0.0, inv_s)
-    b = oracle.rmsnorm_quant_act(x * np.float32(8.0), gamma, 0.0, inv_s)
+    gs = oracle.fold_norm_weight(rng.uniform(0.5, 2, 96), rng.uniform(0.1, 3, 96))
+    a = oracle.rmsnorm_quant_act(x, gs, 0.0)
+    b = oracle.rmsnorm_quant_act(x * np.float32(8.0), gs, 0.0)
     np.testing.assert_array_equal(a[0], b[0])
     np.testing.assert_array_equal(a[1], b[1])
 
