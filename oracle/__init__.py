@@ -54,6 +54,8 @@ def _load():
         i8p = ctypes.POINTER(ctypes.c_int8)
         i32p = ctypes.POINTER(ctypes.c_int32)
         u16p = ctypes.POINTER(ctypes.c_uint16)
+        u8p = ctypes.POINTER(ctypes.c_uint8)
+        f64p = ctypes.POINTER(ctypes.c_double)
         i64 = ctypes.c_int64
         sig = {
             "or_quantize_value": ([ctypes.c_float, ctypes.c_float], ctypes.c_int8),
@@ -73,6 +75,12 @@ def _load():
             "or_rmsnorm_factor": ([f32p, i64, i64, ctypes.c_float, f32p], None),
             "or_static_act_scale": ([f32p, f32p, i64], ctypes.c_float),
             "or_quant_act_static": ([f32p, i64, i64, f32p, ctypes.c_float, i8p, f32p], None),
+            "or_e4m3_decode": ([ctypes.c_uint8], ctypes.c_float),
+            "or_e4m3_encode": ([ctypes.c_float], ctypes.c_uint8),
+            "or_smooth_quant_weight_e4m3": ([f32p, ctypes.c_int, i64, i64, f32p, u8p, f32p], None),
+            "or_quant_act_e4m3": ([f32p, i64, i64, f32p, u8p, f32p], None),
+            "or_gemm_e4m3": ([u8p, u8p, i64, i64, i64, f64p], None),
+            "or_dequant_f32acc": ([f32p, f32p, f32p, i64, i64, f32p], None),
         }
         for name, (args, res) in sig.items():
             fn = getattr(lib, name)
@@ -263,6 +271,72 @@ def quant_act_static(x, inv_s, delta: float):
     _load().or_quant_act_static(_ptr(x, ctypes.c_float), M, K, _ptr(inv_s, ctypes.c_float), ctypes.c_float(delta),
                                 _ptr(xq, ctypes.c_int8), _ptr(dx, ctypes.c_float))
     return xq, dx
+
+
+# ---------------------------------------------------------------------------
+# FP8 (E4M3) variant
+# ---------------------------------------------------------------------------
+
+def e4m3_decode(codes) -> np.ndarray:
+    """Exact float value of each E4M3 code (uint8 array)."""
+    c = np.asarray(codes, dtype=np.uint8)
+    f = _load().or_e4m3_decode
+    return np.array([f(int(v)) for v in c.ravel()], np.float32).reshape(c.shape)
+
+
+def e4m3_encode(values) -> np.ndarray:
+    """Nearest E4M3 code of each fp32 value (ties to even, +-448 beyond)."""
+    v = _f32(values)
+    f = _load().or_e4m3_encode
+    return np.array([f(float(x)) for x in v.ravel()], np.uint8).reshape(v.shape)
+
+
+def smooth_quant_weight_e4m3(w, layout: int, s):
+    """(Wq [N, K] uint8 E4M3 codes, dw [N]) of W~ = diag(s) W, per output channel."""
+    w = _f32(w)
+    s = _f32(s)
+    K, N = _kn(w, layout)
+    wq = np.zeros((N, K), np.uint8)
+    dw = np.zeros(N, np.float32)
+    _load().or_smooth_quant_weight_e4m3(_ptr(w, ctypes.c_float), layout, K, N, _ptr(s, ctypes.c_float),
+                                        _ptr(wq, ctypes.c_uint8), _ptr(dw, ctypes.c_float))
+    return wq, dw
+
+
+def quant_act_e4m3(x, inv_s):
+    """(Xq [M, K] uint8 E4M3 codes, dx [M]) of X~ = X diag(s)^-1, per token."""
+    x = _f32(x)
+    inv_s = _f32(inv_s)
+    M, K = x.shape
+    xq = np.zeros((M, K), np.uint8)
+    dx = np.zeros(M, np.float32)
+    _load().or_quant_act_e4m3(_ptr(x, ctypes.c_float), M, K, _ptr(inv_s, ctypes.c_float),
+                              _ptr(xq, ctypes.c_uint8), _ptr(dx, ctypes.c_float))
+    return xq, dx
+
+
+def gemm_e4m3(xq, wq) -> np.ndarray:
+    """Exact acc[M, N] = sum_j e4m3(xq[t, j]) e4m3(wq[n, j]) in float64."""
+    xq = np.ascontiguousarray(xq, dtype=np.uint8)
+    wq = np.ascontiguousarray(wq, dtype=np.uint8)
+    M, K = xq.shape
+    N = wq.shape[0]
+    acc = np.zeros((M, N), np.float64)
+    _load().or_gemm_e4m3(_ptr(xq, ctypes.c_uint8), _ptr(wq, ctypes.c_uint8), M, N, K,
+                         _ptr(acc, ctypes.c_double))
+    return acc
+
+
+def dequant_f32acc(acc, dx, dw) -> np.ndarray:
+    """y = ((float)acc * dx_t) * dw_n for an fp32 accumulator."""
+    acc = _f32(acc)
+    dx = _f32(dx)
+    dw = _f32(dw)
+    M, N = acc.shape
+    y = np.zeros((M, N), np.float32)
+    _load().or_dequant_f32acc(_ptr(acc, ctypes.c_float), _ptr(dx, ctypes.c_float), _ptr(dw, ctypes.c_float), M, N,
+                              _ptr(y, ctypes.c_float))
+    return y
 
 
 def linear(x, inv_s, wq, dw, out_dtype: str = "f32"):

@@ -301,3 +301,105 @@ void or_quant_act_static(const float *x, int64_t M, int64_t K, const float *inv_
     for (int64_t j = 0; j < K; ++j) xq[t * K + j] = or_quantize_value(x[t * K + j] * inv_s[j], r);
   }
 }
+
+/* ---- FP8 (E4M3) variant --------------------------------------------------
+ * The survey page "Quantization Calibration GPTQ/AWQ/SmoothQuant 2026"
+ * (jisaku.com glossary) lists FP8 SmoothQuant: the same smoothing with FP8
+ * operands (its spec-comparison table: 8-bit weights, FP8 activations).
+ * Readings: both operands in E4M3 -- the 8-bit float with 1 sign bit, 4
+ * exponent bits of bias 7 and 3 mantissa bits, no infinities, the all-ones
+ * exponent with mantissa 111 as NaN, largest finite value 448, subnormals
+ * (m/8) * 2^-6 -- with the INT8 path's granularity: delta = m/448 per token
+ * and per output channel, code = e4m3(v * (448/m)) rounded to nearest, ties
+ * to the even code, saturating at +-448.  The product of two E4M3 values is
+ * exact, and so is the sum over K in double: every product is a multiple of
+ * 2^-18 below 448^2 < 2^18, so K <= 2^15 terms stay within 51 bits. */
+
+/* Exact value of an E4M3 code. */
+float or_e4m3_decode(uint8_t c) {
+  const int e = (c >> 3) & 15, m = c & 7;
+  if (e == 15 && m == 7) return NAN;
+  const float mag = e == 0 ? ldexpf((float)m, -9) : ldexpf((float)(8 + m), e - 10);
+  return (c & 0x80) ? -mag : mag;
+}
+
+/* The E4M3 code nearest to v (ties to the even code), +-448 beyond. */
+uint8_t or_e4m3_encode(float v) {
+  if (isnan(v)) return 0x7f;
+  const uint8_t sign = signbit(v) ? 0x80 : 0x00;
+  const float a = fabsf(v);
+  if (a >= 448.0f) return sign | 0x7e;
+  /* binade of a: a in [2^e, 2^(e+1)); below 2^-6 the spacing stays 2^-9 */
+  int x;
+  frexpf(a, &x);
+  int e = a == 0.0f ? -6 : x - 1;
+  if (e < -6) e = -6;
+  const float quantum = ldexpf(1.0f, e - 3);
+  const float q = rintf(a / quantum); /* a / 2^k is exact; rintf rounds half to even */
+  const float r = q * quantum;         /* the rounded magnitude, <= 448 */
+  if (r < ldexpf(1.0f, -6)) return sign | (uint8_t)(r / ldexpf(1.0f, -9)); /* subnormal or zero */
+  frexpf(r, &x);
+  const int er = x - 1;                                   /* r in [2^er, 2^(er+1)) */
+  const int mant = (int)(r / ldexpf(1.0f, er - 3)) - 8;   /* 0..7 */
+  return sign | (uint8_t)(((er + 7) << 3) | mant);
+}
+
+static uint8_t e4m3_quantize_value(float v, float r) { return or_e4m3_encode(v * r); }
+
+/* Per-output-channel E4M3 weights: m_n = max_j |W~_jn|, dw_n = m_n/448,
+ * Wq[n][j] = e4m3(W~_jn * (448/m_n)), stored [N][K]. */
+void or_smooth_quant_weight_e4m3(const float *w, int layout, int64_t K, int64_t N, const float *s, uint8_t *wq,
+                                 float *dw) {
+  for (int64_t n = 0; n < N; ++n) {
+    float m = 0.0f;
+    for (int64_t j = 0; j < K; ++j) {
+      float v = fabsf(s[j] * w_at(w, layout, K, N, j, n));
+      if (v > m) m = v;
+    }
+    if (m == 0.0f) {
+      dw[n] = 0.0f;
+      for (int64_t j = 0; j < K; ++j) wq[n * K + j] = 0;
+      continue;
+    }
+    dw[n] = m / 448.0f;
+    float r = 448.0f / m;
+    for (int64_t j = 0; j < K; ++j) wq[n * K + j] = e4m3_quantize_value(s[j] * w_at(w, layout, K, N, j, n), r);
+  }
+}
+
+/* Per-token E4M3 activations: m_t = max_j |X~_tj|, dx_t = m_t/448,
+ * Xq[t][j] = e4m3(X~_tj * (448/m_t)). */
+void or_quant_act_e4m3(const float *x, int64_t M, int64_t K, const float *inv_s, uint8_t *xq, float *dx) {
+  for (int64_t t = 0; t < M; ++t) {
+    float m = 0.0f;
+    for (int64_t j = 0; j < K; ++j) {
+      float v = fabsf(x[t * K + j] * inv_s[j]);
+      if (v > m) m = v;
+    }
+    if (m == 0.0f) {
+      dx[t] = 0.0f;
+      for (int64_t j = 0; j < K; ++j) xq[t * K + j] = 0;
+      continue;
+    }
+    dx[t] = m / 448.0f;
+    float r = 448.0f / m;
+    for (int64_t j = 0; j < K; ++j) xq[t * K + j] = e4m3_quantize_value(x[t * K + j] * inv_s[j], r);
+  }
+}
+
+/* acc[t][n] = sum_j e4m3(Xq[t][j]) * e4m3(Wq[n][j]), exact in double. */
+void or_gemm_e4m3(const uint8_t *xq, const uint8_t *wq, int64_t M, int64_t N, int64_t K, double *acc) {
+  for (int64_t t = 0; t < M; ++t)
+    for (int64_t n = 0; n < N; ++n) {
+      double sum = 0.0;
+      for (int64_t j = 0; j < K; ++j)
+        sum += (double)or_e4m3_decode(xq[t * K + j]) * (double)or_e4m3_decode(wq[n * K + j]);
+      acc[t * N + n] = sum;
+    }
+}
+
+/* y[t][n] = ((float)acc[t][n] * dx_t) * dw_n with an fp32 accumulator. */
+void or_dequant_f32acc(const float *acc, const float *dx, const float *dw, int64_t M, int64_t N, float *y) {
+  for (int64_t t = 0; t < M; ++t)
+    for (int64_t n = 0; n < N; ++n) y[t * N + n] = (acc[t * N + n] * dx[t]) * dw[n];
+}
