@@ -50,13 +50,15 @@ WEIGHT_LAUNCHES = 4
 # ncu on a smaller launch of the same kernel, as a ratio to that launch's
 # algorithmic bytes; the bench scales it to its own per-launch bytes (the
 # traffic of these streaming kernels grows in proportion to the bytes they
-# stream).  Each entry is tied to the hash of the kernel source it was
-# measured on and reported as null once that source changes.
+# stream).  Each entry is tied to a hash of the source text of the kernel
+# and of its launcher (grid shape), as measured, and reported as null once
+# either changes.
 TRAFFIC = {
-    # calibration 65536 x 4096 fp16: 536904960 + 3084288 bytes for
+    # calibration 65536 x 4096 fp16: 536940288 + 3097088 bytes for
     # 536870912 + 32768 algorithmic bytes
-    "absmax_cols_kernel": {"source": "sq_bw.cu", "sha": "87bf3f65891378f3",
-                           "ratio": (536904960 + 3084288) / (536870912 + 32768)},
+    "absmax_cols_kernel": {"source": "sq_bw.cu", "functions": ("absmax_cols_kernel", "absmax_cols_t"),
+                           "sha": "7fab8257c9f3f2c0",
+                           "ratio": (536940288 + 3097088) / (536870912 + 32768)},
 }
 
 
@@ -70,16 +72,40 @@ def peaks():
     return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, src="fallback")
 
 
-def src_hash(name: str) -> str:
+def function_text(src: str, name: str) -> str:
+    """Source text of the definition of function `name` in src: from the
+    line that opens it (its template line, if any) to its closing brace."""
+    i = 0
+    while True:
+        i = src.index(name + "(", i)
+        body = src.index("{", i)
+        if src.find(";", i, body) < 0:  # a definition, not a call or declaration
+            break
+        i += len(name)
+    start = src.rfind("\n\n", 0, i) + 2
+    depth, j = 0, body
+    while True:
+        if src[j] == "{":
+            depth += 1
+        elif src[j] == "}":
+            depth -= 1
+            if depth == 0:
+                return src[start:j + 1]
+        j += 1
+
+
+def src_hash(name: str, functions) -> str:
     p = os.path.join(ROOT, "w8a8_post_quantization_channel_b200", "csrc", name)
-    with open(p, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+    with open(p) as f:
+        src = f.read()
+    text = "\n".join(function_text(src, fn) for fn in functions)
+    return hashlib.sha256(text.encode()).hexdigest()[:16]
 
 
 def traffic_for(kernel: str, algorithmic_bytes: float):
     """Per-launch DRAM bytes for a launch moving algorithmic_bytes, or None."""
     t = TRAFFIC.get(kernel)
-    if not t or src_hash(t["source"]) != t["sha"]:
+    if not t or src_hash(t["source"], t["functions"]) != t["sha"]:
         return None
     return int(round(t["ratio"] * algorithmic_bytes))
 

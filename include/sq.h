@@ -116,6 +116,59 @@ sq_status sq_quant_act(const void *x, sq_dtype xt, int64_t M, int64_t K,
                        float *x_scale, sq_stream_t stream);
 
 /*
+ * Fold diag(s)^-1 into the weight of the norm that produces X, once per
+ * layer, the way sq_smooth_quant_weight folds diag(s) into W: smooth_lm(alpha)
+ * in the page's usage example moves the smoothing out of the run-time path.
+ *   gs_j = gamma_j * inv_smooth_j   (fp32, IEEE round to nearest even)
+ *   gamma, inv_smooth [K] fp32 IN; gs [K] fp32 OUT (may alias gamma).
+ * K > 0; 16-byte aligned device pointers.
+ */
+sq_status sq_fold_smooth_into_norm(const float *gamma, const float *inv_smooth,
+                                   int64_t K, float *gs, sq_stream_t stream);
+
+/*
+ * Upstream producer: RMS normalisation of each token with the folded weight
+ * gs (sq_fold_smooth_into_norm), then per-token INT8, in one pass; in
+ * transformer blocks this replaces norm + sq_quant_act:
+ *   r_t  = 1 / sqrt(sum_j x_tj^2 / K + eps)   (squares summed in double
+ *          precision in an unspecified order, root and reciprocal in double,
+ *          rounded once to fp32)
+ *   v_tj = (x_tj * r_t) * gs_j   (fp32, in that order)
+ *   then per-token quantization of v exactly as sq_quant_act.
+ *   gs [K] fp32, eps >= 0 and finite.  Other arguments as sq_quant_act.
+ * Because the order of the double-precision sum is unspecified, r_t may
+ * differ from another implementation's by one fp32 ulp, which moves a code
+ * by one only where v * 127 / max lies within ~2^-20 of a rounding
+ * boundary.  K <= 16384 for 16-bit x, <= 8192 for fp32 x, else
+ * SQ_ERR_UNSUPPORTED.
+ */
+sq_status sq_rmsnorm_quant_act(const void *x, sq_dtype xt, int64_t M, int64_t K,
+                               int64_t ldx, const float *gs, float eps,
+                               int8_t *xq, float *x_scale, sq_stream_t stream);
+
+/*
+ * Static per-tensor activation scale, the alternative to per-token scales
+ * (the page notes activations change per prompt, which is why the main path
+ * measures each token at run time).  After smoothing, channel j's
+ * calibrated maximum is amax_j * inv_smooth_j, so
+ *   *delta = max_j(amax_j * inv_smooth_j) / 127   (one fp32 on the device).
+ */
+sq_status sq_static_act_scale(const float *amax, const float *inv_smooth, int64_t K,
+                              float *delta, sq_stream_t stream);
+
+/*
+ * Static quantization with that scale: xq = clamp(rne((x * inv_smooth) *
+ * (1 / *delta)), -127, 127) -- values beyond the calibrated range
+ * saturate -- and x_scale_t = *delta for every token, so sq_w8a8_linear
+ * consumes the result unchanged.  delta is a device pointer (*delta > 0).
+ * Other arguments as sq_quant_act.
+ */
+sq_status sq_quant_act_static(const void *x, sq_dtype xt, int64_t M, int64_t K,
+                              int64_t ldx, const float *inv_smooth,
+                              const float *delta, int8_t *xq, float *x_scale,
+                              sq_stream_t stream);
+
+/*
  * W8A8 linear on the tensor cores (tcgen05, kind::i8): exact int32
  * accumulation acc_tn = sum_j xq_tj * wq_nj, then the dequant epilogue
  * y_tn = round_yt(((float)acc_tn * x_scale_t) * w_scale_n).
@@ -147,6 +200,48 @@ sq_status sq_w8a8_accumulate(const int8_t *xq, const int8_t *wq, int64_t M,
                              int64_t N, int64_t K, int32_t *acc, int64_t ldacc,
                              void *workspace, size_t workspace_bytes,
                              sq_stream_t stream);
+
+/*
+ * FP8 (E4M3) variant.  The survey page "Quantization Calibration
+ * GPTQ/AWQ/SmoothQuant 2026" (jisaku.com glossary) lists FP8 SmoothQuant:
+ * the same smoothing, with FP8 operands.  Both operands are E4M3 codes (1
+ * sign, 4 exponent bits of bias 7, 3 mantissa bits, no infinities,
+ * S.1111.111 = NaN, largest finite 448) with the INT8 path's granularity:
+ *   scale = m / 448 for a row with absmax m, and
+ *   code  = e4m3(v * (448 / m)), nearest value, ties to the even code,
+ *           saturating at +-448;  an all-zero row gives scale 0, codes +0.
+ * Smoothing (s, 1/s) is computed exactly as for INT8.  The product runs on
+ * the tensor cores' FP8 path with an fp32 accumulator: every product of
+ * two E4M3 values is exact, the additions are fp32 in the hardware's own
+ * order, so the sum is within K * 2^-22 * sum_j |x_j w_j| of the exact one
+ * (and deterministic: the same inputs and launch give the same bits).
+ *
+ * sq_smooth_quant_weight_e4m3: as sq_smooth_quant_weight, with wq [N][K]
+ *   E4M3 codes (uint8) and w_scale = max_j|W~_jn| / 448.
+ * sq_quant_act_e4m3: as sq_quant_act, with xq [M][K] E4M3 codes and
+ *   x_scale = max_j|X~_tj| / 448.
+ * sq_w8a8_linear_e4m3: y = round_yt((acc_tn * x_scale_t) * w_scale_n) with
+ *   the fp32 accumulator acc; arguments, workspace
+ *   (sq_w8a8_linear_workspace_size) and errors as sq_w8a8_linear.
+ * sq_w8a8_accumulate_e4m3: the fp32 accumulator alone, acc [M][ldacc].
+ */
+sq_status sq_smooth_quant_weight_e4m3(const void *w, sq_dtype wt, sq_wlayout layout,
+                                      int64_t K, int64_t N, int64_t ldw,
+                                      const float *amax, float alpha, uint8_t *wq,
+                                      float *w_scale, float *smooth,
+                                      float *inv_smooth, sq_stream_t stream);
+sq_status sq_quant_act_e4m3(const void *x, sq_dtype xt, int64_t M, int64_t K,
+                            int64_t ldx, const float *inv_smooth, uint8_t *xq,
+                            float *x_scale, sq_stream_t stream);
+sq_status sq_w8a8_linear_e4m3(const uint8_t *xq, const float *x_scale,
+                              const uint8_t *wq, const float *w_scale, int64_t M,
+                              int64_t N, int64_t K, void *y, sq_dtype yt,
+                              int64_t ldy, void *workspace, size_t workspace_bytes,
+                              sq_stream_t stream);
+sq_status sq_w8a8_accumulate_e4m3(const uint8_t *xq, const uint8_t *wq, int64_t M,
+                                  int64_t N, int64_t K, float *acc, int64_t ldacc,
+                                  void *workspace, size_t workspace_bytes,
+                                  sq_stream_t stream);
 
 /*
  * Allocation-free variant of sq_w8a8_linear for decode-shaped calls.

@@ -82,6 +82,32 @@ def test_quant_act_argument_checks():
     assert f(MIS, sq.SQ_F32, 8, 256, 256, A16, A16, A16, None) == INV
 
 
+def test_producer_argument_checks():
+    L = sq.lib()
+    fold = L.sq_fold_smooth_into_norm
+    assert fold(None, A16, 256, A16, None) == INV
+    assert fold(A16, None, 256, A16, None) == INV
+    assert fold(A16, A16, 256, MIS, None) == INV
+    assert fold(A16, A16, 0, A16, None) == INV
+    f = L.sq_rmsnorm_quant_act
+    eps = ctypes.c_float(1e-5)
+    assert f(None, sq.SQ_BF16, 0, 256, 256, A16, eps, None, None, None) == sq.SQ_OK     # M == 0: no-op
+    assert f(A16, sq.SQ_BF16, 8, 256, 256, None, eps, A16, A16, None) == INV            # null gs
+    assert f(A16, sq.SQ_BF16, 8, 256, 256, A16, ctypes.c_float(-1.0), A16, A16, None) == INV
+    assert f(A16, sq.SQ_BF16, 8, 256, 256, A16, ctypes.c_float(float("nan")), A16, A16, None) == INV
+    assert f(A16, sq.SQ_BF16, 8, 256, 256, A16, ctypes.c_float(float("inf")), A16, A16, None) == INV
+    assert f(A16, sq.SQ_BF16, 8, 24, 24, A16, eps, A16, A16, None) == INV               # K % 16
+    assert f(A16, sq.SQ_BF16, 8, 16400, 16400, A16, eps, A16, A16, None) == sq.SQ_ERR_UNSUPPORTED
+    assert f(A16, sq.SQ_F32, 8, 8208, 8208, A16, eps, A16, A16, None) == sq.SQ_ERR_UNSUPPORTED
+    st = L.sq_static_act_scale
+    assert st(A16, A16, 256, MIS + 1, None) == INV                                       # delta not 4-B aligned
+    assert st(None, A16, 256, A16, None) == INV
+    qs = L.sq_quant_act_static
+    assert qs(None, sq.SQ_F16, 0, 256, 256, A16, A16, None, None, None) == sq.SQ_OK
+    assert qs(A16, sq.SQ_F16, 8, 256, 256, A16, None, A16, A16, None) == INV             # null delta
+    assert qs(A16, sq.SQ_F16, 8, 256, 256, None, A16, A16, A16, None) == INV             # null inv_s
+
+
 def test_linear_argument_checks():
     f = sq.lib().sq_w8a8_linear
     base = [A16, A16, A16, A16, 64, 256, 256, A16, sq.SQ_BF16, 256, None, 0, None]

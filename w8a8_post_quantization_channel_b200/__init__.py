@@ -34,6 +34,8 @@ __all__ = [
     "sq_calib_absmax", "sq_smooth_quant_weight", "sq_quant_act", "sq_w8a8_linear",
     "sq_w8a8_linear_workspace_size", "sq_w8a8_accumulate", "sq_check_device_error", "sq_status_string",
     "sq_w8a8_linear_decode_noalloc", "SQ_DECODE_STATIC_SCRATCH_BYTES", "sq_selftest_wait_timeout",
+    "sq_fold_smooth_into_norm", "sq_rmsnorm_quant_act", "sq_static_act_scale", "sq_quant_act_static",
+    "sq_smooth_quant_weight_e4m3", "sq_quant_act_e4m3", "sq_w8a8_linear_e4m3", "sq_w8a8_accumulate_e4m3",
 ]
 
 SQ_OK, SQ_ERR_INVALID_ARG, SQ_ERR_UNSUPPORTED, SQ_ERR_CUDA, SQ_ERR_TIMEOUT = 0, 1, 2, 3, 4
@@ -80,6 +82,14 @@ def lib() -> ctypes.CDLL:
             "sq_check_device_error": [vp],
             "sq_w8a8_linear_decode_noalloc": [vp, vp, vp, vp, i64, i64, i64, vp, i32, i64, vp],
             "sq_selftest_wait_timeout": [i32, vp],
+            "sq_fold_smooth_into_norm": [vp, vp, i64, vp, vp],
+            "sq_rmsnorm_quant_act": [vp, i32, i64, i64, i64, vp, f32, vp, vp, vp],
+            "sq_static_act_scale": [vp, vp, i64, vp, vp],
+            "sq_quant_act_static": [vp, i32, i64, i64, i64, vp, vp, vp, vp, vp],
+            "sq_smooth_quant_weight_e4m3": [vp, i32, i32, i64, i64, i64, vp, f32, vp, vp, vp, vp, vp],
+            "sq_quant_act_e4m3": [vp, i32, i64, i64, i64, vp, vp, vp, vp],
+            "sq_w8a8_linear_e4m3": [vp, vp, vp, vp, i64, i64, i64, vp, i32, i64, vp, sz, vp],
+            "sq_w8a8_accumulate_e4m3": [vp, vp, i64, i64, i64, vp, i64, vp, sz, vp],
         }
         for name, args in sigs.items():
             fn = getattr(L, name)
@@ -167,6 +177,45 @@ def sq_quant_act(x: torch.Tensor, inv_smooth: torch.Tensor, xq=None, x_scale=Non
     return xq, x_scale
 
 
+def sq_fold_smooth_into_norm(gamma: torch.Tensor, inv_smooth: torch.Tensor, gs=None, stream=None) -> torch.Tensor:
+    """gs = gamma * inv_smooth (fp32): the smoothing folded into the norm weight."""
+    gs = torch.empty_like(gamma) if gs is None else gs
+    _check(lib().sq_fold_smooth_into_norm(_ptr(gamma), _ptr(inv_smooth), gamma.numel(), _ptr(gs), _stream(stream)),
+           "sq_fold_smooth_into_norm")
+    return gs
+
+
+def sq_rmsnorm_quant_act(x: torch.Tensor, gs: torch.Tensor, eps: float, xq=None, x_scale=None, stream=None):
+    """(xq, x_scale) = per-token INT8 of RMSNorm(x; eps) with the folded weight gs."""
+    _rowmajor(x, "x")
+    M, K = x.shape
+    xq = torch.empty((M, K), dtype=torch.int8, device=x.device) if xq is None else xq
+    x_scale = torch.empty(M, dtype=torch.float32, device=x.device) if x_scale is None else x_scale
+    _check(lib().sq_rmsnorm_quant_act(_ptr(x), _dtype(x, "x"), M, K, x.stride(0), _ptr(gs), ctypes.c_float(eps),
+                                      _ptr(xq), _ptr(x_scale), _stream(stream)), "sq_rmsnorm_quant_act")
+    return xq, x_scale
+
+
+def sq_static_act_scale(amax: torch.Tensor, inv_smooth: torch.Tensor, delta=None, stream=None) -> torch.Tensor:
+    """delta (1-element device tensor) = max_j(amax_j * inv_smooth_j) / 127."""
+    delta = torch.empty(1, dtype=torch.float32, device=amax.device) if delta is None else delta
+    _check(lib().sq_static_act_scale(_ptr(amax), _ptr(inv_smooth), amax.numel(), _ptr(delta), _stream(stream)),
+           "sq_static_act_scale")
+    return delta
+
+
+def sq_quant_act_static(x: torch.Tensor, inv_smooth: torch.Tensor, delta: torch.Tensor, xq=None, x_scale=None,
+                        stream=None):
+    """(xq, x_scale) with one fixed scale *delta (device scalar); saturates."""
+    _rowmajor(x, "x")
+    M, K = x.shape
+    xq = torch.empty((M, K), dtype=torch.int8, device=x.device) if xq is None else xq
+    x_scale = torch.empty(M, dtype=torch.float32, device=x.device) if x_scale is None else x_scale
+    _check(lib().sq_quant_act_static(_ptr(x), _dtype(x, "x"), M, K, x.stride(0), _ptr(inv_smooth), _ptr(delta),
+                                     _ptr(xq), _ptr(x_scale), _stream(stream)), "sq_quant_act_static")
+    return xq, x_scale
+
+
 def sq_w8a8_linear_workspace_size(M: int, N: int, K: int) -> int:
     return int(lib().sq_w8a8_linear_workspace_size(M, N, K))
 
@@ -199,6 +248,69 @@ def sq_w8a8_accumulate(xq: torch.Tensor, wq: torch.Tensor, acc=None, workspace=N
     wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib().sq_w8a8_accumulate(_ptr(xq), _ptr(wq), M, N, K, _ptr(acc), acc.stride(0), _ptr(workspace),
                                     wbytes, _stream(stream)), "sq_w8a8_accumulate")
+    return acc
+
+
+# ---------------------------------------------------------------------------
+# FP8 (E4M3) variant: codes are uint8 tensors holding E4M3 bit patterns
+# ---------------------------------------------------------------------------
+
+def sq_smooth_quant_weight_e4m3(w: torch.Tensor, layout: int, amax: torch.Tensor, alpha: float = 0.5,
+                                wq=None, w_scale=None, smooth=None, inv_smooth=None, stream=None):
+    """(wq [N,K] uint8 E4M3, w_scale [N] = absmax/448, s [K], inv_s [K])."""
+    _rowmajor(w, "w")
+    K, N = (w.shape[0], w.shape[1]) if layout == SQ_W_KN else (w.shape[1], w.shape[0])
+    dev = w.device
+    wq = torch.empty((N, K), dtype=torch.uint8, device=dev) if wq is None else wq
+    w_scale = torch.empty(N, dtype=torch.float32, device=dev) if w_scale is None else w_scale
+    smooth = torch.empty(K, dtype=torch.float32, device=dev) if smooth is None else smooth
+    inv_smooth = torch.empty(K, dtype=torch.float32, device=dev) if inv_smooth is None else inv_smooth
+    _check(lib().sq_smooth_quant_weight_e4m3(_ptr(w), _dtype(w, "w"), layout, K, N, w.stride(0), _ptr(amax),
+                                             ctypes.c_float(alpha), _ptr(wq), _ptr(w_scale), _ptr(smooth),
+                                             _ptr(inv_smooth), _stream(stream)), "sq_smooth_quant_weight_e4m3")
+    return wq, w_scale, smooth, inv_smooth
+
+
+def sq_quant_act_e4m3(x: torch.Tensor, inv_smooth: torch.Tensor, xq=None, x_scale=None, stream=None):
+    """(xq [M,K] uint8 E4M3, x_scale [M] = absmax/448) of x * inv_smooth, per token."""
+    _rowmajor(x, "x")
+    M, K = x.shape
+    xq = torch.empty((M, K), dtype=torch.uint8, device=x.device) if xq is None else xq
+    x_scale = torch.empty(M, dtype=torch.float32, device=x.device) if x_scale is None else x_scale
+    _check(lib().sq_quant_act_e4m3(_ptr(x), _dtype(x, "x"), M, K, x.stride(0), _ptr(inv_smooth), _ptr(xq),
+                                   _ptr(x_scale), _stream(stream)), "sq_quant_act_e4m3")
+    return xq, x_scale
+
+
+def sq_w8a8_linear_e4m3(xq: torch.Tensor, x_scale: torch.Tensor, wq: torch.Tensor, w_scale: torch.Tensor,
+                        out_dtype=torch.bfloat16, y=None, workspace=None, stream=None) -> torch.Tensor:
+    """y [M,N] = dequant(xq . wq^T) for E4M3 codes, fp32 accumulation."""
+    M, K = xq.shape
+    N = wq.shape[0]
+    y = torch.empty((M, N), dtype=out_dtype, device=xq.device) if y is None else y
+    _rowmajor(y, "y")
+    need = sq_w8a8_linear_workspace_size(M, N, K)
+    if workspace is None and need > 0:
+        workspace = torch.zeros(need, dtype=torch.uint8, device=xq.device)
+    wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().sq_w8a8_linear_e4m3(_ptr(xq), _ptr(x_scale), _ptr(wq), _ptr(w_scale), M, N, K, _ptr(y),
+                                     _dtype(y, "y"), y.stride(0), _ptr(workspace), wbytes, _stream(stream)),
+           "sq_w8a8_linear_e4m3")
+    return y
+
+
+def sq_w8a8_accumulate_e4m3(xq: torch.Tensor, wq: torch.Tensor, acc=None, workspace=None,
+                            stream=None) -> torch.Tensor:
+    """acc [M,N] float32 = e4m3(xq) . e4m3(wq)^T on the tensor cores."""
+    M, K = xq.shape
+    N = wq.shape[0]
+    acc = torch.empty((M, N), dtype=torch.float32, device=xq.device) if acc is None else acc
+    need = sq_w8a8_linear_workspace_size(M, N, K)
+    if workspace is None and need > 0:
+        workspace = torch.zeros(need, dtype=torch.uint8, device=xq.device)
+    wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().sq_w8a8_accumulate_e4m3(_ptr(xq), _ptr(wq), M, N, K, _ptr(acc), acc.stride(0), _ptr(workspace),
+                                         wbytes, _stream(stream)), "sq_w8a8_accumulate_e4m3")
     return acc
 
 

@@ -96,9 +96,9 @@ sq_status sq_calib_absmax(const void *x, sq_dtype xt, int64_t T, int64_t K, int6
   return from_cuda(sq::launch_absmax_cols(x, xt, T, K, ldx, nullptr, amax, false, (cudaStream_t)stream));
 }
 
-sq_status sq_smooth_quant_weight(const void *w, sq_dtype wt, sq_wlayout layout, int64_t K, int64_t N, int64_t ldw,
-                                 const float *amax, float alpha, int8_t *wq, float *w_scale, float *smooth,
-                                 float *inv_smooth, sq_stream_t stream) {
+static sq_status smooth_quant_weight_impl(const void *w, sq_dtype wt, sq_wlayout layout, int64_t K, int64_t N,
+                                          int64_t ldw, const float *amax, float alpha, int8_t *wq, float *w_scale,
+                                          float *smooth, float *inv_smooth, sq::QFmt fmt, sq_stream_t stream) {
   if (!valid_dtype(wt) || (layout != SQ_W_KN && layout != SQ_W_NK)) return SQ_ERR_INVALID_ARG;
   if (K <= 0 || N <= 0 || K % 16 != 0 || N % 16 != 0) return SQ_ERR_INVALID_ARG;
   if (!(alpha >= 0.0f && alpha <= 1.0f)) return SQ_ERR_INVALID_ARG;
@@ -123,21 +123,84 @@ sq_status sq_smooth_quant_weight(const void *w, sq_dtype wt, sq_wlayout layout, 
   if (kn) {
     e = sq::launch_zero_fill(w_scale, N, st);
     if (e == cudaSuccess) e = sq::launch_absmax_cols(w, wt, K, N, ldw, smooth, w_scale, true, st);
-    if (e == cudaSuccess) e = sq::launch_quant_cols_transpose(w, wt, K, N, ldw, smooth, w_scale, wq, st);
+    if (e == cudaSuccess) e = sq::launch_quant_cols_transpose(w, wt, K, N, ldw, smooth, w_scale, wq, fmt, st);
   } else {
-    e = sq::launch_quant_rows(w, wt, N, K, ldw, smooth, wq, w_scale, st);
+    e = sq::launch_quant_rows(w, wt, N, K, ldw, smooth, wq, w_scale, fmt, st);
   }
   return from_cuda(e);
 }
 
-sq_status sq_quant_act(const void *x, sq_dtype xt, int64_t M, int64_t K, int64_t ldx, const float *inv_smooth,
-                       int8_t *xq, float *x_scale, sq_stream_t stream) {
+sq_status sq_smooth_quant_weight(const void *w, sq_dtype wt, sq_wlayout layout, int64_t K, int64_t N, int64_t ldw,
+                                 const float *amax, float alpha, int8_t *wq, float *w_scale, float *smooth,
+                                 float *inv_smooth, sq_stream_t stream) {
+  return smooth_quant_weight_impl(w, wt, layout, K, N, ldw, amax, alpha, wq, w_scale, smooth, inv_smooth,
+                                  sq::QFmt::I8, stream);
+}
+
+sq_status sq_smooth_quant_weight_e4m3(const void *w, sq_dtype wt, sq_wlayout layout, int64_t K, int64_t N,
+                                      int64_t ldw, const float *amax, float alpha, uint8_t *wq, float *w_scale,
+                                      float *smooth, float *inv_smooth, sq_stream_t stream) {
+  return smooth_quant_weight_impl(w, wt, layout, K, N, ldw, amax, alpha, reinterpret_cast<int8_t *>(wq), w_scale,
+                                  smooth, inv_smooth, sq::QFmt::E4M3, stream);
+}
+
+static sq_status quant_act_impl(const void *x, sq_dtype xt, int64_t M, int64_t K, int64_t ldx,
+                                const float *inv_smooth, int8_t *xq, float *x_scale, sq::QFmt fmt,
+                                sq_stream_t stream) {
   if (!valid_dtype(xt) || K <= 0 || K % 16 != 0 || K >= kMaxDim || M < 0 || M >= kMaxDim) return SQ_ERR_INVALID_ARG;
   if (ldx < K || (ldx * dsize(xt)) % 16 != 0) return SQ_ERR_INVALID_ARG;
   if (!valid_vec(inv_smooth)) return SQ_ERR_INVALID_ARG;
   if (M == 0) return SQ_OK;
   if (!valid_matrix(x, xt, M, K, ldx) || !valid_vec(xq) || !valid_vec(x_scale)) return SQ_ERR_INVALID_ARG;
-  return from_cuda(sq::launch_quant_rows(x, xt, M, K, ldx, inv_smooth, xq, x_scale, (cudaStream_t)stream));
+  return from_cuda(sq::launch_quant_rows(x, xt, M, K, ldx, inv_smooth, xq, x_scale, fmt, (cudaStream_t)stream));
+}
+
+sq_status sq_quant_act(const void *x, sq_dtype xt, int64_t M, int64_t K, int64_t ldx, const float *inv_smooth,
+                       int8_t *xq, float *x_scale, sq_stream_t stream) {
+  return quant_act_impl(x, xt, M, K, ldx, inv_smooth, xq, x_scale, sq::QFmt::I8, stream);
+}
+
+sq_status sq_quant_act_e4m3(const void *x, sq_dtype xt, int64_t M, int64_t K, int64_t ldx, const float *inv_smooth,
+                            uint8_t *xq, float *x_scale, sq_stream_t stream) {
+  return quant_act_impl(x, xt, M, K, ldx, inv_smooth, reinterpret_cast<int8_t *>(xq), x_scale, sq::QFmt::E4M3,
+                        stream);
+}
+
+sq_status sq_fold_smooth_into_norm(const float *gamma, const float *inv_smooth, int64_t K, float *gs,
+                                   sq_stream_t stream) {
+  if (K <= 0 || K >= kMaxDim || !valid_vec(gamma) || !valid_vec(inv_smooth) || !valid_vec(gs))
+    return SQ_ERR_INVALID_ARG;
+  return from_cuda(sq::launch_fold_norm_weight(gamma, inv_smooth, K, gs, (cudaStream_t)stream));
+}
+
+sq_status sq_rmsnorm_quant_act(const void *x, sq_dtype xt, int64_t M, int64_t K, int64_t ldx, const float *gs,
+                               float eps, int8_t *xq, float *x_scale, sq_stream_t stream) {
+  if (!valid_dtype(xt) || K <= 0 || K % 16 != 0 || K >= kMaxDim || M < 0 || M >= kMaxDim) return SQ_ERR_INVALID_ARG;
+  if (ldx < K || (ldx * dsize(xt)) % 16 != 0) return SQ_ERR_INVALID_ARG;
+  if (!(eps >= 0.0f) || eps > 3.0e38f) return SQ_ERR_INVALID_ARG;  // rejects NaN and infinity too
+  if (!valid_vec(gs)) return SQ_ERR_INVALID_ARG;
+  if (K > (xt == SQ_F32 ? 8192 : 16384)) return SQ_ERR_UNSUPPORTED;
+  if (M == 0) return SQ_OK;
+  if (!valid_matrix(x, xt, M, K, ldx) || !valid_vec(xq) || !valid_vec(x_scale)) return SQ_ERR_INVALID_ARG;
+  return from_cuda(sq::launch_rmsnorm_quant(x, xt, M, K, ldx, gs, eps, xq, x_scale, (cudaStream_t)stream));
+}
+
+sq_status sq_static_act_scale(const float *amax, const float *inv_smooth, int64_t K, float *delta,
+                              sq_stream_t stream) {
+  if (K <= 0 || K >= kMaxDim || !valid_vec(amax) || !valid_vec(inv_smooth)) return SQ_ERR_INVALID_ARG;
+  if (delta == nullptr || (reinterpret_cast<uintptr_t>(delta) & 3u) != 0) return SQ_ERR_INVALID_ARG;
+  return from_cuda(sq::launch_static_scale(amax, inv_smooth, K, delta, (cudaStream_t)stream));
+}
+
+sq_status sq_quant_act_static(const void *x, sq_dtype xt, int64_t M, int64_t K, int64_t ldx, const float *inv_smooth,
+                              const float *delta, int8_t *xq, float *x_scale, sq_stream_t stream) {
+  if (!valid_dtype(xt) || K <= 0 || K % 16 != 0 || K >= kMaxDim || M < 0 || M >= kMaxDim) return SQ_ERR_INVALID_ARG;
+  if (ldx < K || (ldx * dsize(xt)) % 16 != 0) return SQ_ERR_INVALID_ARG;
+  if (!valid_vec(inv_smooth) || delta == nullptr || (reinterpret_cast<uintptr_t>(delta) & 3u) != 0)
+    return SQ_ERR_INVALID_ARG;
+  if (M == 0) return SQ_OK;
+  if (!valid_matrix(x, xt, M, K, ldx) || !valid_vec(xq) || !valid_vec(x_scale)) return SQ_ERR_INVALID_ARG;
+  return from_cuda(sq::launch_quant_static(x, xt, M, K, ldx, inv_smooth, delta, xq, x_scale, (cudaStream_t)stream));
 }
 
 static sq_status gemm_common(const int8_t *xq, const int8_t *wq, int64_t M, int64_t N, int64_t K, const void *y,
@@ -154,9 +217,9 @@ static sq_status gemm_common(const int8_t *xq, const int8_t *wq, int64_t M, int6
   return SQ_OK;
 }
 
-sq_status sq_w8a8_linear(const int8_t *xq, const float *x_scale, const int8_t *wq, const float *w_scale, int64_t M,
-                         int64_t N, int64_t K, void *y, sq_dtype yt, int64_t ldy, void *workspace,
-                         size_t workspace_bytes, sq_stream_t stream) {
+static sq_status linear_impl(const int8_t *xq, const float *x_scale, const int8_t *wq, const float *w_scale,
+                             int64_t M, int64_t N, int64_t K, void *y, sq_dtype yt, int64_t ldy, void *workspace,
+                             size_t workspace_bytes, sq::QFmt fmt, sq_stream_t stream) {
   if (!valid_dtype(yt)) return SQ_ERR_INVALID_ARG;
   if (!valid_vec(w_scale)) return SQ_ERR_INVALID_ARG;
   sq_status s = gemm_common(xq, wq, M, N, K, y, ldy, dsize(yt), workspace, workspace_bytes);
@@ -164,7 +227,30 @@ sq_status sq_w8a8_linear(const int8_t *xq, const float *x_scale, const int8_t *w
   if (!valid_vec(x_scale)) return SQ_ERR_INVALID_ARG;
   const sq::OutKind kind = yt == SQ_F32 ? sq::OutKind::F32 : yt == SQ_F16 ? sq::OutKind::F16 : sq::OutKind::BF16;
   return from_cuda(sq::launch_w8a8_gemm(xq, x_scale, wq, w_scale, M, N, K, y, kind, ldy, workspace,
-                                        workspace_bytes, (cudaStream_t)stream));
+                                        workspace_bytes, (cudaStream_t)stream, fmt));
+}
+
+static sq_status accumulate_impl(const int8_t *xq, const int8_t *wq, int64_t M, int64_t N, int64_t K, void *acc,
+                                 int64_t ldacc, void *workspace, size_t workspace_bytes, sq::QFmt fmt,
+                                 sq_stream_t stream) {
+  sq_status s = gemm_common(xq, wq, M, N, K, acc, ldacc, 4, workspace, workspace_bytes);
+  if (s != SQ_OK || M == 0) return s;
+  return from_cuda(sq::launch_w8a8_gemm(xq, nullptr, wq, nullptr, M, N, K, acc, sq::OutKind::I32, ldacc, workspace,
+                                        workspace_bytes, (cudaStream_t)stream, fmt));
+}
+
+sq_status sq_w8a8_linear(const int8_t *xq, const float *x_scale, const int8_t *wq, const float *w_scale, int64_t M,
+                         int64_t N, int64_t K, void *y, sq_dtype yt, int64_t ldy, void *workspace,
+                         size_t workspace_bytes, sq_stream_t stream) {
+  return linear_impl(xq, x_scale, wq, w_scale, M, N, K, y, yt, ldy, workspace, workspace_bytes, sq::QFmt::I8,
+                     stream);
+}
+
+sq_status sq_w8a8_linear_e4m3(const uint8_t *xq, const float *x_scale, const uint8_t *wq, const float *w_scale,
+                              int64_t M, int64_t N, int64_t K, void *y, sq_dtype yt, int64_t ldy, void *workspace,
+                              size_t workspace_bytes, sq_stream_t stream) {
+  return linear_impl(reinterpret_cast<const int8_t *>(xq), x_scale, reinterpret_cast<const int8_t *>(wq), w_scale,
+                     M, N, K, y, yt, ldy, workspace, workspace_bytes, sq::QFmt::E4M3, stream);
 }
 
 size_t sq_w8a8_linear_workspace_size(int64_t M, int64_t N, int64_t K) {
@@ -174,10 +260,13 @@ size_t sq_w8a8_linear_workspace_size(int64_t M, int64_t N, int64_t K) {
 
 sq_status sq_w8a8_accumulate(const int8_t *xq, const int8_t *wq, int64_t M, int64_t N, int64_t K, int32_t *acc,
                              int64_t ldacc, void *workspace, size_t workspace_bytes, sq_stream_t stream) {
-  sq_status s = gemm_common(xq, wq, M, N, K, acc, ldacc, 4, workspace, workspace_bytes);
-  if (s != SQ_OK || M == 0) return s;
-  return from_cuda(sq::launch_w8a8_gemm(xq, nullptr, wq, nullptr, M, N, K, acc, sq::OutKind::I32, ldacc, workspace,
-                                        workspace_bytes, (cudaStream_t)stream));
+  return accumulate_impl(xq, wq, M, N, K, acc, ldacc, workspace, workspace_bytes, sq::QFmt::I8, stream);
+}
+
+sq_status sq_w8a8_accumulate_e4m3(const uint8_t *xq, const uint8_t *wq, int64_t M, int64_t N, int64_t K, float *acc,
+                                  int64_t ldacc, void *workspace, size_t workspace_bytes, sq_stream_t stream) {
+  return accumulate_impl(reinterpret_cast<const int8_t *>(xq), reinterpret_cast<const int8_t *>(wq), M, N, K, acc,
+                         ldacc, workspace, workspace_bytes, sq::QFmt::E4M3, stream);
 }
 
 sq_status sq_selftest_wait_timeout(int limit_ms, sq_stream_t stream) {

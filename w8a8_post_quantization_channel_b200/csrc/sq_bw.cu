@@ -141,13 +141,14 @@ __global__ void smooth_factor_kernel(const float *__restrict__ amax, float *__re
 // Row quantizer (persistent): each CTA walks rows r = blockIdx.x,
 // blockIdx.x + gridDim.x, ...; per row
 //   v_c = x[r][c] * col_scale[c];  m = max_c |v_c|;
-//   row_scale_out[r] = m / 127;  q[r][c] = rne(v_c * (127 / m)).
+//   row_scale_out[r] = m / Q;  q[r][c] = code(v_c * (Q / m)),
+// Q = F::kMax (127 for INT8 codes, 448 for E4M3).
 // Thread t owns the 16-byte vectors t + i*blockDim (i < kVPT) of every row:
 // their column scales stay in registers for the CTA's lifetime, the next
 // row's vectors are loaded before the current row is reduced, and the row
 // maximum needs one barrier (two alternating reduction slots).
 constexpr int kRowMaxThreads = 512;
-template <typename T, int kVPT>
+template <typename T, int kVPT, typename F>
 __global__ void __launch_bounds__(kRowMaxThreads)
     quant_rows_kernel(const T *__restrict__ x, int64_t rows, int64_t nvec, int64_t ld,
                       const float *__restrict__ col_scale, int8_t *__restrict__ q, float *__restrict__ row_scale_out) {
@@ -204,24 +205,17 @@ __global__ void __launch_bounds__(kRowMaxThreads)
     for (int w = 0; w < nwarps; ++w) m = fmaxf(m, red[slot][w]);
     slot ^= 1;
     // m == 0 (all-zero row): rcp = 0 gives codes 0 and scale 0
-    const float rcp = m > 0.0f ? __fdiv_rn(127.0f, m) : 0.0f;
-    if (tid == 0) row_scale_out[r] = __fdiv_rn(m, 127.0f);
+    const float rcp = m > 0.0f ? __fdiv_rn(F::kMax, m) : 0.0f;
+    if (tid == 0) row_scale_out[r] = __fdiv_rn(m, F::kMax);
     int8_t *qrow = q + r * K;
 #pragma unroll
     for (int i = 0; i < kVPT; ++i) {
       const int64_t v = tid + (int64_t)i * blockDim.x;
       if (v < nvec) {
         if constexpr (V == 8) {
-          uint2 o;
-          o.x = pack4_codes(quantize_dynamic(val[i][0], rcp), quantize_dynamic(val[i][1], rcp),
-                            quantize_dynamic(val[i][2], rcp), quantize_dynamic(val[i][3], rcp));
-          o.y = pack4_codes(quantize_dynamic(val[i][4], rcp), quantize_dynamic(val[i][5], rcp),
-                            quantize_dynamic(val[i][6], rcp), quantize_dynamic(val[i][7], rcp));
-          *reinterpret_cast<uint2 *>(qrow + v * V) = o;
+          *reinterpret_cast<uint2 *>(qrow + v * V) = F::codes8(val[i], rcp);
         } else {
-          *reinterpret_cast<uint32_t *>(qrow + v * V) =
-              pack4_codes(quantize_dynamic(val[i][0], rcp), quantize_dynamic(val[i][1], rcp),
-                          quantize_dynamic(val[i][2], rcp), quantize_dynamic(val[i][3], rcp));
+          *reinterpret_cast<uint32_t *>(qrow + v * V) = F::codes4(val[i], rcp);
         }
       }
     }
@@ -236,7 +230,7 @@ __global__ void __launch_bounds__(kRowMaxThreads)
 // column scales stay in registers; each row is read from shared memory
 // twice (maximum, then codes), so HBM sees every byte once.
 constexpr int kSmemRowThreads = 512;
-template <typename T, int kVPT, int kStages>
+template <typename T, int kVPT, int kStages, typename F>
 __global__ void __launch_bounds__(kSmemRowThreads, 1)
     quant_rows_smem_kernel(const T *__restrict__ x, int64_t rows, int64_t nvec, int64_t ld,
                            const float *__restrict__ col_scale, int8_t *__restrict__ q,
@@ -304,8 +298,8 @@ __global__ void __launch_bounds__(kSmemRowThreads, 1)
 #pragma unroll
     for (int w = 0; w < kSmemRowThreads / 32; ++w) m = fmaxf(m, red[slot * 16 + w]);
     slot ^= 1;
-    const float rcp = m > 0.0f ? __fdiv_rn(127.0f, m) : 0.0f;
-    if (tid == 0) row_scale_out[r] = __fdiv_rn(m, 127.0f);
+    const float rcp = m > 0.0f ? __fdiv_rn(F::kMax, m) : 0.0f;
+    if (tid == 0) row_scale_out[r] = __fdiv_rn(m, F::kMax);
     int8_t *qrow = q + r * K;
 #pragma unroll
     for (int i = 0; i < kVPT; ++i) {
@@ -321,16 +315,9 @@ __global__ void __launch_bounds__(kSmemRowThreads, 1)
           val[e + 1] = p.y;
         }
         if constexpr (V == 8) {
-          uint2 o;
-          o.x = pack4_codes(quantize_dynamic(val[0], rcp), quantize_dynamic(val[1], rcp),
-                            quantize_dynamic(val[2], rcp), quantize_dynamic(val[3], rcp));
-          o.y = pack4_codes(quantize_dynamic(val[4], rcp), quantize_dynamic(val[5], rcp),
-                            quantize_dynamic(val[6], rcp), quantize_dynamic(val[7], rcp));
-          *reinterpret_cast<uint2 *>(qrow + v * V) = o;
+          *reinterpret_cast<uint2 *>(qrow + v * V) = F::codes8(val, rcp);
         } else {
-          *reinterpret_cast<uint32_t *>(qrow + v * V) =
-              pack4_codes(quantize_dynamic(val[0], rcp), quantize_dynamic(val[1], rcp),
-                          quantize_dynamic(val[2], rcp), quantize_dynamic(val[3], rcp));
+          *reinterpret_cast<uint32_t *>(qrow + v * V) = F::codes4(val, rcp);
         }
       }
     }
@@ -353,7 +340,7 @@ __global__ void __launch_bounds__(kSmemRowThreads, 1)
 
 // Row quantizer for rows too long to hold in registers: one pass for the
 // maximum, a second for the codes (the row is re-read, mostly from L2).
-template <typename T>
+template <typename T, typename F>
 __global__ void __launch_bounds__(1024) quant_rows_twopass_kernel(const T *__restrict__ x, int64_t nvec, int64_t ld,
                                                                   const float *__restrict__ col_scale,
                                                                   int8_t *__restrict__ q,
@@ -373,22 +360,19 @@ __global__ void __launch_bounds__(1024) quant_rows_twopass_kernel(const T *__res
     for (int e = 0; e < V; ++e) m = fmaxf(m, fabsf(__fmul_rn(f[e], __ldg(col_scale + v * V + e))));
   }
   m = block_max(m, red);
-  const float rcp = m > 0.0f ? __fdiv_rn(127.0f, m) : 0.0f;
-  if (threadIdx.x == 0) row_scale_out[r] = __fdiv_rn(m, 127.0f);
+  const float rcp = m > 0.0f ? __fdiv_rn(F::kMax, m) : 0.0f;
+  if (threadIdx.x == 0) row_scale_out[r] = __fdiv_rn(m, F::kMax);
   int8_t *qrow = q + r * K;
   for (int64_t v = threadIdx.x; v < nvec; v += blockDim.x) {
     float f[V];
     Vec<T>::to_f32(ld_stream_v4(row + v * V), f);
-    int c[V];
+    float val[V];
 #pragma unroll
-    for (int e = 0; e < V; ++e) c[e] = quantize_dynamic(__fmul_rn(f[e], __ldg(col_scale + v * V + e)), rcp);
+    for (int e = 0; e < V; ++e) val[e] = __fmul_rn(f[e], __ldg(col_scale + v * V + e));
     if constexpr (V == 8) {
-      uint2 o;
-      o.x = pack4_codes(c[0], c[1], c[2], c[3]);
-      o.y = pack4_codes(c[4], c[5], c[6], c[7]);
-      *reinterpret_cast<uint2 *>(qrow + v * V) = o;
+      *reinterpret_cast<uint2 *>(qrow + v * V) = F::codes8(val, rcp);
     } else {
-      *reinterpret_cast<uint32_t *>(qrow + v * V) = pack4_codes(c[0], c[1], c[2], c[3]);
+      *reinterpret_cast<uint32_t *>(qrow + v * V) = F::codes4(val, rcp);
     }
   }
 }
@@ -397,21 +381,21 @@ __global__ void __launch_bounds__(1024) quant_rows_twopass_kernel(const T *__res
 // row-contiguous loads, quantized with its column's maximum, transposed in
 // shared memory and written with row-contiguous stores.
 constexpr int kTT = 64;
-template <typename T>
+template <typename T, typename F>
 __global__ void __launch_bounds__(256) quant_cols_transpose_kernel(const T *__restrict__ w, int64_t K, int64_t N,
                                                                    int64_t ld, const float *__restrict__ s,
                                                                    const float *__restrict__ colmax,
                                                                    int8_t *__restrict__ wq) {
   pdl_wait();  // the previous kernel's results are visible from here on
   pdl_trigger();
-  __shared__ int8_t tile[kTT][kTT + 4];  // [n][j]
+  __shared__ uint8_t tile[kTT][kTT + 4];  // [n][j] codes
   __shared__ float rcp[kTT];
   const int64_t j0 = (int64_t)blockIdx.y * kTT, n0 = (int64_t)blockIdx.x * kTT;
   const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;  // 16 x 16 threads
   if (threadIdx.x < kTT) {
     const int64_t n = n0 + threadIdx.x;
     const float cm = n < N ? __ldg(colmax + n) : 0.0f;
-    rcp[threadIdx.x] = cm > 0.0f ? __fdiv_rn(127.0f, cm) : 0.0f;
+    rcp[threadIdx.x] = cm > 0.0f ? __fdiv_rn(F::kMax, cm) : 0.0f;
   }
   __syncthreads();
   // each thread: 4 consecutive n of one j row, rows ty, ty+16, ...
@@ -419,15 +403,15 @@ __global__ void __launch_bounds__(256) quant_cols_transpose_kernel(const T *__re
   for (int jj = ty; jj < kTT; jj += 16) {
     const int64_t j = j0 + jj;
     const int64_t n = n0 + tx * 4;
-    int c[4] = {0, 0, 0, 0};
+    uint8_t c[4] = {0, 0, 0, 0};
     if (j < K && n < N) {  // N % 16 == 0: a group of 4 is all in or all out
       const float sj = __ldg(s + j);
       const T *p = w + j * ld + n;
 #pragma unroll
-      for (int e = 0; e < 4; ++e) c[e] = quantize(__fmul_rn(sj, Vec<T>::one(p + e)), rcp[tx * 4 + e]);
+      for (int e = 0; e < 4; ++e) c[e] = F::code1(__fmul_rn(sj, Vec<T>::one(p + e)), rcp[tx * 4 + e]);
     }
 #pragma unroll
-    for (int e = 0; e < 4; ++e) tile[tx * 4 + e][jj] = (int8_t)c[e];
+    for (int e = 0; e < 4; ++e) tile[tx * 4 + e][jj] = c[e];
   }
   __syncthreads();
   // write: row n of the tile, 64 bytes of j; each thread 4 bytes
@@ -436,18 +420,19 @@ __global__ void __launch_bounds__(256) quant_cols_transpose_kernel(const T *__re
     const int64_t n = n0 + nn;
     const int64_t j = j0 + tx * 4;
     if (n < N && j < K) {
-      const uint32_t packed = pack4_i8(tile[nn][tx * 4 + 0], tile[nn][tx * 4 + 1], tile[nn][tx * 4 + 2],
-                                       tile[nn][tx * 4 + 3]);
+      const uint32_t packed = (uint32_t)tile[nn][tx * 4 + 0] | ((uint32_t)tile[nn][tx * 4 + 1] << 8) |
+                              ((uint32_t)tile[nn][tx * 4 + 2] << 16) | ((uint32_t)tile[nn][tx * 4 + 3] << 24);
       *reinterpret_cast<uint32_t *>(wq + n * K + j) = packed;
     }
   }
 }
 
+template <typename F>
 __global__ void finalize_scale_kernel(float *__restrict__ m_to_scale, int64_t n) {
   pdl_wait();  // the previous kernel's results are visible from here on
   pdl_trigger();
   const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (i < n) m_to_scale[i] = __fdiv_rn(m_to_scale[i], 127.0f);
+  if (i < n) m_to_scale[i] = __fdiv_rn(m_to_scale[i], F::kMax);
 }
 
 __global__ void zero_fill_kernel(float *__restrict__ p, int64_t n) {
@@ -493,29 +478,29 @@ cudaError_t absmax_rows_t(const void *x, int64_t rows, int64_t cols, int64_t ld,
   return launch_pdl(absmax_rows_kernel<T>, dim3((unsigned)rows), dim3(256), 0, st, 1, (const T *)x, cols / V, ld, out);
 }
 
-template <typename T, int kVPT>
+template <typename T, int kVPT, typename F>
 cudaError_t launch_quant_rows_persistent(const T *x, int64_t rows, int64_t nvec, int64_t ld, const float *col_scale,
                                          int8_t *q, float *row_scale_out, int threads, cudaStream_t st) {
-  static int per_sm[64][5] = {};  // [device][threads / 128]
+  static int per_sm[64][5] = {};  // [device][threads / 128], per instantiation
   int dev = 0;
   cudaGetDevice(&dev);
   int &cached = per_sm[dev & 63][(threads - 1) / 128];
   if (cached == 0) {
     int n = 0;
-    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, quant_rows_kernel<T, kVPT>, threads, 0);
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, quant_rows_kernel<T, kVPT, F>, threads, 0);
     if (e != cudaSuccess) return e;
     cached = n > 0 ? n : 1;
   }
   const int64_t grid = std::min<int64_t>(rows, (int64_t)cached * num_sms());
-  return launch_pdl(quant_rows_kernel<T, kVPT>, dim3((unsigned)grid), dim3(threads), 0, st, 1, x, rows, nvec, ld,
+  return launch_pdl(quant_rows_kernel<T, kVPT, F>, dim3((unsigned)grid), dim3(threads), 0, st, 1, x, rows, nvec, ld,
                     col_scale, q, row_scale_out);
 }
 
-template <typename T, int kVPT, int kStages>
+template <typename T, int kVPT, int kStages, typename F>
 cudaError_t launch_quant_rows_smem(const T *x, int64_t rows, int64_t nvec, int64_t ld, const float *col_scale,
                                    int8_t *q, float *row_scale_out, uint32_t row_bytes, uint32_t smem_bytes,
                                    cudaStream_t st) {
-  auto kern = quant_rows_smem_kernel<T, kVPT, kStages>;
+  auto kern = quant_rows_smem_kernel<T, kVPT, kStages, F>;
   static int attr_bytes[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -529,7 +514,7 @@ cudaError_t launch_quant_rows_smem(const T *x, int64_t rows, int64_t nvec, int64
                     q, row_scale_out, row_bytes, device_error_word());
 }
 
-template <typename T>
+template <typename T, typename F>
 cudaError_t quant_rows_t(const void *x, int64_t rows, int64_t cols, int64_t ld, const float *col_scale, int8_t *q,
                          float *row_scale_out, cudaStream_t st) {
   constexpr int V = Vec<T>::N;
@@ -540,34 +525,34 @@ cudaError_t quant_rows_t(const void *x, int64_t rows, int64_t cols, int64_t ld, 
     return (int)std::max<int64_t>(32, ((t + 31) / 32) * 32);
   };
   if (nvec <= 4 * 32) {
-    return launch_quant_rows_persistent<T, 1>(xp, rows, nvec, ld, col_scale, q, row_scale_out, threads_for(1), st);
+    return launch_quant_rows_persistent<T, 1, F>(xp, rows, nvec, ld, col_scale, q, row_scale_out, threads_for(1), st);
   }
   if (nvec <= 4 * kRowMaxThreads) {
-    return launch_quant_rows_persistent<T, 4>(xp, rows, nvec, ld, col_scale, q, row_scale_out, threads_for(4), st);
+    return launch_quant_rows_persistent<T, 4, F>(xp, rows, nvec, ld, col_scale, q, row_scale_out, threads_for(4), st);
   }
   const uint32_t row_bytes = (uint32_t)(cols * sizeof(T));
   const uint32_t buf = (row_bytes + 127u) & ~127u;
   const uint32_t extra = 128 + 8 * 3 + 2 * 16 * 4 + 16;
   if (nvec <= 8 * kSmemRowThreads && 3 * buf + extra <= 200 * 1024) {
-    return launch_quant_rows_smem<T, 8, 3>(xp, rows, nvec, ld, col_scale, q, row_scale_out, row_bytes,
+    return launch_quant_rows_smem<T, 8, 3, F>(xp, rows, nvec, ld, col_scale, q, row_scale_out, row_bytes,
                                            3 * buf + extra, st);
   }
   if (nvec <= 8 * kSmemRowThreads && 2 * buf + extra <= 220 * 1024) {
-    return launch_quant_rows_smem<T, 8, 2>(xp, rows, nvec, ld, col_scale, q, row_scale_out, row_bytes,
+    return launch_quant_rows_smem<T, 8, 2, F>(xp, rows, nvec, ld, col_scale, q, row_scale_out, row_bytes,
                                            2 * buf + extra, st);
   }
-  return launch_pdl(quant_rows_twopass_kernel<T>, dim3((unsigned)rows), dim3(1024), 0, st, 1, xp, nvec, ld, col_scale,
+  return launch_pdl(quant_rows_twopass_kernel<T, F>, dim3((unsigned)rows), dim3(1024), 0, st, 1, xp, nvec, ld, col_scale,
                     q, row_scale_out);
 }
 
-template <typename T>
+template <typename T, typename F>
 cudaError_t quant_cols_t(const void *w, int64_t K, int64_t N, int64_t ld, const float *s, float *colmax, int8_t *wq,
                          cudaStream_t st) {
   dim3 grid((unsigned)((N + kTT - 1) / kTT), (unsigned)((K + kTT - 1) / kTT));
-  cudaError_t e = launch_pdl(quant_cols_transpose_kernel<T>, grid, dim3(256), 0, st, 1, (const T *)w, K, N, ld, s,
+  cudaError_t e = launch_pdl(quant_cols_transpose_kernel<T, F>, grid, dim3(256), 0, st, 1, (const T *)w, K, N, ld, s,
                              (const float *)colmax, wq);
   if (e != cudaSuccess) return e;
-  return launch_pdl(finalize_scale_kernel, dim3((unsigned)((N + 255) / 256)), dim3(256), 0, st, 1, colmax, N);
+  return launch_pdl(finalize_scale_kernel<F>, dim3((unsigned)((N + 255) / 256)), dim3(256), 0, st, 1, colmax, N);
 }
 
 }  // namespace
@@ -606,22 +591,37 @@ cudaError_t launch_smooth_factor(const float *amax, float *s_inout, float *inv_s
                     K, alpha);
 }
 
-cudaError_t launch_quant_rows(const void *x, sq_dtype xt, int64_t rows, int64_t cols, int64_t ld,
-                              const float *col_scale, int8_t *q, float *row_scale_out, cudaStream_t st) {
+template <typename F>
+cudaError_t quant_rows_fmt(const void *x, sq_dtype xt, int64_t rows, int64_t cols, int64_t ld, const float *col_scale,
+                           int8_t *q, float *row_scale_out, cudaStream_t st) {
   switch (xt) {
-    case SQ_F32: return quant_rows_t<float>(x, rows, cols, ld, col_scale, q, row_scale_out, st);
-    case SQ_F16: return quant_rows_t<__half>(x, rows, cols, ld, col_scale, q, row_scale_out, st);
-    default: return quant_rows_t<__nv_bfloat16>(x, rows, cols, ld, col_scale, q, row_scale_out, st);
+    case SQ_F32: return quant_rows_t<float, F>(x, rows, cols, ld, col_scale, q, row_scale_out, st);
+    case SQ_F16: return quant_rows_t<__half, F>(x, rows, cols, ld, col_scale, q, row_scale_out, st);
+    default: return quant_rows_t<__nv_bfloat16, F>(x, rows, cols, ld, col_scale, q, row_scale_out, st);
+  }
+}
+
+cudaError_t launch_quant_rows(const void *x, sq_dtype xt, int64_t rows, int64_t cols, int64_t ld,
+                              const float *col_scale, int8_t *q, float *row_scale_out, QFmt fmt, cudaStream_t st) {
+  return fmt == QFmt::E4M3 ? quant_rows_fmt<FmtE4M3>(x, xt, rows, cols, ld, col_scale, q, row_scale_out, st)
+                           : quant_rows_fmt<FmtI8>(x, xt, rows, cols, ld, col_scale, q, row_scale_out, st);
+}
+
+template <typename F>
+cudaError_t quant_cols_fmt(const void *w, sq_dtype wt, int64_t K, int64_t N, int64_t ld, const float *s,
+                           float *colmax_to_scale, int8_t *wq, cudaStream_t st) {
+  switch (wt) {
+    case SQ_F32: return quant_cols_t<float, F>(w, K, N, ld, s, colmax_to_scale, wq, st);
+    case SQ_F16: return quant_cols_t<__half, F>(w, K, N, ld, s, colmax_to_scale, wq, st);
+    default: return quant_cols_t<__nv_bfloat16, F>(w, K, N, ld, s, colmax_to_scale, wq, st);
   }
 }
 
 cudaError_t launch_quant_cols_transpose(const void *w, sq_dtype wt, int64_t K, int64_t N, int64_t ld,
-                                        const float *s, float *colmax_to_scale, int8_t *wq, cudaStream_t st) {
-  switch (wt) {
-    case SQ_F32: return quant_cols_t<float>(w, K, N, ld, s, colmax_to_scale, wq, st);
-    case SQ_F16: return quant_cols_t<__half>(w, K, N, ld, s, colmax_to_scale, wq, st);
-    default: return quant_cols_t<__nv_bfloat16>(w, K, N, ld, s, colmax_to_scale, wq, st);
-  }
+                                        const float *s, float *colmax_to_scale, int8_t *wq, QFmt fmt,
+                                        cudaStream_t st) {
+  return fmt == QFmt::E4M3 ? quant_cols_fmt<FmtE4M3>(w, wt, K, N, ld, s, colmax_to_scale, wq, st)
+                           : quant_cols_fmt<FmtI8>(w, wt, K, N, ld, s, colmax_to_scale, wq, st);
 }
 
 }  // namespace sq

@@ -128,9 +128,20 @@ __device__ __forceinline__ uint4 ld_policy_v4(const void *p, uint64_t policy) {
 // The quantizer: clamp(rne(v * r), -127, 127), r = 127 / absmax of the row.
 // __fmul_rn keeps the product a separately rounded IEEE multiply.
 // ---------------------------------------------------------------------------
+// Rounds u to the nearest integer, ties to even, with one exact IEEE
+// addition: for |u| < 2^22, u + 1.5 * 2^23 lies in [2^23, 2^24), where
+// adjacent floats are 1 apart, so the round-to-nearest-even sum equals
+// 1.5 * 2^23 + rne(u) (the shift is even, so ties land on the even integer)
+// and rne(u) sits in the low bits of the sum's encoding: its low byte is
+// the two's-complement int8 code whenever |rne(u)| <= 127.  This keeps the
+// conversion off the float-to-integer unit (one add on the fp32 pipe).
+constexpr float kRneShift = 12582912.0f;  // 1.5 * 2^23
+
+// Clamped code for finite v: clamp(rne(v * r), -127, 127) (clamping before
+// rounding gives the same integer as rounding before clamping).
 __device__ __forceinline__ int quantize(float v, float r) {
-  int q = __float2int_rn(__fmul_rn(v, r));
-  return max(-127, min(127, q));
+  const float u = fminf(fmaxf(__fmul_rn(v, r), -127.0f), 127.0f);
+  return (int)(int8_t)(__float_as_uint(__fadd_rn(u, kRneShift)) & 0xffu);
 }
 
 // Two IEEE fp32 products at once (sm_100 packed fp32 pipe), each rounded
@@ -145,20 +156,82 @@ __device__ __forceinline__ float2 fmul2_rn(float2 a, float2 b) {
 
 // Codes for a row whose scale r = 127/m comes from the row's own absmax m:
 // |v| <= m implies |fl(v*r)| <= fl(m*r) <= 127 + 2^-17, which rounds to at
-// most 127, so the [-127, 127] clamp can never act and rne(v*r) is the code.
-__device__ __forceinline__ int quantize_dynamic(float v, float r) {
-  int q;
-  asm("cvt.rni.s32.f32 %0, %1;" : "=r"(q) : "f"(__fmul_rn(v, r)));
-  return q;
+// most 127, so the [-127, 127] clamp can never act: the low byte of
+// code_word(v, r) is the code.
+__device__ __forceinline__ uint32_t code_word(float v, float r) {
+  return __float_as_uint(__fadd_rn(__fmul_rn(v, r), kRneShift));
 }
 
-// Packs four codes in [-127, 127] into bytes 0..3 of a word.
-__device__ __forceinline__ uint32_t pack4_codes(int q0, int q1, int q2, int q3) {
-  uint32_t hi, out;
-  asm("cvt.pack.sat.s8.s32.b32 %0, %1, %2, 0;" : "=r"(hi) : "r"(q3), "r"(q2));
-  asm("cvt.pack.sat.s8.s32.b32 %0, %1, %2, %3;" : "=r"(out) : "r"(q1), "r"(q0), "r"(hi));
-  return out;
+// Two code words: the products on the packed fp32 pipe, the shifts as
+// scalar __fadd_rn, which is never contracted with the multiply into an
+// fma (a fused multiply-add would round the exact product directly and
+// break ties that the rounded product sits on).
+__device__ __forceinline__ uint2 code_word2(float v0, float v1, float r) {
+  const float2 p = fmul2_rn(make_float2(v0, v1), make_float2(r, r));
+  return make_uint2(__float_as_uint(__fadd_rn(p.x, kRneShift)), __float_as_uint(__fadd_rn(p.y, kRneShift)));
 }
+
+// Bytes 0..3 of the result are the low bytes of a, b, c, d.
+__device__ __forceinline__ uint32_t pack4_low(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040), 0x5410);
+}
+
+// Eight code words of one 16-byte row vector, packed into 8 bytes.
+__device__ __forceinline__ uint2 codes8(const float *v, float r) {
+  const uint2 a = code_word2(v[0], v[1], r), b = code_word2(v[2], v[3], r);
+  const uint2 c = code_word2(v[4], v[5], r), d = code_word2(v[6], v[7], r);
+  return make_uint2(pack4_low(a.x, a.y, b.x, b.y), pack4_low(c.x, c.y, d.x, d.y));
+}
+__device__ __forceinline__ uint32_t codes4(const float *v, float r) {
+  const uint2 a = code_word2(v[0], v[1], r), b = code_word2(v[2], v[3], r);
+  return pack4_low(a.x, a.y, b.x, b.y);
+}
+
+// Two fp32 values to two E4M3 codes (round to nearest even, saturating at
+// +-448): lo in bits 0-7, hi in bits 8-15.
+__device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
+  uint16_t d;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(d) : "f"(hi), "f"(lo));
+  return d;
+}
+
+// Code formats of the quantizers.  kMax is the code magnitude a row's
+// absmax maps to (scale = absmax / kMax, multiplier kMax / absmax).
+//   FmtI8    symmetric INT8, codes in [-127, 127]
+//   FmtE4M3  FP8 E4M3 codes, values in [-448, 448]
+// codes8 / codes4 quantize one 16- or 8-byte row vector's values v with
+// multiplier r; code1 one value (with saturation).
+struct FmtI8 {
+  static constexpr float kMax = 127.0f;
+  static __device__ __forceinline__ uint2 codes8(const float *v, float r) { return sq::codes8(v, r); }
+  static __device__ __forceinline__ uint32_t codes4(const float *v, float r) { return sq::codes4(v, r); }
+  static __device__ __forceinline__ uint8_t code1(float v, float r) { return (uint8_t)(int8_t)quantize(v, r); }
+};
+struct FmtE4M3 {
+  static constexpr float kMax = 448.0f;
+  // r == 0 only for an all-zero row, whose codes are +0 (not the signed
+  // zeros that v * 0 would give)
+  static __device__ __forceinline__ uint2 codes8(const float *v, float r) {
+    if (r == 0.0f) return make_uint2(0u, 0u);
+    float p[8];
+#pragma unroll
+    for (int e = 0; e < 8; e += 2) {
+      const float2 q = fmul2_rn(make_float2(v[e], v[e + 1]), make_float2(r, r));
+      p[e] = q.x;
+      p[e + 1] = q.y;
+    }
+    return make_uint2(e4m3x2(p[0], p[1]) | (e4m3x2(p[2], p[3]) << 16), e4m3x2(p[4], p[5]) | (e4m3x2(p[6], p[7]) << 16));
+  }
+  static __device__ __forceinline__ uint32_t codes4(const float *v, float r) {
+    if (r == 0.0f) return 0u;
+    const float2 a = fmul2_rn(make_float2(v[0], v[1]), make_float2(r, r));
+    const float2 b = fmul2_rn(make_float2(v[2], v[3]), make_float2(r, r));
+    return e4m3x2(a.x, a.y) | (e4m3x2(b.x, b.y) << 16);
+  }
+  static __device__ __forceinline__ uint8_t code1(float v, float r) {
+    return r == 0.0f ? (uint8_t)0 : (uint8_t)(e4m3x2(__fmul_rn(v, r), 0.0f) & 0xffu);
+  }
+};
 
 __device__ __forceinline__ uint32_t pack4_i8(int a, int b, int c, int d) {
   return (uint32_t)(a & 0xff) | ((uint32_t)(b & 0xff) << 8) | ((uint32_t)(c & 0xff) << 16) |
@@ -453,6 +526,60 @@ __device__ __forceinline__ uint64_t desc_sw128_kmajor(uint32_t saddr) {
 // M>>4 at bits 24-28.
 __host__ __device__ constexpr uint32_t idesc_i8(int m, int n) {
   return (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
+}
+
+// Instruction descriptor for kind::f8f6f4 with E4M3 A and B (format code 0
+// at bits 7-9 and 10-12) and an f32 accumulator (bits 4-5 = 1); the other
+// fields as idesc_i8.
+__host__ __device__ constexpr uint32_t idesc_e4m3(int m, int n) {
+  return (1u << 4) | (0u << 7) | (0u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
+}
+
+// 8-bit operands: INT8 (s32 accumulator) or, with F8, E4M3 (f32 accumulator).
+template <bool F8>
+__host__ __device__ constexpr uint32_t idesc8(int m, int n) {
+  return F8 ? idesc_e4m3(m, n) : idesc_i8(m, n);
+}
+
+template <bool F8>
+__device__ __forceinline__ void umma8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                      uint32_t accumulate) {
+  if constexpr (F8) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+  } else {
+    umma_i8(d_tmem, adesc, bdesc, idesc, accumulate);
+  }
+}
+
+template <bool F8>
+__device__ __forceinline__ void umma8_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                           uint32_t accumulate) {
+  if constexpr (F8) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+  } else {
+    umma_i8_pair(d_tmem, adesc, bdesc, idesc, accumulate);
+  }
+}
+
+// The accumulator's 32 bits as a float: an int32 sum (INT8) converted with
+// round to nearest even, or the f32 sum itself (E4M3).
+template <bool F8>
+__device__ __forceinline__ float acc_value(uint32_t bits) {
+  if constexpr (F8) {
+    return __uint_as_float(bits);
+  } else {
+    return __int2float_rn((int)bits);
+  }
 }
 
 }  // namespace sq

@@ -49,7 +49,7 @@ struct GemmSmem {
   static constexpr uint32_t kTmemCols = 2 * BN;
 };
 
-template <OutKind KIND>
+template <OutKind KIND, bool F8>
 __device__ __forceinline__ void store_chunk(const uint32_t (&r)[32], void *y, int64_t ldy, int row, int n0, int N,
                                             float dx, const float *__restrict__ w_scale) {
   // N % 16 == 0 and n0 % 32 == 0, so a chunk has 16 or 32 valid columns.
@@ -66,10 +66,10 @@ __device__ __forceinline__ void store_chunk(const uint32_t (&r)[32], void *y, in
     for (int g = 0; g < 8; ++g) {
       if (g / 4 < groups16) {
         const float4 dw = __ldg(reinterpret_cast<const float4 *>(w_scale + n0) + g);
-        v[4 * g + 0] = __fmul_rn(__fmul_rn(__int2float_rn((int)r[4 * g + 0]), dx), dw.x);
-        v[4 * g + 1] = __fmul_rn(__fmul_rn(__int2float_rn((int)r[4 * g + 1]), dx), dw.y);
-        v[4 * g + 2] = __fmul_rn(__fmul_rn(__int2float_rn((int)r[4 * g + 2]), dx), dw.z);
-        v[4 * g + 3] = __fmul_rn(__fmul_rn(__int2float_rn((int)r[4 * g + 3]), dx), dw.w);
+        v[4 * g + 0] = __fmul_rn(__fmul_rn(acc_value<F8>(r[4 * g + 0]), dx), dw.x);
+        v[4 * g + 1] = __fmul_rn(__fmul_rn(acc_value<F8>(r[4 * g + 1]), dx), dw.y);
+        v[4 * g + 2] = __fmul_rn(__fmul_rn(acc_value<F8>(r[4 * g + 2]), dx), dw.z);
+        v[4 * g + 3] = __fmul_rn(__fmul_rn(acc_value<F8>(r[4 * g + 3]), dx), dw.w);
       } else {
         v[4 * g + 0] = v[4 * g + 1] = v[4 * g + 2] = v[4 * g + 3] = 0.0f;
       }
@@ -101,7 +101,7 @@ __device__ __forceinline__ void store_chunk(const uint32_t (&r)[32], void *y, in
   }
 }
 
-template <int BN, int STAGES, OutKind KIND>
+template <int BN, int STAGES, OutKind KIND, bool F8>
 __global__ void __launch_bounds__(kThreads, 1)
     w8a8_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                         const float *__restrict__ x_scale, const float *__restrict__ w_scale, void *__restrict__ y,
@@ -185,7 +185,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       // ---------------- MMA issuer ----------------
-      constexpr uint32_t idesc = idesc_i8(kBM, BN);
+      constexpr uint32_t idesc = idesc8<F8>(kBM, BN);
       uint32_t stage = 0, phase = 0, ab = 0, aphase = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
@@ -202,7 +202,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t b0 = desc_sw128_kmajor(smem_u32(sB + stage * L::kB));
 #pragma unroll
           for (int k = 0; k < kBK / 32; ++k)  // 32 int8 = 32 bytes = +2 in the >>4 address field
-            umma_i8(d, a0 + 2 * k, b0 + 2 * k, idesc, (kb | k) != 0 ? 1u : 0u);
+            umma8<F8>(d, a0 + 2 * k, b0 + 2 * k, idesc, (kb | k) != 0 ? 1u : 0u);
           umma_commit(&empty[stage]);
           if (++stage == STAGES) {
             stage = 0;
@@ -237,7 +237,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + ab * BN + c * 32, r);
         tmem_ld_wait();
         const int n0 = nb * BN + c * 32;
-        if (row_ok && n0 < N) store_chunk<KIND>(r, y, ldy, row, n0, N, dx, w_scale);
+        if (row_ok && n0 < N) store_chunk<KIND, F8>(r, y, ldy, row, n0, N, dx, w_scale);
       }
       tc_fence_before();
       __syncwarp();
@@ -278,7 +278,7 @@ struct PairSmem {
   static constexpr uint32_t kTmemCols = 2 * kPairBN;  // two 256-column accumulators
 };
 
-template <int STAGES, OutKind KIND>
+template <int STAGES, OutKind KIND, bool F8>
 __global__ void __launch_bounds__(kThreads, 1)
     w8a8_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                           const float *__restrict__ x_scale, const float *__restrict__ w_scale,
@@ -370,7 +370,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     if (lane == 0 && leader) {
       // ---------------- MMA issuer (leader CTA) ----------------
-      constexpr uint32_t idesc = idesc_i8(2 * kBM, kPairBN);
+      constexpr uint32_t idesc = idesc8<F8>(2 * kBM, kPairBN);
       uint32_t stage = 0, phase = 0, ab = 0, aphase = 0;
       bool ok = true;
       for (int tile = pair; tile < tiles && ok; tile += npairs) {
@@ -386,7 +386,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t a0 = desc_sw128_kmajor(smem_u32(sA + stage * L::kA));
           const uint64_t b0 = desc_sw128_kmajor(smem_u32(sB + stage * L::kB));
 #pragma unroll
-          for (int k = 0; k < kBK / 32; ++k) umma_i8_pair(d, a0 + 2 * k, b0 + 2 * k, idesc, (kb | k) != 0 ? 1u : 0u);
+          for (int k = 0; k < kBK / 32; ++k) umma8_pair<F8>(d, a0 + 2 * k, b0 + 2 * k, idesc, (kb | k) != 0 ? 1u : 0u);
           const uint32_t e = smem_u32(&empty[stage]);
           umma_commit_pair(mapa_shared(e, 0));
           umma_commit_pair(mapa_shared(e, 1));
@@ -425,7 +425,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + ab * kPairBN + c * 32, r);
         tmem_ld_wait();
         const int n0 = nb * kPairBN + c * 32;
-        if (row_ok && n0 < N) store_chunk<KIND>(r, y, ldy, row, n0, N, dx, w_scale);
+        if (row_ok && n0 < N) store_chunk<KIND, F8>(r, y, ldy, row, n0, N, dx, w_scale);
       }
       tc_fence_before();
       __syncwarp();
@@ -473,12 +473,12 @@ struct DecSmem {
   static constexpr uint32_t kTmemCols = (2 * MP <= 32) ? 32 : (2 * MP <= 64) ? 64 : 128;
 };
 
-template <OutKind KIND>
-__device__ __forceinline__ void store_one(void *y, int64_t ldy, int t, int n, int32_t acc, float dx, float dw) {
+template <OutKind KIND, bool F8>
+__device__ __forceinline__ void store_one(void *y, int64_t ldy, int t, int n, uint32_t acc, float dx, float dw) {
   if constexpr (KIND == OutKind::I32) {
-    reinterpret_cast<int32_t *>(y)[(int64_t)t * ldy + n] = acc;
+    reinterpret_cast<uint32_t *>(y)[(int64_t)t * ldy + n] = acc;  // the raw accumulator
   } else {
-    const float v = __fmul_rn(__fmul_rn(__int2float_rn(acc), dx), dw);
+    const float v = __fmul_rn(__fmul_rn(acc_value<F8>(acc), dx), dw);
     if constexpr (KIND == OutKind::F32) {
       reinterpret_cast<float *>(y)[(int64_t)t * ldy + n] = v;
     } else if constexpr (KIND == OutKind::BF16) {
@@ -489,7 +489,7 @@ __device__ __forceinline__ void store_one(void *y, int64_t ldy, int t, int n, in
   }
 }
 
-template <int MP, OutKind KIND>
+template <int MP, OutKind KIND, bool F8>
 __global__ void __launch_bounds__(kThreads, 1)
     w8a8_gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                             const float *__restrict__ x_scale, const float *__restrict__ w_scale,
@@ -572,7 +572,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       // ---------------- MMA issuer: one accumulation per segment ----------------
-      constexpr uint32_t idesc = idesc_i8(kDecRows, MP);
+      constexpr uint32_t idesc = idesc8<F8>(kDecRows, MP);
       uint32_t stage = 0, phase = 0, ab = 0, aphase = 0;
       bool ok = true;
       for (int64_t w = w0; w < w1 && ok;) {
@@ -592,7 +592,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t b0 = desc_sw128_kmajor(smem_u32(st + L::kW));
 #pragma unroll
           for (int k = 0; k < kBK / 32; ++k)
-            umma_i8(d, a0 + 2 * k, b0 + 2 * k, idesc, (i != w || k != 0) ? 1u : 0u);
+            umma8<F8>(d, a0 + 2 * k, b0 + 2 * k, idesc, (i != w || k != 0) ? 1u : 0u);
           umma_commit(&empty[stage]);
           if (++stage == L::kStages) {
             stage = 0;
@@ -637,9 +637,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (t < M && n_ok) {
             if (whole) {
               const float dx = KIND != OutKind::I32 ? __ldg(x_scale + t) : 0.0f;
-              store_one<KIND>(y, ldy, t, n, (int32_t)r[j], dx, dw);
+              store_one<KIND, F8>(y, ldy, t, n, r[j], dx, dw);
             } else if (r[j] != 0u) {
-              atomicAdd(ws + (int64_t)t * N + n, (int32_t)r[j]);
+              // int32 sums are exact in any order; an f32 tile here has at
+              // most two contributors (each CTA's share spans >= one tile's
+              // k-blocks when tiles outnumber CTAs), and 0 + a + b rounds
+              // the same in either order
+              if constexpr (F8) {
+                atomicAdd(reinterpret_cast<float *>(ws) + (int64_t)t * N + n, __uint_as_float(r[j]));
+              } else {
+                atomicAdd(ws + (int64_t)t * N + n, (int32_t)r[j]);
+              }
             }
           }
         }
@@ -663,15 +671,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             // loads, then dequantize, store, and leave the workspace zero
 #pragma unroll 1
             for (int t0 = 0; t0 < M; t0 += 16) {
-              int32_t acc[16];
+              uint32_t acc[16];
 #pragma unroll
-              for (int j = 0; j < 16; ++j) acc[j] = t0 + j < M ? __ldcg(ws + (int64_t)(t0 + j) * N + n) : 0;
+              for (int j = 0; j < 16; ++j)
+                acc[j] = t0 + j < M ? (uint32_t)__ldcg(ws + (int64_t)(t0 + j) * N + n) : 0u;
 #pragma unroll
               for (int j = 0; j < 16; ++j) {
                 const int t = t0 + j;
                 if (t < M) {
                   const float dx = KIND != OutKind::I32 ? __ldg(x_scale + t) : 0.0f;
-                  store_one<KIND>(y, ldy, t, n, acc[j], dx, dw);
+                  store_one<KIND, F8>(y, ldy, t, n, acc[j], dx, dw);
                   __stcg(ws + (int64_t)t * N + n, 0);
                 }
               }
@@ -705,7 +714,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 // and CTA c sums rows [c 128 / S, (c+1) 128 / S) over all S partials and
 // dequantizes them.  No workspace, no global atomics, no fences.
 // ---------------------------------------------------------------------------
-template <int MP, OutKind KIND>
+template <int MP, OutKind KIND, bool F8>
 __global__ void __launch_bounds__(kThreads, 1)
     w8a8_gemm_decode_cluster_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                                     const float *__restrict__ x_scale, const float *__restrict__ w_scale,
@@ -721,7 +730,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
   // after the MMAs have drained the ring, it holds this CTA's partial sums
   // as part[t][row] (t < MP, row < 128)
-  int32_t *part = reinterpret_cast<int32_t *>(smem);
+  uint32_t *part = reinterpret_cast<uint32_t *>(smem);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
@@ -787,7 +796,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_i8(kDecRows, MP);
+      constexpr uint32_t idesc = idesc8<F8>(kDecRows, MP);
       uint32_t stage = 0, phase = 0;
       for (int i = 0; i < cnt; ++i) {
         if (!mbar_wait(&full[stage], phase, abort_flag, err)) break;
@@ -797,7 +806,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint64_t b0 = desc_sw128_kmajor(smem_u32(st + L::kW));
 #pragma unroll
         for (int k = 0; k < kBK / 32; ++k)
-          umma_i8(tmem_base, a0 + 2 * k, b0 + 2 * k, idesc, (i != 0 || k != 0) ? 1u : 0u);
+          umma8<F8>(tmem_base, a0 + 2 * k, b0 + 2 * k, idesc, (i != 0 || k != 0) ? 1u : 0u);
         umma_commit(&empty[stage]);
         if (++stage == L::kStages) {
           stage = 0;
@@ -833,11 +842,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
         const int t = c * 16 + j;
-        const int32_t v = have ? (int32_t)r[j] : 0;
+        const uint32_t v = have ? r[j] : 0u;
         if (whole) {
           if (t < M && n_ok) {
             const float dx = KIND != OutKind::I32 ? __ldg(x_scale + t) : 0.0f;
-            store_one<KIND>(y, ldy, t, n, v, dx, dw);
+            store_one<KIND, F8>(y, ldy, t, n, v, dx, dw);
           }
         } else {
           part[t * kDecRows + row] = v;
@@ -856,7 +865,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       // issued together, so a round costs about one latency per peer
       for (int base = threadIdx.x - 64; base < items; base += 4 * 128) {
         uint32_t off[4];
-        int32_t sum[4] = {0, 0, 0, 0};
+        // int32 sums, or (E4M3) f32 sums taken in peer order
+        uint32_t sum[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
         for (int b = 0; b < 4; ++b) {
           const int idx = base + b * 128;
@@ -867,7 +877,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int p = 0; p < S; ++p) {
 #pragma unroll
           for (int b = 0; b < 4; ++b)
-            if (base + b * 128 < items) sum[b] += (int32_t)ld_shared_cluster_u32(mapa_shared(off[b], (uint32_t)p));
+            if (base + b * 128 < items) {
+              const uint32_t pv = ld_shared_cluster_u32(mapa_shared(off[b], (uint32_t)p));
+              if constexpr (F8) {
+                sum[b] = __float_as_uint(__fadd_rn(__uint_as_float(sum[b]), __uint_as_float(pv)));
+              } else {
+                sum[b] += pv;
+              }
+            }
         }
 #pragma unroll
         for (int b = 0; b < 4; ++b) {
@@ -878,7 +895,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (n < N) {
               const float dx = KIND != OutKind::I32 ? __ldg(x_scale + t) : 0.0f;
               const float dw = KIND != OutKind::I32 ? __ldg(w_scale + n) : 0.0f;
-              store_one<KIND>(y, ldy, t, n, sum[b], dx, dw);
+              store_one<KIND, F8>(y, ldy, t, n, sum[b], dx, dw);
             }
           }
         }
@@ -925,11 +942,11 @@ bool make_tmap_i8(CUtensorMap *m, const int8_t *base, int64_t rows, int64_t cols
   return r == CUDA_SUCCESS;
 }
 
-template <int BN, int STAGES, OutKind KIND>
+template <int BN, int STAGES, OutKind KIND, bool F8>
 cudaError_t launch_tc(const CUtensorMap &tmA, const CUtensorMap &tmB, const float *x_scale, const float *w_scale,
                       void *y, int64_t ldy, int M, int N, int K, cudaStream_t st) {
   using L = GemmSmem<BN, STAGES>;
-  auto kern = w8a8_gemm_tc_kernel<BN, STAGES, KIND>;
+  auto kern = w8a8_gemm_tc_kernel<BN, STAGES, KIND, F8>;
   static bool attr_set[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -944,11 +961,11 @@ cudaError_t launch_tc(const CUtensorMap &tmA, const CUtensorMap &tmB, const floa
                     device_error_word());
 }
 
-template <int STAGES, OutKind KIND>
+template <int STAGES, OutKind KIND, bool F8>
 cudaError_t launch_pair(const CUtensorMap &tmA, const CUtensorMap &tmB, const float *x_scale, const float *w_scale,
                         void *y, int64_t ldy, int M, int N, int K, int max_clusters, cudaStream_t st) {
   using L = PairSmem<STAGES>;
-  auto kern = w8a8_gemm_pair_kernel<STAGES, KIND>;
+  auto kern = w8a8_gemm_pair_kernel<STAGES, KIND, F8>;
   const int tiles = ((M + 2 * kBM - 1) / (2 * kBM)) * ((N + kPairBN - 1) / kPairBN);
   const int clusters = tiles < max_clusters ? tiles : max_clusters;
   return launch_pdl(kern, dim3(2 * clusters), dim3(kThreads), L::kTotal, st, 2, tmA, tmB, x_scale, w_scale, y, ldy, M,
@@ -956,7 +973,7 @@ cudaError_t launch_pair(const CUtensorMap &tmA, const CUtensorMap &tmB, const fl
 }
 
 // Clusters of two 1-CTA-per-SM blocks that fit on the device at once.
-template <int STAGES, OutKind KIND>
+template <int STAGES, OutKind KIND, bool F8>
 int pair_capacity() {
   using L = PairSmem<STAGES>;
   static int cache[64] = {};
@@ -964,7 +981,7 @@ int pair_capacity() {
   cudaGetDevice(&dev);
   int &c = cache[dev & 63];
   if (c == 0) {
-    auto kern = w8a8_gemm_pair_kernel<STAGES, KIND>;
+    auto kern = w8a8_gemm_pair_kernel<STAGES, KIND, F8>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::kTotal) != cudaSuccess)
       return -1;
     cudaLaunchConfig_t cfg = {};
@@ -987,14 +1004,14 @@ int pair_capacity() {
 
 constexpr int kPairStages = 7;
 
-template <int MP, OutKind KIND>
+template <int MP, OutKind KIND, bool F8>
 void prepare_decode_cluster_kernel() {
   using L = DecSmem<MP>;
   static bool done[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (!done[dev & 63]) {
-    auto kern = w8a8_gemm_decode_cluster_kernel<MP, KIND>;
+    auto kern = w8a8_gemm_decode_cluster_kernel<MP, KIND, F8>;
     cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::kTotal);
     cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     done[dev & 63] = true;
@@ -1003,7 +1020,7 @@ void prepare_decode_cluster_kernel() {
 
 // Clusters of S one-CTA-per-SM blocks of the decode cluster kernel that can
 // be resident at once (0 if none or the query fails).
-template <int MP, OutKind KIND>
+template <int MP, OutKind KIND, bool F8>
 int cluster_capacity(int S) {
   using L = DecSmem<MP>;
   static int cache[64][5] = {};  // [device][log2 S]
@@ -1013,7 +1030,7 @@ int cluster_capacity(int S) {
   while ((1 << lg) < S) ++lg;
   int &c = cache[dev & 63][lg];
   if (c == 0) {
-    prepare_decode_cluster_kernel<MP, KIND>();
+    prepare_decode_cluster_kernel<MP, KIND, F8>();
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(S, 1, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);
@@ -1026,7 +1043,7 @@ int cluster_capacity(int S) {
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, w8a8_gemm_decode_cluster_kernel<MP, KIND>, &cfg) != cudaSuccess) {
+    if (cudaOccupancyMaxActiveClusters(&n, w8a8_gemm_decode_cluster_kernel<MP, KIND, F8>, &cfg) != cudaSuccess) {
       cudaGetLastError();  // clear the query's error
       n = -1;
     }
@@ -1035,21 +1052,21 @@ int cluster_capacity(int S) {
   return c > 0 ? c : 0;
 }
 
-template <int MP, OutKind KIND>
+template <int MP, OutKind KIND, bool F8>
 cudaError_t launch_decode_cluster(const CUtensorMap &tmW, const CUtensorMap &tmX, const float *x_scale,
                                   const float *w_scale, int M, int N, int K, void *y, int64_t ldy, int nt, int S,
                                   cudaStream_t st) {
   using L = DecSmem<MP>;
-  prepare_decode_cluster_kernel<MP, KIND>();
-  return launch_pdl(w8a8_gemm_decode_cluster_kernel<MP, KIND>, dim3(nt * S), dim3(kThreads), L::kTotal, st,
+  prepare_decode_cluster_kernel<MP, KIND, F8>();
+  return launch_pdl(w8a8_gemm_decode_cluster_kernel<MP, KIND, F8>, dim3(nt * S), dim3(kThreads), L::kTotal, st,
                     (unsigned)S, tmW, tmX, x_scale, w_scale, y, ldy, M, N, K, S, device_error_word());
 }
 
-template <int MP, OutKind KIND>
+template <int MP, OutKind KIND, bool F8>
 cudaError_t launch_decode(const int8_t *xq, const float *x_scale, const int8_t *wq, const float *w_scale, int M,
                           int N, int K, void *y, int64_t ldy, void *workspace, cudaStream_t st) {
   using L = DecSmem<MP>;
-  auto kern = w8a8_gemm_decode_kernel<MP, KIND>;
+  auto kern = w8a8_gemm_decode_kernel<MP, KIND, F8>;
   static bool attr_set[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -1066,8 +1083,8 @@ cudaError_t launch_decode(const int8_t *xq, const float *x_scale, const int8_t *
     // one wave of tiles: split K across a cluster of S CTAs per tile
     int S = 1;
     for (int cand = 2; cand <= 16; cand *= 2)
-      if (cand <= nk && (int64_t)nt * cand <= num_sms() && cluster_capacity<MP, KIND>(cand) >= nt) S = cand;
-    return launch_decode_cluster<MP, KIND>(tmW, tmX, x_scale, w_scale, M, N, K, y, ldy, nt, S, st);
+      if (cand <= nk && (int64_t)nt * cand <= num_sms() && cluster_capacity<MP, KIND, F8>(cand) >= nt) S = cand;
+    return launch_decode_cluster<MP, KIND, F8>(tmW, tmX, x_scale, w_scale, M, N, K, y, ldy, nt, S, st);
   }
   const int64_t items = (int64_t)nt * nk;
   const int grid = (int)(items < num_sms() ? items : num_sms());
@@ -1077,34 +1094,34 @@ return launch_pdl(kern, dim3(grid), dim3(kThreads), L::kTotal, st, 1, tmW, tmX, 
                     ws, counts, device_error_word());
 }
 
-template <OutKind KIND>
+template <OutKind KIND, bool F8>
 cudaError_t gemm_dispatch(const int8_t *xq, const float *x_scale, const int8_t *wq, const float *w_scale, int M,
                           int N, int K, void *y, int64_t ldy, void *workspace, cudaStream_t st) {
   if (M <= kDecodeMaxM) {  // weight-streaming regime
-    if (M <= 16) return launch_decode<16, KIND>(xq, x_scale, wq, w_scale, M, N, K, y, ldy, workspace, st);
-    if (M <= 32) return launch_decode<32, KIND>(xq, x_scale, wq, w_scale, M, N, K, y, ldy, workspace, st);
-    if (M <= 48) return launch_decode<48, KIND>(xq, x_scale, wq, w_scale, M, N, K, y, ldy, workspace, st);
-    return launch_decode<64, KIND>(xq, x_scale, wq, w_scale, M, N, K, y, ldy, workspace, st);
+    if (M <= 16) return launch_decode<16, KIND, F8>(xq, x_scale, wq, w_scale, M, N, K, y, ldy, workspace, st);
+    if (M <= 32) return launch_decode<32, KIND, F8>(xq, x_scale, wq, w_scale, M, N, K, y, ldy, workspace, st);
+    if (M <= 48) return launch_decode<48, KIND, F8>(xq, x_scale, wq, w_scale, M, N, K, y, ldy, workspace, st);
+    return launch_decode<64, KIND, F8>(xq, x_scale, wq, w_scale, M, N, K, y, ldy, workspace, st);
   }
   const int sms = num_sms();
   CUtensorMap tmA, tmB;
   // CTA pairs once there are enough 256 x 256 tiles to occupy every pair
   const int tiles_pair = ((M + 255) / 256) * ((N + 255) / 256);
-  const int cap = pair_capacity<kPairStages, KIND>();
+  const int cap = pair_capacity<kPairStages, KIND, F8>();
   if (cap > 0 && tiles_pair >= cap) {
     if (!make_tmap_i8(&tmA, xq, M, K, kBM)) return cudaErrorInvalidValue;
     if (!make_tmap_i8(&tmB, wq, N, K, kPairBN / 2)) return cudaErrorInvalidValue;
-    return launch_pair<kPairStages, KIND>(tmA, tmB, x_scale, w_scale, y, ldy, M, N, K, cap, st);
+    return launch_pair<kPairStages, KIND, F8>(tmA, tmB, x_scale, w_scale, y, ldy, M, N, K, cap, st);
   }
   const int tiles256 = ((M + kBM - 1) / kBM) * ((N + 255) / 256);
   const bool wide = tiles256 >= sms || (N % 256 == 0 && tiles256 * 2 > sms);
   if (!make_tmap_i8(&tmA, xq, M, K, kBM)) return cudaErrorInvalidValue;
   if (wide) {
     if (!make_tmap_i8(&tmB, wq, N, K, 256)) return cudaErrorInvalidValue;
-    return launch_tc<256, 4, KIND>(tmA, tmB, x_scale, w_scale, y, ldy, M, N, K, st);
+    return launch_tc<256, 4, KIND, F8>(tmA, tmB, x_scale, w_scale, y, ldy, M, N, K, st);
   }
   if (!make_tmap_i8(&tmB, wq, N, K, 128)) return cudaErrorInvalidValue;
-  return launch_tc<128, 6, KIND>(tmA, tmB, x_scale, w_scale, y, ldy, M, N, K, st);
+  return launch_tc<128, 6, KIND, F8>(tmA, tmB, x_scale, w_scale, y, ldy, M, N, K, st);
 }
 
 }  // namespace
@@ -1114,16 +1131,23 @@ size_t w8a8_workspace_bytes(int64_t M, int64_t N, int64_t) {
   return decode_ws_elems(M, N) * 4 + decode_counter_bytes(N);
 }
 
+template <bool F8>
+cudaError_t gemm_kind(const int8_t *xq, const float *x_scale, const int8_t *wq, const float *w_scale, int m, int n,
+                      int k, void *y, OutKind kind, int64_t ldy, void *ws, cudaStream_t st) {
+  switch (kind) {
+    case OutKind::F32: return gemm_dispatch<OutKind::F32, F8>(xq, x_scale, wq, w_scale, m, n, k, y, ldy, ws, st);
+    case OutKind::F16: return gemm_dispatch<OutKind::F16, F8>(xq, x_scale, wq, w_scale, m, n, k, y, ldy, ws, st);
+    case OutKind::BF16: return gemm_dispatch<OutKind::BF16, F8>(xq, x_scale, wq, w_scale, m, n, k, y, ldy, ws, st);
+    default: return gemm_dispatch<OutKind::I32, F8>(xq, nullptr, wq, nullptr, m, n, k, y, ldy, ws, st);
+  }
+}
+
 cudaError_t launch_w8a8_gemm(const int8_t *xq, const float *x_scale, const int8_t *wq, const float *w_scale,
                              int64_t M, int64_t N, int64_t K, void *y, OutKind kind, int64_t ldy, void *ws, size_t,
-                             cudaStream_t st) {
+                             cudaStream_t st, QFmt fmt) {
   const int m = (int)M, n = (int)N, k = (int)K;
-  switch (kind) {
-    case OutKind::F32: return gemm_dispatch<OutKind::F32>(xq, x_scale, wq, w_scale, m, n, k, y, ldy, ws, st);
-    case OutKind::F16: return gemm_dispatch<OutKind::F16>(xq, x_scale, wq, w_scale, m, n, k, y, ldy, ws, st);
-    case OutKind::BF16: return gemm_dispatch<OutKind::BF16>(xq, x_scale, wq, w_scale, m, n, k, y, ldy, ws, st);
-    default: return gemm_dispatch<OutKind::I32>(xq, nullptr, wq, nullptr, m, n, k, y, ldy, ws, st);
-  }
+  if (fmt == QFmt::E4M3) return gemm_kind<true>(xq, x_scale, wq, w_scale, m, n, k, y, kind, ldy, ws, st);
+  return gemm_kind<false>(xq, x_scale, wq, w_scale, m, n, k, y, kind, ldy, ws, st);
 }
 
 }  // namespace sq
@@ -1184,6 +1208,6 @@ extern "C" sq_status sq_w8a8_linear_decode_noalloc(const int8_t *xq, const float
   // the decode kernel expects zero partial sums and zero tile counters
   if (cudaMemsetAsync(scratch, 0, need, st) != cudaSuccess) return SQ_ERR_CUDA;
   const sq::OutKind kind = yt == SQ_F32 ? sq::OutKind::F32 : yt == SQ_F16 ? sq::OutKind::F16 : sq::OutKind::BF16;
-  e = sq::launch_w8a8_gemm(xq, x_scale, wq, w_scale, M, N, K, y, kind, ldy, scratch, need, st);
+  e = sq::launch_w8a8_gemm(xq, x_scale, wq, w_scale, M, N, K, y, kind, ldy, scratch, need, st, sq::QFmt::I8);
   return e == cudaSuccess ? SQ_OK : SQ_ERR_CUDA;
 }

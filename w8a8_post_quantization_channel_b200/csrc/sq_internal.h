@@ -30,19 +30,38 @@ cudaError_t launch_zero_fill(float *p, int64_t n, cudaStream_t st);
 // s[j] (holding w_j on entry) <- s_j, inv_s[j] <- 1/s_j from amax[j], w_j.
 cudaError_t launch_smooth_factor(const float *amax, float *s_inout, float *inv_s, int64_t K, float alpha,
                                  cudaStream_t st);
+// Code format of a quantizer: symmetric INT8 (absmax -> 127) or FP8 E4M3
+// (absmax -> 448).
+enum class QFmt { I8, E4M3 };
 // Row-wise: v = x[r][c] * col_scale[c]; per row absmax -> scale, codes.
 cudaError_t launch_quant_rows(const void *x, sq_dtype xt, int64_t rows, int64_t cols, int64_t ld,
-                              const float *col_scale, int8_t *q, float *row_scale_out, cudaStream_t st);
+                              const float *col_scale, int8_t *q, float *row_scale_out, QFmt fmt, cudaStream_t st);
 // W[K][N] -> Wq[N][K] with v = s[j] * W[j][n] quantized per column n with
-// the column maxima colmax[n]; then colmax[n] <- colmax[n] / 127.
+// the column maxima colmax[n]; then colmax[n] <- colmax[n] / Q.
 cudaError_t launch_quant_cols_transpose(const void *w, sq_dtype wt, int64_t K, int64_t N, int64_t ld,
-                                        const float *s, float *colmax_to_scale, int8_t *wq, cudaStream_t st);
+                                        const float *s, float *colmax_to_scale, int8_t *wq, QFmt fmt,
+                                        cudaStream_t st);
 
-// Output kinds of the tensor-core GEMM epilogue.
+// gs[j] = gamma[j] * inv_s[j].
+cudaError_t launch_fold_norm_weight(const float *gamma, const float *inv_s, int64_t K, float *gs, cudaStream_t st);
+// RMSNorm with the folded weight gs (eps) + per-token INT8 (K <= 16384 at
+// 16 bits, 8192 at 32; cudaErrorNotSupported beyond).
+cudaError_t launch_rmsnorm_quant(const void *x, sq_dtype xt, int64_t rows, int64_t cols, int64_t ld,
+                                 const float *gs, float eps, int8_t *q, float *row_scale_out, cudaStream_t st);
+// *delta = max_j(amax_j * inv_s_j) / 127.
+cudaError_t launch_static_scale(const float *amax, const float *inv_s, int64_t K, float *delta, cudaStream_t st);
+// Static per-tensor quantization with the device scalar *delta.
+cudaError_t launch_quant_static(const void *x, sq_dtype xt, int64_t rows, int64_t cols, int64_t ld,
+                                const float *inv_s, const float *delta, int8_t *q, float *row_scale_out,
+                                cudaStream_t st);
+
+// Output kinds of the tensor-core GEMM epilogue (I32: the raw 32-bit
+// accumulator -- an int32 sum for INT8 operands, an f32 sum for E4M3).
 enum class OutKind { F32, F16, BF16, I32 };
+// Operands are INT8 codes (fmt I8) or E4M3 codes (fmt E4M3), both [rows][K].
 cudaError_t launch_w8a8_gemm(const int8_t *xq, const float *x_scale, const int8_t *wq, const float *w_scale,
                              int64_t M, int64_t N, int64_t K, void *y, OutKind kind, int64_t ldy, void *workspace,
-                             size_t workspace_bytes, cudaStream_t st);
+                             size_t workspace_bytes, cudaStream_t st, QFmt fmt);
 size_t w8a8_workspace_bytes(int64_t M, int64_t N, int64_t K);
 
 }  // namespace sq

@@ -5,7 +5,9 @@ of the workloads' shapes, for profilers and roofline measurements.
       --M 2048 --K 4096 --N 16384 --dtype f16 --iters 3
   python -m w8a8_post_quantization_channel_b200.profile_case --sweep decode
 
---op is calib (T = M tokens), weight (W [N, K]), act or linear.  With
+--op is calib (T = M tokens), weight (W [N, K]), act, rmsnorm (the fused
+norm producer), static (static-scale quantizer), linear, or the FP8 (E4M3)
+forms act8, weight8 and linear8.  With
 --time (implied by --sweep) every iteration is timed with CUDA events on
 the launching stream, a 512 MB buffer is read between iterations so that
 L2 (126 MB) holds none of the operands (a read leaves clean lines behind, so
@@ -48,6 +50,15 @@ SWEEPS = {
     # smoothing + weight quantization, [K, K] and the OPT shapes
     "weight": [("weight", 0, K, K, "bf16") for K in (4096, 7168, 8192, 28672)] + [("weight", 0, 4096, 12288, "f16"),
                                                                                      ("weight", 0, 16384, 4096, "f16")],
+    # upstream producer (RMSNorm + smoothing + per-token INT8) and the static
+    # per-tensor quantizer on 16384-token batches
+    "producer": [("rmsnorm", 16384, K, 0, "bf16") for K in (4096, 8192)] + [("rmsnorm", 2048, 4096, 0, "f16")]
+                + [("static", 16384, K, 0, "bf16") for K in (4096, 8192)],
+    # FP8 (E4M3): activation quantization, weight path, prefill and decode linears
+    "fp8": [("act8", 16384, 4096, 0, "bf16"), ("weight8", 0, 8192, 8192, "bf16")]
+           + [("linear8", 2048, K, N, "f16") for _, K, N in synth.OPT_6_7B]
+           + [("linear8", 4096, K, N, "bf16") for _, K, N in synth.LLAMA2_70B[3:]]
+           + [("linear8", M, 8192, 28672, "bf16") for M in (1, 16, 64)],
     # prefill-shaped linears
     "prefill": [("linear", 2048, K, N, "f16") for _, K, N in synth.OPT_6_7B]
                + [("linear", 4096, K, N, "bf16") for _, K, N in synth.LLAMA2_70B[1:]]
@@ -67,6 +78,18 @@ def peaks():
 def make_case(op, M, K, N, dtype, dev="cuda"):
     dt = DT[dtype]
     o = synth.outliers(K, frac=0.01, mult=100.0, seed=1)
+    if op in ("rmsnorm", "static"):
+        x = synth.activations(M, K, o, 2, dt, device=dev)
+        inv = torch.rand(K, device=dev) + 0.5
+        gamma = torch.rand(K, device=dev) + 0.5
+        xq = torch.empty(M, K, dtype=torch.int8, device=dev)
+        xs = torch.empty(M, device=dev)
+        delta = torch.full((1,), 0.05, device=dev)
+        nbytes = M * K * (ESZ[dtype] + 1) + 4 * (M + K)
+        if op == "rmsnorm":
+            gs = sq.sq_fold_smooth_into_norm(gamma, inv)
+            return (lambda: sq.sq_rmsnorm_quant_act(x, gs, 1e-5, xq=xq, x_scale=xs)), nbytes, None
+        return (lambda: sq.sq_quant_act_static(x, inv, delta, xq=xq, x_scale=xs)), nbytes, None
     if op in ("calib", "act"):
         x = synth.activations(M, K, o, 2, dt, device=dev)
         amax = torch.zeros(K, device=dev)
@@ -76,6 +99,12 @@ def make_case(op, M, K, N, dtype, dev="cuda"):
         if op == "calib":
             return (lambda: sq.sq_calib_absmax(x, amax)), M * K * ESZ[dtype] + 8 * K, None
         return (lambda: sq.sq_quant_act(x, inv, xq=xq, x_scale=xs)), M * K * (ESZ[dtype] + 1) + 4 * (M + K), None
+    if op == "act8":
+        x = synth.activations(M, K, o, 2, dt, device=dev)
+        inv = torch.rand(K, device=dev) + 0.5
+        xq = torch.empty(M, K, dtype=torch.uint8, device=dev)
+        xs = torch.empty(M, device=dev)
+        return (lambda: sq.sq_quant_act_e4m3(x, inv, xq=xq, x_scale=xs)), M * K * (ESZ[dtype] + 1) + 4 * (M + K), None
     if op == "weight":
         w = synth.weights(K, N, 3, dt, "nk", device=dev)
         amax = torch.rand(K, device=dev) * 10
@@ -83,6 +112,27 @@ def make_case(op, M, K, N, dtype, dev="cuda"):
                     smooth=torch.empty(K, device=dev), inv_smooth=torch.empty(K, device=dev))
         fn = lambda: sq.sq_smooth_quant_weight(w, sq.SQ_W_NK, amax, 0.5, **outs)  # noqa: E731
         return fn, 2 * N * K * ESZ[dtype] + N * K + 4 * N + 16 * K, None
+    if op == "weight8":
+        w = synth.weights(K, N, 3, dt, "nk", device=dev)
+        amax = torch.rand(K, device=dev) * 10
+        outs = dict(wq=torch.empty(N, K, dtype=torch.uint8, device=dev), w_scale=torch.empty(N, device=dev),
+                    smooth=torch.empty(K, device=dev), inv_smooth=torch.empty(K, device=dev))
+        fn = lambda: sq.sq_smooth_quant_weight_e4m3(w, sq.SQ_W_NK, amax, 0.5, **outs)  # noqa: E731
+        return fn, 2 * N * K * ESZ[dtype] + N * K + 4 * N + 16 * K, None
+    if op == "linear8":
+        g = synth.gen(4, dev)
+        # E4M3 codes of N(0,1) draws scaled to use the format's range
+        xq = (torch.randn(M, K, generator=g, device=dev) * 60).clamp(-448, 448).to(torch.float8_e4m3fn).view(
+            torch.uint8)
+        wq = (torch.randn(N, K, generator=g, device=dev) * 60).clamp(-448, 448).to(torch.float8_e4m3fn).view(
+            torch.uint8)
+        xs = torch.rand(M, device=dev) * 1e-2
+        ws = torch.rand(N, device=dev) * 1e-2
+        y = torch.empty(M, N, dtype=dt, device=dev)
+        need = sq.sq_w8a8_linear_workspace_size(M, N, K)
+        work = torch.zeros(max(need, 1), dtype=torch.uint8, device=dev) if need else None
+        fn = lambda: sq.sq_w8a8_linear_e4m3(xq, xs, wq, ws, dt, y=y, workspace=work)  # noqa: E731
+        return fn, M * K + N * K + M * N * ESZ[dtype] + 4 * (M + N), 2 * M * N * K
     g = synth.gen(4, dev)
     xq = torch.randint(-127, 128, (M, K), generator=g, dtype=torch.int8, device=dev)
     wq = torch.randint(-127, 128, (N, K), generator=g, dtype=torch.int8, device=dev)
@@ -117,7 +167,8 @@ def time_case(op, M, K, N, dtype, iters):
            "GB/s": round(nbytes / t / 1e9, 1), "frac_hbm": round(nbytes / t / 1e9 / hbm, 3)}
     if ops is not None:
         out["TOPS"] = round(ops / t / 1e12, 1)
-        out["frac_int8_peak"] = round(ops / t / 1e12 / int8_peak, 3)
+        # the FP8 and INT8 dense peaks are both 2 x bf16 (4.5 vs 2.25 PFLOP/s nominal)
+        out["frac_fp8_peak" if op == "linear8" else "frac_int8_peak"] = round(ops / t / 1e12 / int8_peak, 3)
         out["bound"] = "hbm" if M <= 64 else "tensor"
     else:
         out["bound"] = "hbm"
@@ -127,7 +178,8 @@ def time_case(op, M, K, N, dtype, iters):
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--op", choices=["calib", "weight", "act", "linear"])
+    ap.add_argument("--op", choices=["calib", "weight", "act", "linear", "rmsnorm", "static", "act8", "weight8",
+                                     "linear8"])
     ap.add_argument("--sweep", choices=sorted(SWEEPS))
     ap.add_argument("--M", type=int, default=2048)
     ap.add_argument("--K", type=int, default=4096)
