@@ -103,9 +103,9 @@ def _ptr(a: np.ndarray, ctype):
 # numpy-facing wrappers, one per oracle step
 # ---------------------------------------------------------------------------
 
-def quantize_value(v: float, r: float) -> int:
-    """clamp(rne(v * r), -127, 127) in fp32."""
-    return int(_load().or_quantize_value(ctypes.c_float(v), ctypes.c_float(r)))
+def quantize_value(v: float, delta: float) -> int:
+    """clamp(rne(v / delta), -127, 127) in fp32 (IEEE division)."""
+    return int(_load().or_quantize_value(ctypes.c_float(v), ctypes.c_float(delta)))
 
 
 def calib_absmax(x, amax=None) -> np.ndarray:

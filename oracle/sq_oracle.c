@@ -27,8 +27,8 @@
  *   - X~ = X * (1/s): the stored reciprocal is multiplied in;
  *   - activations are quantized per token (dynamic), weights per output
  *     channel: for a row v with absmax m, delta = m/127 and
- *     q = clamp(rne(v * (127/m)), -127, 127); an all-zero row gives
- *     delta = 0 and q = 0;
+ *     q = clamp(rne(v / delta), -127, 127) with an IEEE division; an
+ *     all-zero row gives delta = 0 and q = 0;
  *   - the int32 product is dequantized as ((float)acc * dx_t) * dw_n and
  *     then rounded to the output type.
  */
@@ -46,10 +46,11 @@ static float w_at(const float *w, int layout, int64_t K, int64_t N,
 }
 
 /* ---- quantizer for one value --------------------------------------------
- * Round half to even (rintf under the default rounding mode), then clamp to
- * the symmetric range [-127, 127].  r is 127/absmax of the value's row. */
-int8_t or_quantize_value(float v, float r) {
-  float t = v * r;
+ * v / delta with an IEEE division, rounded half to even (rintf under the
+ * default rounding mode), then clamped to the symmetric range [-127, 127].
+ * delta > 0 is the scale of the value's row (absmax / 127). */
+int8_t or_quantize_value(float v, float delta) {
+  float t = v / delta;
   float q = rintf(t);
   if (q > 127.0f) q = 127.0f;
   if (q < -127.0f) q = -127.0f;
@@ -129,7 +130,7 @@ void or_smooth_weight(const float *w, int layout, int64_t K, int64_t N,
 
 /* ---- step 5: per-output-channel weight quantization ---------------------
  * For output channel n: m_n = max_j |W~_jn|, dw_n = m_n/127,
- * Wq[n][j] = clamp(rne(W~_jn * (127/m_n))).  Wq is stored [N][K]
+ * Wq[n][j] = clamp(rne(W~_jn / dw_n)).  Wq is stored [N][K]
  * (K contiguous) whatever W's layout. */
 void or_smooth_quant_weight(const float *w, int layout, int64_t K, int64_t N,
                             const float *s, int8_t *wq, float *dw) {
@@ -145,9 +146,8 @@ void or_smooth_quant_weight(const float *w, int layout, int64_t K, int64_t N,
       continue;
     }
     dw[n] = m / 127.0f;
-    float r = 127.0f / m;
     for (int64_t j = 0; j < K; ++j)
-      wq[n * K + j] = or_quantize_value(s[j] * w_at(w, layout, K, N, j, n), r);
+      wq[n * K + j] = or_quantize_value(s[j] * w_at(w, layout, K, N, j, n), dw[n]);
   }
 }
 
@@ -160,7 +160,7 @@ void or_smooth_act(const float *x, int64_t M, int64_t K, const float *inv_s,
 
 /* ---- step 7: per-token dynamic activation quantization ------------------
  * For token t: m_t = max_j |X~_tj|, dx_t = m_t/127,
- * Xq[t][j] = clamp(rne(X~_tj * (127/m_t))). */
+ * Xq[t][j] = clamp(rne(X~_tj / dx_t)). */
 void or_quant_act(const float *x, int64_t M, int64_t K, const float *inv_s,
                   int8_t *xq, float *dx) {
   for (int64_t t = 0; t < M; ++t) {
@@ -175,9 +175,8 @@ void or_quant_act(const float *x, int64_t M, int64_t K, const float *inv_s,
       continue;
     }
     dx[t] = m / 127.0f;
-    float r = 127.0f / m;
     for (int64_t j = 0; j < K; ++j)
-      xq[t * K + j] = or_quantize_value(x[t * K + j] * inv_s[j], r);
+      xq[t * K + j] = or_quantize_value(x[t * K + j] * inv_s[j], dx[t]);
   }
 }
 
@@ -261,8 +260,7 @@ void or_rmsnorm_quant_act(const float *x, int64_t M, int64_t K, const float *gs,
       continue;
     }
     dx[t] = m / 127.0f;
-    float rq = 127.0f / m;
-    for (int64_t j = 0; j < K; ++j) xq[t * K + j] = or_quantize_value((x[t * K + j] * r) * gs[j], rq);
+    for (int64_t j = 0; j < K; ++j) xq[t * K + j] = or_quantize_value((x[t * K + j] * r) * gs[j], dx[t]);
   }
 }
 
@@ -290,15 +288,14 @@ float or_static_act_scale(const float *amax, const float *inv_s, int64_t K) {
   return m / 127.0f;
 }
 
-/* Static quantization with a fixed scale delta > 0: every token is scaled
- * by r = 1 / delta (one IEEE division) and rounded; values beyond the
- * calibrated range saturate at +-127.  dx_t = delta for every token. */
+/* Static quantization with a fixed scale delta > 0: every smoothed value
+ * is divided by delta and rounded; values beyond the calibrated range
+ * saturate at +-127.  dx_t = delta for every token. */
 void or_quant_act_static(const float *x, int64_t M, int64_t K, const float *inv_s, float delta,
                          int8_t *xq, float *dx) {
-  const float r = 1.0f / delta;
   for (int64_t t = 0; t < M; ++t) {
     dx[t] = delta;
-    for (int64_t j = 0; j < K; ++j) xq[t * K + j] = or_quantize_value(x[t * K + j] * inv_s[j], r);
+    for (int64_t j = 0; j < K; ++j) xq[t * K + j] = or_quantize_value(x[t * K + j] * inv_s[j], delta);
   }
 }
 
@@ -310,8 +307,8 @@ void or_quant_act_static(const float *x, int64_t M, int64_t K, const float *inv_
  * exponent bits of bias 7 and 3 mantissa bits, no infinities, the all-ones
  * exponent with mantissa 111 as NaN, largest finite value 448, subnormals
  * (m/8) * 2^-6 -- with the INT8 path's granularity: delta = m/448 per token
- * and per output channel, code = e4m3(v * (448/m)) rounded to nearest, ties
- * to the even code, saturating at +-448.  The product of two E4M3 values is
+ * and per output channel, code = e4m3(v / delta) (IEEE division) rounded to
+ * nearest, ties to the even code, saturating at +-448.  The product of two E4M3 values is
  * exact, and so is the sum over K in double: every product is a multiple of
  * 2^-18 below 448^2 < 2^18, so K <= 2^15 terms stay within 51 bits. */
 
@@ -344,10 +341,10 @@ uint8_t or_e4m3_encode(float v) {
   return sign | (uint8_t)(((er + 7) << 3) | mant);
 }
 
-static uint8_t e4m3_quantize_value(float v, float r) { return or_e4m3_encode(v * r); }
+static uint8_t e4m3_quantize_value(float v, float delta) { return or_e4m3_encode(v / delta); }
 
 /* Per-output-channel E4M3 weights: m_n = max_j |W~_jn|, dw_n = m_n/448,
- * Wq[n][j] = e4m3(W~_jn * (448/m_n)), stored [N][K]. */
+ * Wq[n][j] = e4m3(W~_jn / dw_n), stored [N][K]. */
 void or_smooth_quant_weight_e4m3(const float *w, int layout, int64_t K, int64_t N, const float *s, uint8_t *wq,
                                  float *dw) {
   for (int64_t n = 0; n < N; ++n) {
@@ -362,13 +359,12 @@ void or_smooth_quant_weight_e4m3(const float *w, int layout, int64_t K, int64_t 
       continue;
     }
     dw[n] = m / 448.0f;
-    float r = 448.0f / m;
-    for (int64_t j = 0; j < K; ++j) wq[n * K + j] = e4m3_quantize_value(s[j] * w_at(w, layout, K, N, j, n), r);
+    for (int64_t j = 0; j < K; ++j) wq[n * K + j] = e4m3_quantize_value(s[j] * w_at(w, layout, K, N, j, n), dw[n]);
   }
 }
 
 /* Per-token E4M3 activations: m_t = max_j |X~_tj|, dx_t = m_t/448,
- * Xq[t][j] = e4m3(X~_tj * (448/m_t)). */
+ * Xq[t][j] = e4m3(X~_tj / dx_t). */
 void or_quant_act_e4m3(const float *x, int64_t M, int64_t K, const float *inv_s, uint8_t *xq, float *dx) {
   for (int64_t t = 0; t < M; ++t) {
     float m = 0.0f;
@@ -382,8 +378,7 @@ void or_quant_act_e4m3(const float *x, int64_t M, int64_t K, const float *inv_s,
       continue;
     }
     dx[t] = m / 448.0f;
-    float r = 448.0f / m;
-    for (int64_t j = 0; j < K; ++j) xq[t * K + j] = e4m3_quantize_value(x[t * K + j] * inv_s[j], r);
+    for (int64_t j = 0; j < K; ++j) xq[t * K + j] = e4m3_quantize_value(x[t * K + j] * inv_s[j], dx[t]);
   }
 }
 

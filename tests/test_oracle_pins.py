@@ -204,6 +204,50 @@ def test_weight_absmax_both_layouts():
 # quantizers: defining property of rounding to a uniform symmetric grid
 # ---------------------------------------------------------------------------
 
+def _fp32_round(q):
+    """A rational rounded to the nearest fp32 value (ties to even)."""
+    from fractions import Fraction
+    if q == 0:
+        return Fraction(0)
+    sign = -1 if q < 0 else 1
+    a = abs(q)
+    e = a.numerator.bit_length() - a.denominator.bit_length()
+    while Fraction(2) ** e > a:
+        e -= 1
+    while Fraction(2) ** (e + 1) <= a:
+        e += 1
+    ulp = Fraction(2) ** (e - 23)
+    n, r = divmod(a, ulp)
+    if r > ulp / 2 or (r == ulp / 2 and n % 2 == 1):
+        n += 1
+    return sign * n * ulp
+
+
+def _rne_int(q):
+    from fractions import Fraction
+    n = q.numerator // q.denominator
+    r = q - n
+    if r > Fraction(1, 2) or (r == Fraction(1, 2) and n % 2 == 1):
+        n += 1
+    return n
+
+
+@pytest.mark.parametrize("v,delta", [(-22.80670928955078, 0.5366284251213074), (-8.67187786102295, 0.4955359101295471),
+                                     (-31.285537719726562, 0.3935287892818451),
+                                     (-50.01250457763672, 0.5989521741867065)])
+def test_quantizer_divides_by_the_scale(v, delta):
+    # The reading: q = rne(fl(v / delta)) with an IEEE division.  These
+    # inputs put v / delta within an ulp of a half-integer, where a multiply
+    # by the rounded reciprocal 1/delta lands on the other side; the expected
+    # code is worked in exact rational arithmetic.
+    from fractions import Fraction
+    v32, d32 = np.float32(v), np.float32(delta)
+    expected = _rne_int(_fp32_round(Fraction(float(v32)) / Fraction(float(d32))))
+    assert oracle.quantize_value(float(v32), float(d32)) == expected
+    via_reciprocal = int(np.rint(np.float32(v32 * np.float32(np.float32(1.0) / d32))))
+    assert via_reciprocal != expected
+
+
 def test_quantize_value_saturation_and_ties():
     assert oracle.quantize_value(200.0, 1.0) == 127
     assert oracle.quantize_value(-200.0, 1.0) == -127
