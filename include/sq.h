@@ -28,8 +28,10 @@
  *     contracted into an FMA.  INT8 codes, scales, s and int32 sums are
  *     therefore reproducible bit for bit on any input.
  *   - Quantization of a row v with absmax m: scale = m / 127 and
- *     q = clamp(rne(v * (127 / m)), -127, 127); an all-zero row gives
- *     scale 0 and codes 0.  -128 is never produced.
+ *     q = clamp(rne(v / scale), -127, 127) with an IEEE division (the
+ *     kernels reach the same codes with a reciprocal multiply and an exact
+ *     check, dividing only next to a rounding boundary); an all-zero row
+ *     gives scale 0 and codes 0.  -128 is never produced.
  *   - Inputs must be finite; NaN/Inf give unspecified results.
  *   - Errors: argument checks run on the host before anything is enqueued
  *     and return SQ_ERR_INVALID_ARG / SQ_ERR_UNSUPPORTED with no side
@@ -87,7 +89,7 @@ sq_status sq_calib_absmax(const void *x, sq_dtype xt, int64_t T, int64_t K,
  *   amax      [K] fp32 calibration maxima from sq_calib_absmax.
  *   alpha     migration strength in [0, 1].
  *   wq        [N][K] int8 OUT, K contiguous (row n = output channel n):
- *             Wq = clamp(rne(W~ * 127 / max_j|W~_jn|)), W~ = diag(s) W.
+ *             Wq = clamp(rne(W~ / w_scale_n)), W~ = diag(s) W.
  *   w_scale   [N] fp32 OUT, per-output-channel scale max_j|W~_jn| / 127.
  *   smooth    [K] fp32 OUT, s_j (also used as scratch during the call).
  *   inv_smooth[K] fp32 OUT, 1/s_j (what sq_quant_act multiplies by).
@@ -138,7 +140,7 @@ sq_status sq_fold_smooth_into_norm(const float *gamma, const float *inv_smooth,
  *   gs [K] fp32, eps >= 0 and finite.  Other arguments as sq_quant_act.
  * Because the order of the double-precision sum is unspecified, r_t may
  * differ from another implementation's by one fp32 ulp, which moves a code
- * by one only where v * 127 / max lies within ~2^-20 of a rounding
+ * by one only where v / scale lies within ~2^-20 of a rounding
  * boundary.  K <= 16384 for 16-bit x, <= 8192 for fp32 x, else
  * SQ_ERR_UNSUPPORTED.
  */
@@ -157,8 +159,8 @@ sq_status sq_static_act_scale(const float *amax, const float *inv_smooth, int64_
                               float *delta, sq_stream_t stream);
 
 /*
- * Static quantization with that scale: xq = clamp(rne((x * inv_smooth) *
- * (1 / *delta)), -127, 127) -- values beyond the calibrated range
+ * Static quantization with that scale: xq = clamp(rne((x * inv_smooth) /
+ * *delta), -127, 127) -- values beyond the calibrated range
  * saturate -- and x_scale_t = *delta for every token, so sq_w8a8_linear
  * consumes the result unchanged.  delta is a device pointer (*delta > 0).
  * Other arguments as sq_quant_act.
@@ -202,13 +204,35 @@ sq_status sq_w8a8_accumulate(const int8_t *xq, const int8_t *wq, int64_t M,
                              sq_stream_t stream);
 
 /*
+ * Column-parallel linear: the output-channel shard of one rank, stored into
+ * several destinations in the same pass.  With G ranks each holding the rows
+ * [n0, n0 + N) of Wq and w_scale (a shard of the output channels) and the
+ * same xq / x_scale, every rank's call produces Y[:, n0:n0+N] and writes each
+ * tile into all n_dst destination matrices -- its own Y and the other ranks'
+ * copies, which may be peer-mapped device pointers (plain stores over
+ * NVLink) -- so that after every rank's call (and a barrier that orders it)
+ * each rank holds the full Y without a separate all-gather.  The page's
+ * OPT-175B runs use 8 GPUs; this is how the linear shards over them.
+ *   y_dst      HOST array of n_dst (1..8) device pointers; y_dst[d] points at
+ *              the destination's element (row 0, column n0), row stride ldy
+ *              elements of type yt, 16-byte aligned.
+ * Other arguments, workspace and errors as sq_w8a8_linear (N is the shard's
+ * width).  Writes from different ranks go to disjoint columns.
+ */
+sq_status sq_w8a8_linear_scatter(const int8_t *xq, const float *x_scale,
+                                 const int8_t *wq, const float *w_scale, int64_t M,
+                                 int64_t N, int64_t K, void *const *y_dst, int n_dst,
+                                 sq_dtype yt, int64_t ldy, void *workspace,
+                                 size_t workspace_bytes, sq_stream_t stream);
+
+/*
  * FP8 (E4M3) variant.  The survey page "Quantization Calibration
  * GPTQ/AWQ/SmoothQuant 2026" (jisaku.com glossary) lists FP8 SmoothQuant:
  * the same smoothing, with FP8 operands.  Both operands are E4M3 codes (1
  * sign, 4 exponent bits of bias 7, 3 mantissa bits, no infinities,
  * S.1111.111 = NaN, largest finite 448) with the INT8 path's granularity:
  *   scale = m / 448 for a row with absmax m, and
- *   code  = e4m3(v * (448 / m)), nearest value, ties to the even code,
+ *   code  = e4m3(v / scale) (IEEE division), nearest value, ties to even,
  *           saturating at +-448;  an all-zero row gives scale 0, codes +0.
  * Smoothing (s, 1/s) is computed exactly as for INT8.  The product runs on
  * the tensor cores' FP8 path with an fp32 accumulator: every product of

@@ -82,6 +82,18 @@ def test_quant_act_argument_checks():
     assert f(MIS, sq.SQ_F32, 8, 256, 256, A16, A16, A16, None) == INV
 
 
+def test_scatter_argument_checks_host():
+    f = sq.lib().sq_w8a8_linear_scatter
+    dsts = (ctypes.c_void_p * 2)(A16, A16 + 4096)
+    mis = (ctypes.c_void_p * 2)(A16, MIS)
+    assert f(A16, A16, A16, A16, 0, 256, 256, dsts, 2, sq.SQ_BF16, 256, None, 0, None) == sq.SQ_OK  # M == 0
+    assert f(A16, A16, A16, A16, 64, 256, 256, None, 2, sq.SQ_BF16, 256, None, 0, None) == INV
+    assert f(A16, A16, A16, A16, 64, 256, 256, dsts, 0, sq.SQ_BF16, 256, None, 0, None) == INV
+    assert f(A16, A16, A16, A16, 64, 256, 256, dsts, 9, sq.SQ_BF16, 256, None, 0, None) == INV
+    assert f(A16, A16, A16, A16, 64, 256, 256, mis, 2, sq.SQ_BF16, 256, None, 0, None) == INV
+    assert f(A16, A16, A16, None, 64, 256, 256, dsts, 2, sq.SQ_BF16, 256, None, 0, None) == INV
+
+
 def test_producer_argument_checks():
     L = sq.lib()
     fold = L.sq_fold_smooth_into_norm

@@ -62,6 +62,34 @@ def test_conversion_matches_the_format_everywhere():
     np.testing.assert_array_equal(xq.cpu().numpy(), oracle.e4m3_encode(x))
 
 
+def test_codes_next_to_e4m3_midpoints():
+    # rows with absmax m (first value) and values within a few ulps of
+    # (E4M3 midpoint) * delta, delta = fl(m / 448): v / delta lands next to a
+    # rounding boundary of the format, where fl(v * fl(1/delta)) alone could
+    # round to the neighbouring code
+    vals = _finite_values()
+    mids = ((vals[1:] + vals[:-1]) / 2)
+    mids = mids[np.abs(mids) < 448]
+    rng = np.random.default_rng(43)
+    K, n_rows = 512, 32
+    x = np.zeros((n_rows, K), np.float32)
+    for t in range(n_rows):
+        m = np.float32(rng.uniform(0.01, 100.0))
+        d = np.float32(m / np.float32(448.0))
+        x[t, 0] = m
+        base = (rng.choice(mids, K - 1) * np.float64(d)).astype(np.float32)
+        steps = rng.integers(-2, 3, K - 1)
+        for i in range(K - 1):
+            for _ in range(abs(int(steps[i]))):
+                base[i] = np.nextafter(base[i], np.float32(np.inf) if steps[i] > 0 else np.float32(-np.inf))
+        x[t, 1:] = np.clip(base, -m, m)
+    ones = np.ones(K, np.float32)
+    xq, xs = sq.sq_quant_act_e4m3(torch.from_numpy(x).to(DEV), torch.from_numpy(ones).to(DEV))
+    xq_ref, xs_ref = oracle.quant_act_e4m3(x, ones)
+    np.testing.assert_array_equal(xs.cpu().numpy(), xs_ref)
+    np.testing.assert_array_equal(xq.cpu().numpy(), xq_ref)
+
+
 @pytest.mark.parametrize("dt,K", [("bf16", 16), ("f32", 256), ("bf16", 1040), ("f16", 4096), ("bf16", 16384),
                                   ("f16", 28672), ("bf16", 40960)])
 @pytest.mark.parametrize("M", [1, 37])

@@ -14,7 +14,7 @@ import torch
 import torch.distributed as dist
 import torch.multiprocessing as mp
 
-from w8a8_post_quantization_channel_b200.dist import allreduce_amax, shard_range
+from w8a8_post_quantization_channel_b200.dist import allreduce_amax, column_parallel_linear, column_shard, shard_range
 
 
 def test_shard_range_partitions():
@@ -83,3 +83,62 @@ def test_two_rank_calibration_merge_gloo():
         assert ok_amax is True, f"rank {rank}: {ok_amax}"
         assert ok_w
     assert any(r[3] for r in results)
+
+
+def test_column_shard_partitions():
+    for n in (16, 48, 4096, 12288, 28672):
+        for world in (1, 2, 3, 4, 8):
+            spans = [column_shard(n, world, r) for r in range(world)]
+            assert spans[0][0] == 0 and spans[-1][1] == n
+            for (a, b), (c, d) in zip(spans, spans[1:]):
+                assert b == c
+            assert all(a % 16 == 0 and b % 16 == 0 for a, b in spans)
+            sizes = [b - a for a, b in spans]
+            assert max(sizes) - min(sizes) <= 16
+    with pytest.raises(ValueError):
+        column_shard(100, 2, 0)
+
+
+def _oracle_linear(xq, x_scale, wq, w_scale, out_dtype):
+    import oracle
+    acc = oracle.gemm_i8(xq.numpy(), wq.numpy())
+    return torch.from_numpy(oracle.dequant(acc, x_scale.numpy(), w_scale.numpy()))
+
+
+def _column_worker(rank, world, port, q):
+    try:
+        os.environ["MASTER_ADDR"] = "127.0.0.1"
+        os.environ["MASTER_PORT"] = str(port)
+        dist.init_process_group("gloo", rank=rank, world_size=world)
+        import oracle
+        M, K, N = 24, 64, 48
+        g = torch.Generator().manual_seed(11)
+        xq = torch.randint(-127, 128, (M, K), generator=g, dtype=torch.int8)
+        wq = torch.randint(-127, 128, (N, K), generator=g, dtype=torch.int8)
+        xs = torch.rand(M, generator=g) * 1e-2
+        ws = torch.rand(N, generator=g) * 1e-2
+        n0, n1 = column_shard(N, world, rank)
+        y = column_parallel_linear(xq, xs, wq[n0:n1].contiguous(), ws[n0:n1].contiguous(), N,
+                                   out_dtype=torch.float32, linear=_oracle_linear)
+        full = oracle.dequant(oracle.gemm_i8(xq.numpy(), wq.numpy()), xs.numpy(), ws.numpy())
+        q.put((rank, bool(np.array_equal(y.numpy(), full)), n1 - n0))
+        dist.destroy_process_group()
+    except Exception as e:  # pragma: no cover
+        q.put((rank, repr(e), -1))
+
+
+@pytest.mark.parametrize("world", [2, 4])
+def test_column_parallel_linear_gathers_every_shard_gloo(world):
+    # N = 48 over 4 ranks leaves the last rank without columns
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_column_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    results = sorted(q.get(timeout=240) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+    assert all(ok is True for _, ok, _ in results), results
+    assert sum(w for _, _, w in results) == 48
+

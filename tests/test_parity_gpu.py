@@ -141,6 +141,59 @@ def test_quant_act(dt, K, M):
     no_device_error()
 
 
+def _near_boundary_rows(n_rows, K, seed):
+    """fp32 rows whose first value is the row's absmax m and whose other
+    values sit within a few ulps of (k + 1/2) * delta, delta = fl(m / 127):
+    v / delta lands next to a rounding boundary, where a reciprocal multiply
+    alone could round to the other integer."""
+    rng = np.random.default_rng(seed)
+    x = np.zeros((n_rows, K), np.float32)
+    for t in range(n_rows):
+        m = np.float32(rng.uniform(0.5, 100.0))
+        d = np.float32(m / np.float32(127.0))
+        x[t, 0] = m
+        k = rng.integers(-127, 127, K - 1)
+        base = ((k + 0.5) * np.float64(d)).astype(np.float32)
+        steps = rng.integers(-3, 4, K - 1)
+        v = base.copy()
+        for i in range(K - 1):
+            for _ in range(abs(int(steps[i]))):
+                v[i] = np.nextafter(v[i], np.float32(np.inf) if steps[i] > 0 else np.float32(-np.inf))
+        x[t, 1:] = np.clip(v, -m, m)
+    return x
+
+
+@pytest.mark.parametrize("K", [16, 272, 4096, 20480])
+def test_quant_act_near_rounding_boundaries(K):
+    x = _near_boundary_rows(24, K, seed=K)
+    ones = np.ones(K, np.float32)
+    xq, xs = sq.sq_quant_act(torch.from_numpy(x).to(DEV), torch.from_numpy(ones).to(DEV))
+    xq_ref, xs_ref = oracle.quant_act(x, ones)
+    np.testing.assert_array_equal(xs.cpu().numpy(), xs_ref)
+    np.testing.assert_array_equal(xq.cpu().numpy(), xq_ref)
+    # the same values through the static path, with each row's own scale
+    for t in (0, 5):
+        delta = torch.tensor([xs_ref[t]], device=DEV)
+        q, _ = sq.sq_quant_act_static(torch.from_numpy(x[t:t + 1]).to(DEV), torch.from_numpy(ones).to(DEV), delta)
+        q_ref, _ = oracle.quant_act_static(x[t:t + 1], ones, float(xs_ref[t]))
+        np.testing.assert_array_equal(q.cpu().numpy(), q_ref)
+    no_device_error()
+
+
+def test_weight_cols_near_rounding_boundaries():
+    # W[K][N] columns with the same construction go through the column
+    # quantizer (smoothing factor forced to 1: amax = w_j, alpha = 0.5)
+    K, N = 64, 48
+    w = np.ascontiguousarray(_near_boundary_rows(N, K, seed=7).T)  # [K][N]: column n = row n above
+    amax = np.abs(w).max(axis=1).astype(np.float32)
+    wq, ws, s, inv = sq.sq_smooth_quant_weight(torch.from_numpy(w).to(DEV), sq.SQ_W_KN, torch.from_numpy(amax).to(DEV),
+                                               0.5)
+    s_ref, _ = oracle.smooth_factor(amax, oracle.weight_absmax(w, oracle.LAYOUT_KN), 0.5)
+    wq_ref, ws_ref = oracle.smooth_quant_weight(w, oracle.LAYOUT_KN, s_ref)
+    np.testing.assert_array_equal(ws.cpu().numpy(), ws_ref)
+    np.testing.assert_array_equal(wq.cpu().numpy(), wq_ref)
+
+
 def test_quant_act_padded_rows_and_empty():
     M, K, ld = 9, 512, 640
     base = synth.activations(M, ld, synth.outliers(ld, count=5, seed=3), seed=4, dtype=torch.float16)

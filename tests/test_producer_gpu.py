@@ -30,15 +30,15 @@ def f32(t):
 
 
 def _boundary_mask(x, gs, eps):
-    """Elements whose oracle value v * (127 / max|v|) sits within 1e-4 of a
+    """Elements whose oracle value v / (max|v| / 127) sits within 1e-4 of a
     half-integer, recomputed in fp32 with the oracle's own r."""
     r = oracle.rmsnorm_factor(x, eps)
     v = (x * r[:, None]).astype(np.float32)
     v = (v * gs).astype(np.float32)
     m = np.abs(v).max(axis=1)
+    delta = (m / np.float32(127.0)).astype(np.float32)
     with np.errstate(divide="ignore", invalid="ignore"):
-        rq = np.where(m > 0, np.float32(127.0) / m, np.float32(0.0)).astype(np.float32)
-    u = np.abs((v * rq[:, None]).astype(np.float32)).astype(np.float64)
+        u = np.abs(np.where(delta[:, None] > 0, v / delta[:, None], 0).astype(np.float32)).astype(np.float64)
     return np.abs(u - np.floor(u) - 0.5) < 1e-4
 
 

@@ -36,6 +36,7 @@ __all__ = [
     "sq_w8a8_linear_decode_noalloc", "SQ_DECODE_STATIC_SCRATCH_BYTES", "sq_selftest_wait_timeout",
     "sq_fold_smooth_into_norm", "sq_rmsnorm_quant_act", "sq_static_act_scale", "sq_quant_act_static",
     "sq_smooth_quant_weight_e4m3", "sq_quant_act_e4m3", "sq_w8a8_linear_e4m3", "sq_w8a8_accumulate_e4m3",
+    "sq_w8a8_linear_scatter",
 ]
 
 SQ_OK, SQ_ERR_INVALID_ARG, SQ_ERR_UNSUPPORTED, SQ_ERR_CUDA, SQ_ERR_TIMEOUT = 0, 1, 2, 3, 4
@@ -90,6 +91,7 @@ def lib() -> ctypes.CDLL:
             "sq_quant_act_e4m3": [vp, i32, i64, i64, i64, vp, vp, vp, vp],
             "sq_w8a8_linear_e4m3": [vp, vp, vp, vp, i64, i64, i64, vp, i32, i64, vp, sz, vp],
             "sq_w8a8_accumulate_e4m3": [vp, vp, i64, i64, i64, vp, i64, vp, sz, vp],
+            "sq_w8a8_linear_scatter": [vp, vp, vp, vp, i64, i64, i64, vp, i32, i32, i64, vp, sz, vp],
         }
         for name, args in sigs.items():
             fn = getattr(L, name)
@@ -235,6 +237,32 @@ def sq_w8a8_linear(xq: torch.Tensor, x_scale: torch.Tensor, wq: torch.Tensor, w_
                                 _dtype(y, "y"), y.stride(0), _ptr(workspace), wbytes, _stream(stream)),
            "sq_w8a8_linear")
     return y
+
+
+def sq_w8a8_linear_scatter(xq: torch.Tensor, x_scale: torch.Tensor, wq: torch.Tensor, w_scale: torch.Tensor,
+                           ys, col0: int, workspace=None, stream=None) -> None:
+    """Column-parallel linear: this shard's Y[:, col0:col0+N] (wq, w_scale are
+    the shard's rows) stored into every full [M, N_total] tensor in ys (this
+    rank's Y and peers' copies; all of one dtype and row stride)."""
+    M, K = xq.shape
+    N = wq.shape[0]
+    if not 1 <= len(ys) <= 8:
+        raise ValueError("1 to 8 destinations")
+    y0 = ys[0]
+    for y in ys:
+        if y.dim() != 2 or y.stride(1) != 1 or y.dtype != y0.dtype or y.stride(0) != y0.stride(0):
+            raise ValueError("destinations must be row-major 2-D tensors of one dtype and row stride")
+        if y.shape[0] != M or col0 < 0 or col0 + N > y.shape[1]:
+            raise ValueError("shard does not fit the destination")
+    esz = y0.element_size()
+    ptrs = (ctypes.c_void_p * len(ys))(*[y.data_ptr() + col0 * esz for y in ys])
+    need = sq_w8a8_linear_workspace_size(M, N, K)
+    if workspace is None and need > 0:
+        workspace = torch.zeros(need, dtype=torch.uint8, device=xq.device)
+    wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().sq_w8a8_linear_scatter(_ptr(xq), _ptr(x_scale), _ptr(wq), _ptr(w_scale), M, N, K, ptrs, len(ys),
+                                        _dtype(y0, "y"), y0.stride(0), _ptr(workspace), wbytes, _stream(stream)),
+           "sq_w8a8_linear_scatter")
 
 
 def sq_w8a8_accumulate(xq: torch.Tensor, wq: torch.Tensor, acc=None, workspace=None, stream=None) -> torch.Tensor:

@@ -253,6 +253,25 @@ sq_status sq_w8a8_linear_e4m3(const uint8_t *xq, const float *x_scale, const uin
                      M, N, K, y, yt, ldy, workspace, workspace_bytes, sq::QFmt::E4M3, stream);
 }
 
+sq_status sq_w8a8_linear_scatter(const int8_t *xq, const float *x_scale, const int8_t *wq, const float *w_scale,
+                                 int64_t M, int64_t N, int64_t K, void *const *y_dst, int n_dst, sq_dtype yt,
+                                 int64_t ldy, void *workspace, size_t workspace_bytes, sq_stream_t stream) {
+  if (!valid_dtype(yt) || !valid_vec(w_scale)) return SQ_ERR_INVALID_ARG;
+  if (y_dst == nullptr || n_dst < 1 || n_dst > sq::kMaxDest) return SQ_ERR_INVALID_ARG;
+  sq::YDest dst{};
+  for (int d = 0; d < n_dst; ++d) {
+    if (!valid_vec(y_dst[d])) return SQ_ERR_INVALID_ARG;
+    dst.p[d] = y_dst[d];
+  }
+  dst.n = n_dst;
+  sq_status s = gemm_common(xq, wq, M, N, K, y_dst[0], ldy, dsize(yt), workspace, workspace_bytes);
+  if (s != SQ_OK || M == 0) return s;
+  if (!valid_vec(x_scale)) return SQ_ERR_INVALID_ARG;
+  const sq::OutKind kind = yt == SQ_F32 ? sq::OutKind::F32 : yt == SQ_F16 ? sq::OutKind::F16 : sq::OutKind::BF16;
+  return from_cuda(sq::launch_w8a8_gemm_dest(xq, x_scale, wq, w_scale, M, N, K, dst, kind, ldy, workspace,
+                                             (cudaStream_t)stream, sq::QFmt::I8));
+}
+
 size_t sq_w8a8_linear_workspace_size(int64_t M, int64_t N, int64_t K) {
   if (M <= 0 || N <= 0 || K <= 0) return 0;
   return sq::w8a8_workspace_bytes(M, N, K);

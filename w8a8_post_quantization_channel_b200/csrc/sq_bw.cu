@@ -98,7 +98,7 @@ __global__ void __launch_bounds__(256) absmax_rows_kernel(const T *__restrict__ 
     float f[V];
     Vec<T>::to_f32(ld_stream_v4(row + v * V), f);
 #pragma unroll
-    for (int e = 0; e < V; ++e) m = fmaxf(m, fabsf(f[e]));
+    for (int e = 0; e < V; e += 2) m = fmax3(m, fabsf(f[e]), fabsf(f[e + 1]));
   }
   m = block_max(m, red);
   if (threadIdx.x == 0) out[blockIdx.x] = m;
@@ -141,7 +141,7 @@ __global__ void smooth_factor_kernel(const float *__restrict__ amax, float *__re
 // Row quantizer (persistent): each CTA walks rows r = blockIdx.x,
 // blockIdx.x + gridDim.x, ...; per row
 //   v_c = x[r][c] * col_scale[c];  m = max_c |v_c|;
-//   row_scale_out[r] = m / Q;  q[r][c] = code(v_c * (Q / m)),
+//   row_scale_out[r] = delta = m / Q;  q[r][c] = code(v_c / delta),
 // Q = F::kMax (127 for INT8 codes, 448 for E4M3).
 // Thread t owns the 16-byte vectors t + i*blockDim (i < kVPT) of every row:
 // their column scales stay in registers for the CTA's lifetime, the next
@@ -196,7 +196,7 @@ __global__ void __launch_bounds__(kRowMaxThreads)
         val[i][e + 1] = p.y;
       }
 #pragma unroll
-      for (int e = 0; e < V; ++e) m = fmaxf(m, fabsf(val[i][e]));
+      for (int e = 0; e < V; e += 2) m = fmax3(m, fabsf(val[i][e]), fabsf(val[i][e + 1]));
     }
     m = warp_max(m);
     if (lane == 0) red[slot][warp] = m;
@@ -205,17 +205,19 @@ __global__ void __launch_bounds__(kRowMaxThreads)
     for (int w = 0; w < nwarps; ++w) m = fmaxf(m, red[slot][w]);
     slot ^= 1;
     // m == 0 (all-zero row): rcp = 0 gives codes 0 and scale 0
-    const float rcp = m > 0.0f ? __fdiv_rn(F::kMax, m) : 0.0f;
-    if (tid == 0) row_scale_out[r] = __fdiv_rn(m, F::kMax);
+    // scale delta = m / Q; codes of fl(v / delta) (rcp = 0 for a zero row)
+    const float delta = __fdiv_rn(m, F::kMax);
+    const float rcp = m > 0.0f ? __frcp_rn(delta) : 0.0f;
+    if (tid == 0) row_scale_out[r] = delta;
     int8_t *qrow = q + r * K;
 #pragma unroll
     for (int i = 0; i < kVPT; ++i) {
       const int64_t v = tid + (int64_t)i * blockDim.x;
       if (v < nvec) {
         if constexpr (V == 8) {
-          *reinterpret_cast<uint2 *>(qrow + v * V) = F::codes8(val[i], rcp);
+          *reinterpret_cast<uint2 *>(qrow + v * V) = F::codes8(val[i], delta, rcp);
         } else {
-          *reinterpret_cast<uint32_t *>(qrow + v * V) = F::codes4(val[i], rcp);
+          *reinterpret_cast<uint32_t *>(qrow + v * V) = F::codes4(val[i], delta, rcp);
         }
       }
     }
@@ -287,7 +289,7 @@ __global__ void __launch_bounds__(kSmemRowThreads, 1)
 #pragma unroll
         for (int e = 0; e < V; e += 2) {
           const float2 p = fmul2_rn(make_float2(f[e], f[e + 1]), make_float2(sc[i][e], sc[i][e + 1]));
-          m = fmaxf(m, fmaxf(fabsf(p.x), fabsf(p.y)));
+          m = fmax3(m, fabsf(p.x), fabsf(p.y));
         }
       }
     }
@@ -298,8 +300,10 @@ __global__ void __launch_bounds__(kSmemRowThreads, 1)
 #pragma unroll
     for (int w = 0; w < kSmemRowThreads / 32; ++w) m = fmaxf(m, red[slot * 16 + w]);
     slot ^= 1;
-    const float rcp = m > 0.0f ? __fdiv_rn(F::kMax, m) : 0.0f;
-    if (tid == 0) row_scale_out[r] = __fdiv_rn(m, F::kMax);
+    // scale delta = m / Q; codes of fl(v / delta) (rcp = 0 for a zero row)
+    const float delta = __fdiv_rn(m, F::kMax);
+    const float rcp = m > 0.0f ? __frcp_rn(delta) : 0.0f;
+    if (tid == 0) row_scale_out[r] = delta;
     int8_t *qrow = q + r * K;
 #pragma unroll
     for (int i = 0; i < kVPT; ++i) {
@@ -315,9 +319,9 @@ __global__ void __launch_bounds__(kSmemRowThreads, 1)
           val[e + 1] = p.y;
         }
         if constexpr (V == 8) {
-          *reinterpret_cast<uint2 *>(qrow + v * V) = F::codes8(val, rcp);
+          *reinterpret_cast<uint2 *>(qrow + v * V) = F::codes8(val, delta, rcp);
         } else {
-          *reinterpret_cast<uint32_t *>(qrow + v * V) = F::codes4(val, rcp);
+          *reinterpret_cast<uint32_t *>(qrow + v * V) = F::codes4(val, delta, rcp);
         }
       }
     }
@@ -360,8 +364,9 @@ __global__ void __launch_bounds__(1024) quant_rows_twopass_kernel(const T *__res
     for (int e = 0; e < V; ++e) m = fmaxf(m, fabsf(__fmul_rn(f[e], __ldg(col_scale + v * V + e))));
   }
   m = block_max(m, red);
-  const float rcp = m > 0.0f ? __fdiv_rn(F::kMax, m) : 0.0f;
-  if (threadIdx.x == 0) row_scale_out[r] = __fdiv_rn(m, F::kMax);
+  const float delta = __fdiv_rn(m, F::kMax);
+  const float rcp = m > 0.0f ? __frcp_rn(delta) : 0.0f;
+  if (threadIdx.x == 0) row_scale_out[r] = delta;
   int8_t *qrow = q + r * K;
   for (int64_t v = threadIdx.x; v < nvec; v += blockDim.x) {
     float f[V];
@@ -370,9 +375,9 @@ __global__ void __launch_bounds__(1024) quant_rows_twopass_kernel(const T *__res
 #pragma unroll
     for (int e = 0; e < V; ++e) val[e] = __fmul_rn(f[e], __ldg(col_scale + v * V + e));
     if constexpr (V == 8) {
-      *reinterpret_cast<uint2 *>(qrow + v * V) = F::codes8(val, rcp);
+      *reinterpret_cast<uint2 *>(qrow + v * V) = F::codes8(val, delta, rcp);
     } else {
-      *reinterpret_cast<uint32_t *>(qrow + v * V) = F::codes4(val, rcp);
+      *reinterpret_cast<uint32_t *>(qrow + v * V) = F::codes4(val, delta, rcp);
     }
   }
 }
@@ -389,13 +394,15 @@ __global__ void __launch_bounds__(256) quant_cols_transpose_kernel(const T *__re
   pdl_wait();  // the previous kernel's results are visible from here on
   pdl_trigger();
   __shared__ uint8_t tile[kTT][kTT + 4];  // [n][j] codes
-  __shared__ float rcp[kTT];
+  __shared__ float dlt[kTT], rcp[kTT];  // per column: scale, fl(1 / scale)
   const int64_t j0 = (int64_t)blockIdx.y * kTT, n0 = (int64_t)blockIdx.x * kTT;
   const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;  // 16 x 16 threads
   if (threadIdx.x < kTT) {
     const int64_t n = n0 + threadIdx.x;
     const float cm = n < N ? __ldg(colmax + n) : 0.0f;
-    rcp[threadIdx.x] = cm > 0.0f ? __fdiv_rn(F::kMax, cm) : 0.0f;
+    // the scale finalize_scale_kernel stores: fl(colmax / Q)
+    dlt[threadIdx.x] = __fdiv_rn(cm, F::kMax);
+    rcp[threadIdx.x] = cm > 0.0f ? __frcp_rn(dlt[threadIdx.x]) : 0.0f;
   }
   __syncthreads();
   // each thread: 4 consecutive n of one j row, rows ty, ty+16, ...
@@ -408,7 +415,7 @@ __global__ void __launch_bounds__(256) quant_cols_transpose_kernel(const T *__re
       const float sj = __ldg(s + j);
       const T *p = w + j * ld + n;
 #pragma unroll
-      for (int e = 0; e < 4; ++e) c[e] = F::code1(__fmul_rn(sj, Vec<T>::one(p + e)), rcp[tx * 4 + e]);
+      for (int e = 0; e < 4; ++e) c[e] = F::code1(__fmul_rn(sj, Vec<T>::one(p + e)), dlt[tx * 4 + e], rcp[tx * 4 + e]);
     }
 #pragma unroll
     for (int e = 0; e < 4; ++e) tile[tx * 4 + e][jj] = c[e];

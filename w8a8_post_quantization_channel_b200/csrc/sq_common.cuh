@@ -125,8 +125,10 @@ __device__ __forceinline__ uint4 ld_policy_v4(const void *p, uint64_t policy) {
 }
 
 // ---------------------------------------------------------------------------
-// The quantizer: clamp(rne(v * r), -127, 127), r = 127 / absmax of the row.
-// __fmul_rn keeps the product a separately rounded IEEE multiply.
+// The quantizer: code = rne(fl(v / delta)) for a row with scale delta =
+// absmax / Q (Q = 127 for INT8, 448 for E4M3), clamped to [-127, 127] for
+// INT8.  Every product and sum below is a separately rounded IEEE operation
+// (explicit _rn intrinsics or .rn PTX), never contracted.
 // ---------------------------------------------------------------------------
 // Rounds u to the nearest integer, ties to even, with one exact IEEE
 // addition: for |u| < 2^22, u + 1.5 * 2^23 lies in [2^23, 2^24), where
@@ -134,15 +136,21 @@ __device__ __forceinline__ uint4 ld_policy_v4(const void *p, uint64_t policy) {
 // 1.5 * 2^23 + rne(u) (the shift is even, so ties land on the even integer)
 // and rne(u) sits in the low bits of the sum's encoding: its low byte is
 // the two's-complement int8 code whenever |rne(u)| <= 127.  This keeps the
-// conversion off the float-to-integer unit (one add on the fp32 pipe).
+// conversion off the float-to-integer unit.
 constexpr float kRneShift = 12582912.0f;  // 1.5 * 2^23
 
-// Clamped code for finite v: clamp(rne(v * r), -127, 127) (clamping before
-// rounding gives the same integer as rounding before clamping).
-__device__ __forceinline__ int quantize(float v, float r) {
-  const float u = fminf(fmaxf(__fmul_rn(v, r), -127.0f), 127.0f);
-  return (int)(int8_t)(__float_as_uint(__fadd_rn(u, kRneShift)) & 0xffu);
-}
+// A value's code is rne(fl(v / delta)) (IEEE division by the row's scale),
+// formed here without a division per value.  With rcp = fl(1 / delta) the
+// exact product P = v * rcp is within |v / delta| * 2^-24 <= 2^-17 of
+// Q = v / delta (|Q| < 128), and fl(Q) within 2^-18 of Q, so fl(Q) and P
+// differ by less than 2^-16.  fma(v, rcp, 1.5 * 2^23) rounds P to its
+// nearest integer k (the code, in the low byte), and fma(v, rcp, -k) is
+// P - k rounded once (error <= 2^-25).  When that is below 1/2 - 2^-15 in
+// magnitude, P is farther than 2^-15 - 2^-25 from every half-integer, so
+// fl(Q) lies on the same side and rounds to k too.  Otherwise -- a value
+// within ~2^-15 of a rounding boundary -- the quotient is taken with an
+// IEEE division.
+constexpr float kNearTie = 0.5f - 0x1p-15f;
 
 // Two IEEE fp32 products at once (sm_100 packed fp32 pipe), each rounded
 // to nearest even exactly as a scalar __fmul_rn would be.
@@ -154,21 +162,72 @@ __device__ __forceinline__ float2 fmul2_rn(float2 a, float2 b) {
   return *reinterpret_cast<float2 *>(&d);
 }
 
-// Codes for a row whose scale r = 127/m comes from the row's own absmax m:
-// |v| <= m implies |fl(v*r)| <= fl(m*r) <= 127 + 2^-17, which rounds to at
-// most 127, so the [-127, 127] clamp can never act: the low byte of
-// code_word(v, r) is the code.
-__device__ __forceinline__ uint32_t code_word(float v, float r) {
-  return __float_as_uint(__fadd_rn(__fmul_rn(v, r), kRneShift));
+// max(a, b, c) in one instruction (sm_100 three-input max).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
 }
 
-// Two code words: the products on the packed fp32 pipe, the shifts as
-// scalar __fadd_rn, which is never contracted with the multiply into an
-// fma (a fused multiply-add would round the exact product directly and
-// break ties that the rounded product sits on).
-__device__ __forceinline__ uint2 code_word2(float v0, float v1, float r) {
-  const float2 p = fmul2_rn(make_float2(v0, v1), make_float2(r, r));
-  return make_uint2(__float_as_uint(__fadd_rn(p.x, kRneShift)), __float_as_uint(__fadd_rn(p.y, kRneShift)));
+// Two fused multiply-adds at once, each rounded once as __fmaf_rn.
+__device__ __forceinline__ float2 ffma2_rn(float2 a, float2 b, float2 c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;"
+      : "=l"(d)
+      : "l"(*reinterpret_cast<const uint64_t *>(&a)), "l"(*reinterpret_cast<const uint64_t *>(&b)),
+        "l"(*reinterpret_cast<const uint64_t *>(&c)));
+  return *reinterpret_cast<float2 *>(&d);
+}
+
+__device__ __forceinline__ float2 fsub2_rn(float2 a, float2 b) {
+  uint64_t d;
+  asm("sub.rn.f32x2 %0, %1, %2;"
+      : "=l"(d)
+      : "l"(*reinterpret_cast<const uint64_t *>(&a)), "l"(*reinterpret_cast<const uint64_t *>(&b)));
+  return *reinterpret_cast<float2 *>(&d);
+}
+
+// Code words (low byte = code) of n values (n even) of one row with
+// |v / delta| <= 127.5 -- every value bounded by the row's absmax m and
+// delta = fl(m / 127).  delta == 0 (an all-zero row, rcp == 0) gives 0.
+// All on the packed fp32 pipe: sh = fma(v, rcp, S) holds k, S - sh = -k
+// exactly, fma(v, rcp, -k) = P - k; one compare of the largest distance
+// per call decides whether any value needs the division.
+template <int n>
+__device__ __forceinline__ void code_words(const float *v, float delta, float rcp, uint32_t *w) {
+  const float2 r2 = make_float2(rcp, rcp), s2 = make_float2(kRneShift, kRneShift);
+  float dm = 0.0f;
+#pragma unroll
+  for (int e = 0; e < n; e += 2) {
+    const float2 v2 = make_float2(v[e], v[e + 1]);
+    const float2 sh = ffma2_rn(v2, r2, s2);
+    w[e] = __float_as_uint(sh.x);
+    w[e + 1] = __float_as_uint(sh.y);
+    const float2 d = ffma2_rn(v2, r2, fsub2_rn(s2, sh));
+    dm = fmax3(dm, fabsf(d.x), fabsf(d.y));
+  }
+  if (!(dm < kNearTie)) {  // rare: recompute the values next to a boundary exactly
+#pragma unroll
+    for (int e = 0; e < n; ++e) {
+      const float k = __fsub_rn(__uint_as_float(w[e]), kRneShift);
+      if (!(fabsf(__fmaf_rn(v[e], rcp, -k)) < kNearTie))
+        w[e] = __float_as_uint(__fadd_rn(__fdiv_rn(v[e], delta), kRneShift));
+    }
+  }
+}
+
+// Clamped code for a finite v of any magnitude (static scales):
+// clamp(rne(fl(v / delta)), -127, 127).  lim = fl(127 * delta) >=
+// 127 * delta * (1 - 2^-24), so |v| >= lim means |v / delta| > 126.5 and a
+// saturated code, which the clamped value lim also gives (lim / delta is
+// within 2^-17 of 127); below lim, |v / delta| <= 127 * (1 + 2^-24).
+__device__ __forceinline__ float clamp_to_range(float v, float lim) { return fminf(fmaxf(v, -lim), lim); }
+
+__device__ __forceinline__ int quantize_div(float v, float delta, float rcp) {
+  float vc[2] = {clamp_to_range(v, __fmul_rn(127.0f, delta)), 0.0f};
+  uint32_t w[2];
+  code_words<2>(vc, delta, rcp, w);
+  return (int)(int8_t)(w[0] & 0xffu);
 }
 
 // Bytes 0..3 of the result are the low bytes of a, b, c, d.
@@ -176,15 +235,16 @@ __device__ __forceinline__ uint32_t pack4_low(uint32_t a, uint32_t b, uint32_t c
   return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040), 0x5410);
 }
 
-// Eight code words of one 16-byte row vector, packed into 8 bytes.
-__device__ __forceinline__ uint2 codes8(const float *v, float r) {
-  const uint2 a = code_word2(v[0], v[1], r), b = code_word2(v[2], v[3], r);
-  const uint2 c = code_word2(v[4], v[5], r), d = code_word2(v[6], v[7], r);
-  return make_uint2(pack4_low(a.x, a.y, b.x, b.y), pack4_low(c.x, c.y, d.x, d.y));
+// Eight codes of one 16-byte row vector, packed into 8 bytes (4 into 4).
+__device__ __forceinline__ uint2 codes8(const float *v, float delta, float rcp) {
+  uint32_t w[8];
+  code_words<8>(v, delta, rcp, w);
+  return make_uint2(pack4_low(w[0], w[1], w[2], w[3]), pack4_low(w[4], w[5], w[6], w[7]));
 }
-__device__ __forceinline__ uint32_t codes4(const float *v, float r) {
-  const uint2 a = code_word2(v[0], v[1], r), b = code_word2(v[2], v[3], r);
-  return pack4_low(a.x, a.y, b.x, b.y);
+__device__ __forceinline__ uint32_t codes4(const float *v, float delta, float rcp) {
+  uint32_t w[4];
+  code_words<4>(v, delta, rcp, w);
+  return pack4_low(w[0], w[1], w[2], w[3]);
 }
 
 // Two fp32 values to two E4M3 codes (round to nearest even, saturating at
@@ -196,40 +256,68 @@ __device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
 }
 
 // Code formats of the quantizers.  kMax is the code magnitude a row's
-// absmax maps to (scale = absmax / kMax, multiplier kMax / absmax).
+// absmax maps to: scale delta = absmax / kMax, codes of fl(v / delta).
 //   FmtI8    symmetric INT8, codes in [-127, 127]
 //   FmtE4M3  FP8 E4M3 codes, values in [-448, 448]
-// codes8 / codes4 quantize one 16- or 8-byte row vector's values v with
-// multiplier r; code1 one value (with saturation).
+// codes8 / codes4 quantize one 16- or 8-byte vector of a dynamic row
+// (scale delta, rcp = fl(1 / delta)); code1 one value of any magnitude
+// (saturating).
 struct FmtI8 {
   static constexpr float kMax = 127.0f;
-  static __device__ __forceinline__ uint2 codes8(const float *v, float r) { return sq::codes8(v, r); }
-  static __device__ __forceinline__ uint32_t codes4(const float *v, float r) { return sq::codes4(v, r); }
-  static __device__ __forceinline__ uint8_t code1(float v, float r) { return (uint8_t)(int8_t)quantize(v, r); }
+  static __device__ __forceinline__ uint2 codes8(const float *v, float delta, float rcp) {
+    return sq::codes8(v, delta, rcp);
+  }
+  static __device__ __forceinline__ uint32_t codes4(const float *v, float delta, float rcp) {
+    return sq::codes4(v, delta, rcp);
+  }
+  static __device__ __forceinline__ uint8_t code1(float v, float delta, float rcp) {
+    return (uint8_t)(int8_t)quantize_div(v, delta, rcp);
+  }
 };
 struct FmtE4M3 {
   static constexpr float kMax = 448.0f;
-  // r == 0 only for an all-zero row, whose codes are +0 (not the signed
-  // zeros that v * 0 would give)
-  static __device__ __forceinline__ uint2 codes8(const float *v, float r) {
-    if (r == 0.0f) return make_uint2(0u, 0u);
-    float p[8];
+  // Codes of fl(v / delta) without a division per value: y = fl(v * rcp)
+  // is within |y| * 2^-22 of fl(v / delta) (two roundings of 2^-24 each,
+  // plus rcp's).  y * (1 -+ 2^-21), each rounded once, bracket that
+  // interval, and E4M3 rounding is monotone, so when both ends give the
+  // same code every value between them -- fl(v / delta) included -- does
+  // too.  Otherwise (a value next to an E4M3 midpoint) the quotient is taken
+  // with an IEEE division.  An all-zero row (delta == 0) gets codes +0.
+  static __device__ __forceinline__ void pairs(const float *v, float delta, float rcp, int n, uint32_t *out) {
+    const float2 r2 = make_float2(rcp, rcp);
+    const float2 lo2 = make_float2(1.0f - 0x1p-21f, 1.0f - 0x1p-21f), hi2 = make_float2(1.0f + 0x1p-21f, 1.0f + 0x1p-21f);
+    uint32_t diff = 0;
+    uint32_t hi[4];
 #pragma unroll
     for (int e = 0; e < 8; e += 2) {
-      const float2 q = fmul2_rn(make_float2(v[e], v[e + 1]), make_float2(r, r));
-      p[e] = q.x;
-      p[e + 1] = q.y;
+      if (e < n) {
+        const float2 y = fmul2_rn(make_float2(v[e], v[e + 1]), r2);
+        const float2 yl = fmul2_rn(y, lo2), yh = fmul2_rn(y, hi2);
+        out[e / 2] = e4m3x2(yl.x, yl.y);
+        hi[e / 2] = e4m3x2(yh.x, yh.y);
+        diff |= out[e / 2] ^ hi[e / 2];
+      }
     }
-    return make_uint2(e4m3x2(p[0], p[1]) | (e4m3x2(p[2], p[3]) << 16), e4m3x2(p[4], p[5]) | (e4m3x2(p[6], p[7]) << 16));
+    if (diff != 0u) {  // rare
+#pragma unroll
+      for (int e = 0; e < 8; e += 2)
+        if (e < n && out[e / 2] != hi[e / 2]) out[e / 2] = e4m3x2(__fdiv_rn(v[e], delta), __fdiv_rn(v[e + 1], delta));
+    }
   }
-  static __device__ __forceinline__ uint32_t codes4(const float *v, float r) {
-    if (r == 0.0f) return 0u;
-    const float2 a = fmul2_rn(make_float2(v[0], v[1]), make_float2(r, r));
-    const float2 b = fmul2_rn(make_float2(v[2], v[3]), make_float2(r, r));
-    return e4m3x2(a.x, a.y) | (e4m3x2(b.x, b.y) << 16);
+  static __device__ __forceinline__ uint2 codes8(const float *v, float delta, float rcp) {
+    if (delta == 0.0f) return make_uint2(0u, 0u);
+    uint32_t c[4];
+    pairs(v, delta, rcp, 8, c);
+    return make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
   }
-  static __device__ __forceinline__ uint8_t code1(float v, float r) {
-    return r == 0.0f ? (uint8_t)0 : (uint8_t)(e4m3x2(__fmul_rn(v, r), 0.0f) & 0xffu);
+  static __device__ __forceinline__ uint32_t codes4(const float *v, float delta, float rcp) {
+    if (delta == 0.0f) return 0u;
+    uint32_t c[4];
+    pairs(v, delta, rcp, 4, c);
+    return c[0] | (c[1] << 16);
+  }
+  static __device__ __forceinline__ uint8_t code1(float v, float delta, float) {
+    return delta == 0.0f ? (uint8_t)0 : (uint8_t)(e4m3x2(__fdiv_rn(v, delta), 0.0f) & 0xffu);
   }
 };
 

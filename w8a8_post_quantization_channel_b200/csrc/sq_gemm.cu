@@ -50,16 +50,16 @@ struct GemmSmem {
 };
 
 template <OutKind KIND, bool F8>
-__device__ __forceinline__ void store_chunk(const uint32_t (&r)[32], void *y, int64_t ldy, int row, int n0, int N,
-                                            float dx, const float *__restrict__ w_scale) {
+__device__ __forceinline__ void store_chunk(const uint32_t (&r)[32], const YDest &dst, int64_t ldy, int row, int n0,
+                                            int N, float dx, const float *__restrict__ w_scale) {
   // N % 16 == 0 and n0 % 32 == 0, so a chunk has 16 or 32 valid columns.
   const int groups16 = min(2, (N - n0) / 16);
+  constexpr int kEsz = KIND == OutKind::F16 || KIND == OutKind::BF16 ? 2 : 4;
+  constexpr int kVecs = 32 * kEsz / 16;  // 16-byte vectors of a 32-column chunk
+  uint4 out[kVecs];
   if constexpr (KIND == OutKind::I32) {
-    int32_t *yr = reinterpret_cast<int32_t *>(y) + (int64_t)row * ldy + n0;
 #pragma unroll
-    for (int g = 0; g < 8; ++g)
-      if (g / 4 < groups16)
-        reinterpret_cast<uint4 *>(yr)[g] = make_uint4(r[4 * g], r[4 * g + 1], r[4 * g + 2], r[4 * g + 3]);
+    for (int g = 0; g < 8; ++g) out[g] = make_uint4(r[4 * g], r[4 * g + 1], r[4 * g + 2], r[4 * g + 3]);
   } else {
     float v[32];
 #pragma unroll
@@ -75,11 +75,10 @@ __device__ __forceinline__ void store_chunk(const uint32_t (&r)[32], void *y, in
       }
     }
     if constexpr (KIND == OutKind::F32) {
-      float *yr = reinterpret_cast<float *>(y) + (int64_t)row * ldy + n0;
 #pragma unroll
       for (int g = 0; g < 8; ++g)
-        if (g / 4 < groups16)
-          reinterpret_cast<float4 *>(yr)[g] = make_float4(v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]);
+        out[g] = make_uint4(__float_as_uint(v[4 * g]), __float_as_uint(v[4 * g + 1]), __float_as_uint(v[4 * g + 2]),
+                            __float_as_uint(v[4 * g + 3]));
     } else {
       uint32_t p[16];
 #pragma unroll
@@ -92,19 +91,24 @@ __device__ __forceinline__ void store_chunk(const uint32_t (&r)[32], void *y, in
           p[i] = *reinterpret_cast<uint32_t *>(&h);
         }
       }
-      uint16_t *yr = reinterpret_cast<uint16_t *>(y) + (int64_t)row * ldy + n0;
 #pragma unroll
-      for (int g = 0; g < 4; ++g)
-        if (g / 2 < groups16)
-          reinterpret_cast<uint4 *>(yr)[g] = make_uint4(p[4 * g], p[4 * g + 1], p[4 * g + 2], p[4 * g + 3]);
+      for (int g = 0; g < 4; ++g) out[g] = make_uint4(p[4 * g], p[4 * g + 1], p[4 * g + 2], p[4 * g + 3]);
     }
+  }
+  // the same words to every destination (this rank's Y, and peers' copies)
+#pragma unroll 1
+  for (int d = 0; d < dst.n; ++d) {
+    uint4 *yr = reinterpret_cast<uint4 *>(static_cast<uint8_t *>(dst.p[d]) + ((int64_t)row * ldy + n0) * kEsz);
+#pragma unroll
+    for (int g = 0; g < kVecs; ++g)
+      if (g * 2 / kVecs < groups16) yr[g] = out[g];
   }
 }
 
 template <int BN, int STAGES, OutKind KIND, bool F8>
 __global__ void __launch_bounds__(kThreads, 1)
     w8a8_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                        const float *__restrict__ x_scale, const float *__restrict__ w_scale, void *__restrict__ y,
+                        const float *__restrict__ x_scale, const float *__restrict__ w_scale, const YDest dst,
                         int64_t ldy, int M, int N, int K, unsigned *err) {
   using L = GemmSmem<BN, STAGES>;
   extern __shared__ uint8_t smem_raw[];
@@ -237,7 +241,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + ab * BN + c * 32, r);
         tmem_ld_wait();
         const int n0 = nb * BN + c * 32;
-        if (row_ok && n0 < N) store_chunk<KIND, F8>(r, y, ldy, row, n0, N, dx, w_scale);
+        if (row_ok && n0 < N) store_chunk<KIND, F8>(r, dst, ldy, row, n0, N, dx, w_scale);
       }
       tc_fence_before();
       __syncwarp();
@@ -282,7 +286,7 @@ template <int STAGES, OutKind KIND, bool F8>
 __global__ void __launch_bounds__(kThreads, 1)
     w8a8_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                           const float *__restrict__ x_scale, const float *__restrict__ w_scale,
-                          void *__restrict__ y, int64_t ldy, int M, int N, int K, unsigned *err) {
+                          const YDest dst, int64_t ldy, int M, int N, int K, unsigned *err) {
   using L = PairSmem<STAGES>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -425,7 +429,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + ab * kPairBN + c * 32, r);
         tmem_ld_wait();
         const int n0 = nb * kPairBN + c * 32;
-        if (row_ok && n0 < N) store_chunk<KIND, F8>(r, y, ldy, row, n0, N, dx, w_scale);
+        if (row_ok && n0 < N) store_chunk<KIND, F8>(r, dst, ldy, row, n0, N, dx, w_scale);
       }
       tc_fence_before();
       __syncwarp();
@@ -474,17 +478,25 @@ struct DecSmem {
 };
 
 template <OutKind KIND, bool F8>
-__device__ __forceinline__ void store_one(void *y, int64_t ldy, int t, int n, uint32_t acc, float dx, float dw) {
+__device__ __forceinline__ void store_one(const YDest &dst, int64_t ldy, int t, int n, uint32_t acc, float dx,
+                                          float dw) {
+  const int64_t i = (int64_t)t * ldy + n;
   if constexpr (KIND == OutKind::I32) {
-    reinterpret_cast<uint32_t *>(y)[(int64_t)t * ldy + n] = acc;  // the raw accumulator
+#pragma unroll 1
+    for (int d = 0; d < dst.n; ++d) static_cast<uint32_t *>(dst.p[d])[i] = acc;  // the raw accumulator
   } else {
     const float v = __fmul_rn(__fmul_rn(acc_value<F8>(acc), dx), dw);
     if constexpr (KIND == OutKind::F32) {
-      reinterpret_cast<float *>(y)[(int64_t)t * ldy + n] = v;
+#pragma unroll 1
+      for (int d = 0; d < dst.n; ++d) static_cast<float *>(dst.p[d])[i] = v;
     } else if constexpr (KIND == OutKind::BF16) {
-      reinterpret_cast<__nv_bfloat16 *>(y)[(int64_t)t * ldy + n] = __float2bfloat16_rn(v);
+      const __nv_bfloat16 h = __float2bfloat16_rn(v);
+#pragma unroll 1
+      for (int d = 0; d < dst.n; ++d) static_cast<__nv_bfloat16 *>(dst.p[d])[i] = h;
     } else {
-      reinterpret_cast<__half *>(y)[(int64_t)t * ldy + n] = __float2half_rn(v);
+      const __half h = __float2half_rn(v);
+#pragma unroll 1
+      for (int d = 0; d < dst.n; ++d) static_cast<__half *>(dst.p[d])[i] = h;
     }
   }
 }
@@ -493,7 +505,7 @@ template <int MP, OutKind KIND, bool F8>
 __global__ void __launch_bounds__(kThreads, 1)
     w8a8_gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                             const float *__restrict__ x_scale, const float *__restrict__ w_scale,
-                            void *__restrict__ y, int64_t ldy, int M, int N, int K, int32_t *__restrict__ ws,
+                            const YDest dst, int64_t ldy, int M, int N, int K, int32_t *__restrict__ ws,
                             unsigned *__restrict__ tile_count, unsigned *err) {
   using L = DecSmem<MP>;
   extern __shared__ uint8_t smem_raw[];
@@ -637,7 +649,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (t < M && n_ok) {
             if (whole) {
               const float dx = KIND != OutKind::I32 ? __ldg(x_scale + t) : 0.0f;
-              store_one<KIND, F8>(y, ldy, t, n, r[j], dx, dw);
+              store_one<KIND, F8>(dst, ldy, t, n, r[j], dx, dw);
             } else if (r[j] != 0u) {
               // int32 sums are exact in any order; an f32 tile here has at
               // most two contributors (each CTA's share spans >= one tile's
@@ -680,7 +692,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int t = t0 + j;
                 if (t < M) {
                   const float dx = KIND != OutKind::I32 ? __ldg(x_scale + t) : 0.0f;
-                  store_one<KIND, F8>(y, ldy, t, n, acc[j], dx, dw);
+                  store_one<KIND, F8>(dst, ldy, t, n, acc[j], dx, dw);
                   __stcg(ws + (int64_t)t * N + n, 0);
                 }
               }
@@ -718,7 +730,7 @@ template <int MP, OutKind KIND, bool F8>
 __global__ void __launch_bounds__(kThreads, 1)
     w8a8_gemm_decode_cluster_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                                     const float *__restrict__ x_scale, const float *__restrict__ w_scale,
-                                    void *__restrict__ y, int64_t ldy, int M, int N, int K, int S, unsigned *err) {
+                                    const YDest dst, int64_t ldy, int M, int N, int K, int S, unsigned *err) {
   using L = DecSmem<MP>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -846,7 +858,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (whole) {
           if (t < M && n_ok) {
             const float dx = KIND != OutKind::I32 ? __ldg(x_scale + t) : 0.0f;
-            store_one<KIND, F8>(y, ldy, t, n, v, dx, dw);
+            store_one<KIND, F8>(dst, ldy, t, n, v, dx, dw);
           }
         } else {
           part[t * kDecRows + row] = v;
@@ -895,7 +907,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (n < N) {
               const float dx = KIND != OutKind::I32 ? __ldg(x_scale + t) : 0.0f;
               const float dw = KIND != OutKind::I32 ? __ldg(w_scale + n) : 0.0f;
-              store_one<KIND, F8>(y, ldy, t, n, sum[b], dx, dw);
+              store_one<KIND, F8>(dst, ldy, t, n, sum[b], dx, dw);
             }
           }
         }
@@ -944,7 +956,7 @@ bool make_tmap_i8(CUtensorMap *m, const int8_t *base, int64_t rows, int64_t cols
 
 template <int BN, int STAGES, OutKind KIND, bool F8>
 cudaError_t launch_tc(const CUtensorMap &tmA, const CUtensorMap &tmB, const float *x_scale, const float *w_scale,
-                      void *y, int64_t ldy, int M, int N, int K, cudaStream_t st) {
+                      const YDest &dst, int64_t ldy, int M, int N, int K, cudaStream_t st) {
   using L = GemmSmem<BN, STAGES>;
   auto kern = w8a8_gemm_tc_kernel<BN, STAGES, KIND, F8>;
   static bool attr_set[64] = {};
@@ -957,18 +969,18 @@ cudaError_t launch_tc(const CUtensorMap &tmA, const CUtensorMap &tmB, const floa
   }
   const int tiles = ((M + kBM - 1) / kBM) * ((N + BN - 1) / BN);
   const int grid = tiles < num_sms() ? tiles : num_sms();
-  return launch_pdl(kern, dim3(grid), dim3(kThreads), L::kTotal, st, 1, tmA, tmB, x_scale, w_scale, y, ldy, M, N, K,
+  return launch_pdl(kern, dim3(grid), dim3(kThreads), L::kTotal, st, 1, tmA, tmB, x_scale, w_scale, dst, ldy, M, N, K,
                     device_error_word());
 }
 
 template <int STAGES, OutKind KIND, bool F8>
 cudaError_t launch_pair(const CUtensorMap &tmA, const CUtensorMap &tmB, const float *x_scale, const float *w_scale,
-                        void *y, int64_t ldy, int M, int N, int K, int max_clusters, cudaStream_t st) {
+                        const YDest &dst, int64_t ldy, int M, int N, int K, int max_clusters, cudaStream_t st) {
   using L = PairSmem<STAGES>;
   auto kern = w8a8_gemm_pair_kernel<STAGES, KIND, F8>;
   const int tiles = ((M + 2 * kBM - 1) / (2 * kBM)) * ((N + kPairBN - 1) / kPairBN);
   const int clusters = tiles < max_clusters ? tiles : max_clusters;
-  return launch_pdl(kern, dim3(2 * clusters), dim3(kThreads), L::kTotal, st, 2, tmA, tmB, x_scale, w_scale, y, ldy, M,
+  return launch_pdl(kern, dim3(2 * clusters), dim3(kThreads), L::kTotal, st, 2, tmA, tmB, x_scale, w_scale, dst, ldy, M,
                     N, K, device_error_word());
 }
 
@@ -1054,17 +1066,18 @@ int cluster_capacity(int S) {
 
 template <int MP, OutKind KIND, bool F8>
 cudaError_t launch_decode_cluster(const CUtensorMap &tmW, const CUtensorMap &tmX, const float *x_scale,
-                                  const float *w_scale, int M, int N, int K, void *y, int64_t ldy, int nt, int S,
+                                  const float *w_scale, int M, int N, int K, const YDest &dst, int64_t ldy, int nt,
+                                  int S,
                                   cudaStream_t st) {
   using L = DecSmem<MP>;
   prepare_decode_cluster_kernel<MP, KIND, F8>();
   return launch_pdl(w8a8_gemm_decode_cluster_kernel<MP, KIND, F8>, dim3(nt * S), dim3(kThreads), L::kTotal, st,
-                    (unsigned)S, tmW, tmX, x_scale, w_scale, y, ldy, M, N, K, S, device_error_word());
+                    (unsigned)S, tmW, tmX, x_scale, w_scale, dst, ldy, M, N, K, S, device_error_word());
 }
 
 template <int MP, OutKind KIND, bool F8>
 cudaError_t launch_decode(const int8_t *xq, const float *x_scale, const int8_t *wq, const float *w_scale, int M,
-                          int N, int K, void *y, int64_t ldy, void *workspace, cudaStream_t st) {
+                          int N, int K, const YDest &dst, int64_t ldy, void *workspace, cudaStream_t st) {
   using L = DecSmem<MP>;
   auto kern = w8a8_gemm_decode_kernel<MP, KIND, F8>;
   static bool attr_set[64] = {};
@@ -1084,24 +1097,24 @@ cudaError_t launch_decode(const int8_t *xq, const float *x_scale, const int8_t *
     int S = 1;
     for (int cand = 2; cand <= 16; cand *= 2)
       if (cand <= nk && (int64_t)nt * cand <= num_sms() && cluster_capacity<MP, KIND, F8>(cand) >= nt) S = cand;
-    return launch_decode_cluster<MP, KIND, F8>(tmW, tmX, x_scale, w_scale, M, N, K, y, ldy, nt, S, st);
+    return launch_decode_cluster<MP, KIND, F8>(tmW, tmX, x_scale, w_scale, M, N, K, dst, ldy, nt, S, st);
   }
   const int64_t items = (int64_t)nt * nk;
   const int grid = (int)(items < num_sms() ? items : num_sms());
   int32_t *ws = static_cast<int32_t *>(workspace);
   unsigned *counts = reinterpret_cast<unsigned *>(static_cast<uint8_t *>(workspace) + decode_ws_elems(M, N) * 4);
-return launch_pdl(kern, dim3(grid), dim3(kThreads), L::kTotal, st, 1, tmW, tmX, x_scale, w_scale, y, ldy, M, N, K,
+return launch_pdl(kern, dim3(grid), dim3(kThreads), L::kTotal, st, 1, tmW, tmX, x_scale, w_scale, dst, ldy, M, N, K,
                     ws, counts, device_error_word());
 }
 
 template <OutKind KIND, bool F8>
 cudaError_t gemm_dispatch(const int8_t *xq, const float *x_scale, const int8_t *wq, const float *w_scale, int M,
-                          int N, int K, void *y, int64_t ldy, void *workspace, cudaStream_t st) {
+                          int N, int K, const YDest &dst, int64_t ldy, void *workspace, cudaStream_t st) {
   if (M <= kDecodeMaxM) {  // weight-streaming regime
-    if (M <= 16) return launch_decode<16, KIND, F8>(xq, x_scale, wq, w_scale, M, N, K, y, ldy, workspace, st);
-    if (M <= 32) return launch_decode<32, KIND, F8>(xq, x_scale, wq, w_scale, M, N, K, y, ldy, workspace, st);
-    if (M <= 48) return launch_decode<48, KIND, F8>(xq, x_scale, wq, w_scale, M, N, K, y, ldy, workspace, st);
-    return launch_decode<64, KIND, F8>(xq, x_scale, wq, w_scale, M, N, K, y, ldy, workspace, st);
+    if (M <= 16) return launch_decode<16, KIND, F8>(xq, x_scale, wq, w_scale, M, N, K, dst, ldy, workspace, st);
+    if (M <= 32) return launch_decode<32, KIND, F8>(xq, x_scale, wq, w_scale, M, N, K, dst, ldy, workspace, st);
+    if (M <= 48) return launch_decode<48, KIND, F8>(xq, x_scale, wq, w_scale, M, N, K, dst, ldy, workspace, st);
+    return launch_decode<64, KIND, F8>(xq, x_scale, wq, w_scale, M, N, K, dst, ldy, workspace, st);
   }
   const int sms = num_sms();
   CUtensorMap tmA, tmB;
@@ -1111,17 +1124,17 @@ cudaError_t gemm_dispatch(const int8_t *xq, const float *x_scale, const int8_t *
   if (cap > 0 && tiles_pair >= cap) {
     if (!make_tmap_i8(&tmA, xq, M, K, kBM)) return cudaErrorInvalidValue;
     if (!make_tmap_i8(&tmB, wq, N, K, kPairBN / 2)) return cudaErrorInvalidValue;
-    return launch_pair<kPairStages, KIND, F8>(tmA, tmB, x_scale, w_scale, y, ldy, M, N, K, cap, st);
+    return launch_pair<kPairStages, KIND, F8>(tmA, tmB, x_scale, w_scale, dst, ldy, M, N, K, cap, st);
   }
   const int tiles256 = ((M + kBM - 1) / kBM) * ((N + 255) / 256);
   const bool wide = tiles256 >= sms || (N % 256 == 0 && tiles256 * 2 > sms);
   if (!make_tmap_i8(&tmA, xq, M, K, kBM)) return cudaErrorInvalidValue;
   if (wide) {
     if (!make_tmap_i8(&tmB, wq, N, K, 256)) return cudaErrorInvalidValue;
-    return launch_tc<256, 4, KIND, F8>(tmA, tmB, x_scale, w_scale, y, ldy, M, N, K, st);
+    return launch_tc<256, 4, KIND, F8>(tmA, tmB, x_scale, w_scale, dst, ldy, M, N, K, st);
   }
   if (!make_tmap_i8(&tmB, wq, N, K, 128)) return cudaErrorInvalidValue;
-  return launch_tc<128, 6, KIND, F8>(tmA, tmB, x_scale, w_scale, y, ldy, M, N, K, st);
+  return launch_tc<128, 6, KIND, F8>(tmA, tmB, x_scale, w_scale, dst, ldy, M, N, K, st);
 }
 
 }  // namespace
@@ -1133,21 +1146,30 @@ size_t w8a8_workspace_bytes(int64_t M, int64_t N, int64_t) {
 
 template <bool F8>
 cudaError_t gemm_kind(const int8_t *xq, const float *x_scale, const int8_t *wq, const float *w_scale, int m, int n,
-                      int k, void *y, OutKind kind, int64_t ldy, void *ws, cudaStream_t st) {
+                      int k, const YDest &dst, OutKind kind, int64_t ldy, void *ws, cudaStream_t st) {
   switch (kind) {
-    case OutKind::F32: return gemm_dispatch<OutKind::F32, F8>(xq, x_scale, wq, w_scale, m, n, k, y, ldy, ws, st);
-    case OutKind::F16: return gemm_dispatch<OutKind::F16, F8>(xq, x_scale, wq, w_scale, m, n, k, y, ldy, ws, st);
-    case OutKind::BF16: return gemm_dispatch<OutKind::BF16, F8>(xq, x_scale, wq, w_scale, m, n, k, y, ldy, ws, st);
-    default: return gemm_dispatch<OutKind::I32, F8>(xq, nullptr, wq, nullptr, m, n, k, y, ldy, ws, st);
+    case OutKind::F32: return gemm_dispatch<OutKind::F32, F8>(xq, x_scale, wq, w_scale, m, n, k, dst, ldy, ws, st);
+    case OutKind::F16: return gemm_dispatch<OutKind::F16, F8>(xq, x_scale, wq, w_scale, m, n, k, dst, ldy, ws, st);
+    case OutKind::BF16: return gemm_dispatch<OutKind::BF16, F8>(xq, x_scale, wq, w_scale, m, n, k, dst, ldy, ws, st);
+    default: return gemm_dispatch<OutKind::I32, F8>(xq, nullptr, wq, nullptr, m, n, k, dst, ldy, ws, st);
   }
+}
+
+cudaError_t launch_w8a8_gemm_dest(const int8_t *xq, const float *x_scale, const int8_t *wq, const float *w_scale,
+                                  int64_t M, int64_t N, int64_t K, const YDest &dst, OutKind kind, int64_t ldy,
+                                  void *ws, cudaStream_t st, QFmt fmt) {
+  const int m = (int)M, n = (int)N, k = (int)K;
+  if (fmt == QFmt::E4M3) return gemm_kind<true>(xq, x_scale, wq, w_scale, m, n, k, dst, kind, ldy, ws, st);
+  return gemm_kind<false>(xq, x_scale, wq, w_scale, m, n, k, dst, kind, ldy, ws, st);
 }
 
 cudaError_t launch_w8a8_gemm(const int8_t *xq, const float *x_scale, const int8_t *wq, const float *w_scale,
                              int64_t M, int64_t N, int64_t K, void *y, OutKind kind, int64_t ldy, void *ws, size_t,
                              cudaStream_t st, QFmt fmt) {
-  const int m = (int)M, n = (int)N, k = (int)K;
-  if (fmt == QFmt::E4M3) return gemm_kind<true>(xq, x_scale, wq, w_scale, m, n, k, y, kind, ldy, ws, st);
-  return gemm_kind<false>(xq, x_scale, wq, w_scale, m, n, k, y, kind, ldy, ws, st);
+  YDest dst{};
+  dst.p[0] = y;
+  dst.n = 1;
+  return launch_w8a8_gemm_dest(xq, x_scale, wq, w_scale, M, N, K, dst, kind, ldy, ws, st, fmt);
 }
 
 }  // namespace sq

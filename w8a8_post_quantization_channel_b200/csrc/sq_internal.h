@@ -58,7 +58,19 @@ cudaError_t launch_quant_static(const void *x, sq_dtype xt, int64_t rows, int64_
 // Output kinds of the tensor-core GEMM epilogue (I32: the raw 32-bit
 // accumulator -- an int32 sum for INT8 operands, an f32 sum for E4M3).
 enum class OutKind { F32, F16, BF16, I32 };
+// Where the epilogue stores Y: n destination matrices (this rank's Y and,
+// for a column-parallel linear, peers' copies -- possibly peer-mapped
+// pointers), each [M][ldy] and already offset to this shard's first column.
+// Every tile is written to all n with plain stores.
+constexpr int kMaxDest = 8;
+struct YDest {
+  void *p[kMaxDest];
+  int n;
+};
 // Operands are INT8 codes (fmt I8) or E4M3 codes (fmt E4M3), both [rows][K].
+cudaError_t launch_w8a8_gemm_dest(const int8_t *xq, const float *x_scale, const int8_t *wq, const float *w_scale,
+                                  int64_t M, int64_t N, int64_t K, const YDest &dst, OutKind kind, int64_t ldy,
+                                  void *workspace, cudaStream_t st, QFmt fmt);
 cudaError_t launch_w8a8_gemm(const int8_t *xq, const float *x_scale, const int8_t *wq, const float *w_scale,
                              int64_t M, int64_t N, int64_t K, void *y, OutKind kind, int64_t ldy, void *workspace,
                              size_t workspace_bytes, cudaStream_t st, QFmt fmt);
