@@ -81,6 +81,10 @@ def _load():
             "or_quant_act_e4m3": ([f32p, i64, i64, f32p, u8p, f32p], None),
             "or_gemm_e4m3": ([u8p, u8p, i64, i64, i64, f64p], None),
             "or_dequant_f32acc": ([f32p, f32p, f32p, i64, i64, f32p], None),
+            "or_butterfly_rotate": ([f32p, i64, i64, f32p, f32p], None),
+            "or_quant_act_rotated": ([f32p, i64, i64, f32p, i64, f32p, f32p, f32p, i8p, f32p], None),
+            "or_smooth_quant_weight_rotated": ([f32p, ctypes.c_int, i64, i64, f32p, i64, f32p, f32p, f32p, i8p,
+                                                f32p], None),
         }
         for name, (args, res) in sig.items():
             fn = getattr(lib, name)
@@ -337,6 +341,63 @@ def dequant_f32acc(acc, dx, dw) -> np.ndarray:
     _load().or_dequant_f32acc(_ptr(acc, ctypes.c_float), _ptr(dx, ctypes.c_float), _ptr(dw, ctypes.c_float), M, N,
                               _ptr(y, ctypes.c_float))
     return y
+
+
+# ---------------------------------------------------------------------------
+# butterfly rotation (Givens rotations in an FFT butterfly, per n-block)
+# ---------------------------------------------------------------------------
+
+def _angles(n: int, c, s):
+    L = n.bit_length() - 1
+    if n < 2 or (1 << L) != n:
+        raise ValueError("n must be a power of two >= 2")
+    c = _f32(c).reshape(L, n // 2)
+    s = _f32(s).reshape(L, n // 2)
+    return np.ascontiguousarray(c), np.ascontiguousarray(s)
+
+
+def butterfly_rotate(v, n: int, c, s) -> np.ndarray:
+    """Every row of v [rows, K] rotated block by block (K % n == 0) by the
+    butterfly with cos/sin tables c, s [log2 n, n/2]."""
+    v = _f32(v).copy()
+    c, s = _angles(n, c, s)
+    rows, K = v.shape
+    for r in range(rows):
+        row = np.ascontiguousarray(v[r])
+        _load().or_butterfly_rotate(_ptr(row, ctypes.c_float), K, n, _ptr(c, ctypes.c_float), _ptr(s, ctypes.c_float))
+        v[r] = row
+    return v
+
+
+def quant_act_rotated(x, inv_s, n: int, c, s):
+    """(Xq, dx): per-token INT8 of the rotated smoothed activations R(x * inv_s)."""
+    x = _f32(x)
+    inv_s = _f32(inv_s)
+    c, s = _angles(n, c, s)
+    M, K = x.shape
+    xq = np.zeros((M, K), np.int8)
+    dx = np.zeros(M, np.float32)
+    work = np.zeros(K, np.float32)
+    _load().or_quant_act_rotated(_ptr(x, ctypes.c_float), M, K, _ptr(inv_s, ctypes.c_float), n,
+                                 _ptr(c, ctypes.c_float), _ptr(s, ctypes.c_float), _ptr(work, ctypes.c_float),
+                                 _ptr(xq, ctypes.c_int8), _ptr(dx, ctypes.c_float))
+    return xq, dx
+
+
+def smooth_quant_weight_rotated(w, layout: int, smooth, n: int, c, s):
+    """(Wq [N, K], dw [N]) of the rotated smoothed weights R(s * w_n)."""
+    w = _f32(w)
+    smooth = _f32(smooth)
+    c, s = _angles(n, c, s)
+    K, N = _kn(w, layout)
+    wq = np.zeros((N, K), np.int8)
+    dw = np.zeros(N, np.float32)
+    work = np.zeros(K, np.float32)
+    _load().or_smooth_quant_weight_rotated(_ptr(w, ctypes.c_float), layout, K, N, _ptr(smooth, ctypes.c_float), n,
+                                           _ptr(c, ctypes.c_float), _ptr(s, ctypes.c_float),
+                                           _ptr(work, ctypes.c_float), _ptr(wq, ctypes.c_int8),
+                                           _ptr(dw, ctypes.c_float))
+    return wq, dw
 
 
 def linear(x, inv_s, wq, dw, out_dtype: str = "f32"):

@@ -398,3 +398,89 @@ void or_dequant_f32acc(const float *acc, const float *dx, const float *dw, int64
   for (int64_t t = 0; t < M; ++t)
     for (int64_t n = 0; n < N; ++n) y[t * N + n] = (acc[t * N + n] * dx[t]) * dw[n];
 }
+
+/* ---- butterfly rotation (NEXT-4) -------------------------------------------
+ * "ButterflyQuant" (lifetechia.com): a learnable orthogonal butterfly
+ * transform of dimension n = 2^L built from Givens rotations, one per pair
+ * per stage (angles theta[L][n/2]), applied to the activations before
+ * quantization; the fixed Hadamard transform is the special case of every
+ * angle pi/4.  Readings:
+ *   - stage i (i = 0 .. L-1) pairs positions p and p + 2^i for every p
+ *     whose bit i is clear -- the FFT butterfly the section describes.  The
+ *     page's listing pairs neighbours (2j, 2j+1) at every stage without a
+ *     permutation in between, which never mixes different pairs and so
+ *     cannot give the O(n log n) transform containing Hadamard that its text
+ *     names; the pairing above is the one that does.
+ *   - the pair's index within stage i is j = ((p >> (i + 1)) << i) | (p mod 2^i)
+ *     and its rotation, with c = cos(theta[i][j]), s = sin(theta[i][j]) as
+ *     given fp32 tables, maps (a, b) = (v_p, v_{p+2^i}) to
+ *       a' = c*a - s*b,   b' = s*a + c*b   (fp32, each product rounded)
+ *   - a row of K channels is rotated block by block (K % n == 0), every
+ *     n-block with the same angles;
+ *   - with SmoothQuant, the rotation R acts on the smoothed activations and,
+ *     as R is orthogonal, on the smoothed weights' K-vectors too:
+ *     (R x~) . (R w~_n) = x~ . w~_n.  Both are then quantized as before. */
+void or_butterfly_rotate(float *v, int64_t K, int64_t n, const float *c, const float *s) {
+  int L = 0;
+  while (((int64_t)1 << L) < n) ++L;
+  for (int64_t b0 = 0; b0 < K; b0 += n) {
+    float *blk = v + b0;
+    for (int i = 0; i < L; ++i) {
+      const int64_t h = (int64_t)1 << i;
+      for (int64_t p = 0; p < n; ++p) {
+        if (p & h) continue;
+        const int64_t j = ((p >> (i + 1)) << i) | (p & (h - 1));
+        const float ci = c[(int64_t)i * (n / 2) + j], si = s[(int64_t)i * (n / 2) + j];
+        const float a = blk[p], b = blk[p + h];
+        blk[p] = ci * a - si * b;
+        blk[p + h] = si * a + ci * b;
+      }
+    }
+  }
+}
+
+/* Per-token quantization of the rotated, smoothed activations:
+ * x^_t = R(x_t * inv_s), then as or_quant_act. */
+void or_quant_act_rotated(const float *x, int64_t M, int64_t K, const float *inv_s, int64_t n, const float *c,
+                          const float *s, float *work, int8_t *xq, float *dx) {
+  for (int64_t t = 0; t < M; ++t) {
+    for (int64_t j = 0; j < K; ++j) work[j] = x[t * K + j] * inv_s[j];
+    or_butterfly_rotate(work, K, n, c, s);
+    float m = 0.0f;
+    for (int64_t j = 0; j < K; ++j) {
+      float a = fabsf(work[j]);
+      if (a > m) m = a;
+    }
+    if (m == 0.0f) {
+      dx[t] = 0.0f;
+      for (int64_t j = 0; j < K; ++j) xq[t * K + j] = 0;
+      continue;
+    }
+    dx[t] = m / 127.0f;
+    for (int64_t j = 0; j < K; ++j) xq[t * K + j] = or_quantize_value(work[j], dx[t]);
+  }
+}
+
+/* Per-output-channel quantization of the rotated, smoothed weights:
+ * w^_n = R(s * w_n) over the K input channels, then as
+ * or_smooth_quant_weight.  Wq [N][K]. */
+void or_smooth_quant_weight_rotated(const float *w, int layout, int64_t K, int64_t N, const float *smooth,
+                                    int64_t n, const float *c, const float *s, float *work, int8_t *wq,
+                                    float *dw) {
+  for (int64_t o = 0; o < N; ++o) {
+    for (int64_t j = 0; j < K; ++j) work[j] = smooth[j] * w_at(w, layout, K, N, j, o);
+    or_butterfly_rotate(work, K, n, c, s);
+    float m = 0.0f;
+    for (int64_t j = 0; j < K; ++j) {
+      float a = fabsf(work[j]);
+      if (a > m) m = a;
+    }
+    if (m == 0.0f) {
+      dw[o] = 0.0f;
+      for (int64_t j = 0; j < K; ++j) wq[o * K + j] = 0;
+      continue;
+    }
+    dw[o] = m / 127.0f;
+    for (int64_t j = 0; j < K; ++j) wq[o * K + j] = or_quantize_value(work[j], dw[o]);
+  }
+}
