@@ -226,6 +226,38 @@ sq_status sq_w8a8_linear_scatter(const int8_t *xq, const float *x_scale,
                                  size_t workspace_bytes, sq_stream_t stream);
 
 /*
+ * Outlier handling beyond smoothing: a butterfly rotation before the INT8
+ * quantization ("ButterflyQuant", lifetechia.com: an orthogonal transform
+ * built from Givens rotations in an FFT butterfly, O(n log n), with the
+ * Hadamard transform as the special case of every angle pi/4).  Rows are
+ * rotated block by block, blocks of n = 2^L channels (K % n == 0):
+ *   stage i = 0 .. L-1 pairs positions p and p + 2^i (bit i of p clear);
+ *   the pair's index is j = ((p >> (i + 1)) << i) | (p mod 2^i);
+ *   (a, b) -> (c a - s b, s a + c b), (c, s) = rot_cs[i][j][0..1],
+ *   each product and sum an IEEE fp32 operation.
+ * As the rotation R is orthogonal, (R x~) . (R w~_n) = x~ . w~_n: rotating
+ * both the smoothed activations and the smoothed weights' K-vectors keeps
+ * the product while spreading outliers over a block.
+ *   rot_cs   [L][n / 2][2] fp32 (cos, sin) pairs, device memory.
+ *   n        2 <= n <= 256 (16-bit rows) or 128 (fp32 rows), a power of two
+ *            dividing K; K <= 16384 (16-bit) or 8192 (fp32); else
+ *            SQ_ERR_UNSUPPORTED / SQ_ERR_INVALID_ARG.
+ * sq_quant_act_rotated: xq, x_scale of R(x * inv_smooth), as sq_quant_act.
+ * sq_smooth_quant_weight_rotated: s and 1/s as sq_smooth_quant_weight
+ *   (layout SQ_W_NK only), then wq, w_scale of R(s * w_n) per output
+ *   channel n.
+ */
+sq_status sq_quant_act_rotated(const void *x, sq_dtype xt, int64_t M, int64_t K,
+                               int64_t ldx, const float *inv_smooth, int64_t n,
+                               const float *rot_cs, int8_t *xq, float *x_scale,
+                               sq_stream_t stream);
+sq_status sq_smooth_quant_weight_rotated(const void *w, sq_dtype wt, int64_t K,
+                                         int64_t N, int64_t ldw, const float *amax,
+                                         float alpha, int64_t n, const float *rot_cs,
+                                         int8_t *wq, float *w_scale, float *smooth,
+                                         float *inv_smooth, sq_stream_t stream);
+
+/*
  * FP8 (E4M3) variant.  The survey page "Quantization Calibration
  * GPTQ/AWQ/SmoothQuant 2026" (jisaku.com glossary) lists FP8 SmoothQuant:
  * the same smoothing, with FP8 operands.  Both operands are E4M3 codes (1

@@ -94,6 +94,21 @@ def test_scatter_argument_checks_host():
     assert f(A16, A16, A16, None, 64, 256, 256, dsts, 2, sq.SQ_BF16, 256, None, 0, None) == INV
 
 
+def test_rotation_argument_checks():
+    f = sq.lib().sq_quant_act_rotated
+    assert f(None, sq.SQ_BF16, 0, 256, 256, A16, 16, A16, None, None, None) == sq.SQ_OK          # M == 0
+    assert f(A16, sq.SQ_BF16, 8, 256, 256, A16, 24, A16, A16, A16, None) == INV                  # n not 2^k
+    assert f(A16, sq.SQ_BF16, 8, 256, 256, A16, 1, A16, A16, A16, None) == INV                   # n < 2
+    assert f(A16, sq.SQ_BF16, 8, 272, 272, A16, 32, A16, A16, A16, None) == INV                  # K % n
+    assert f(A16, sq.SQ_BF16, 8, 1024, 1024, A16, 512, A16, A16, A16, None) == sq.SQ_ERR_UNSUPPORTED
+    assert f(A16, sq.SQ_F32, 8, 1024, 1024, A16, 256, A16, A16, A16, None) == sq.SQ_ERR_UNSUPPORTED
+    assert f(A16, sq.SQ_BF16, 8, 256, 256, A16, 16, None, A16, A16, None) == INV                 # null table
+    g = sq.lib().sq_smooth_quant_weight_rotated
+    a = ctypes.c_float(0.5)
+    assert g(A16, sq.SQ_BF16, 256, 64, 256, A16, ctypes.c_float(2.0), 16, A16, A16, A16, A16, A16, None) == INV
+    assert g(A16, sq.SQ_BF16, 256, 64, 256, A16, a, 12, A16, A16, A16, A16, A16, None) == INV
+
+
 def test_producer_argument_checks():
     L = sq.lib()
     fold = L.sq_fold_smooth_into_norm

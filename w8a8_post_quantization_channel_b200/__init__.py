@@ -36,7 +36,7 @@ __all__ = [
     "sq_w8a8_linear_decode_noalloc", "SQ_DECODE_STATIC_SCRATCH_BYTES", "sq_selftest_wait_timeout",
     "sq_fold_smooth_into_norm", "sq_rmsnorm_quant_act", "sq_static_act_scale", "sq_quant_act_static",
     "sq_smooth_quant_weight_e4m3", "sq_quant_act_e4m3", "sq_w8a8_linear_e4m3", "sq_w8a8_accumulate_e4m3",
-    "sq_w8a8_linear_scatter",
+    "sq_w8a8_linear_scatter", "sq_quant_act_rotated", "sq_smooth_quant_weight_rotated",
 ]
 
 SQ_OK, SQ_ERR_INVALID_ARG, SQ_ERR_UNSUPPORTED, SQ_ERR_CUDA, SQ_ERR_TIMEOUT = 0, 1, 2, 3, 4
@@ -92,6 +92,8 @@ def lib() -> ctypes.CDLL:
             "sq_w8a8_linear_e4m3": [vp, vp, vp, vp, i64, i64, i64, vp, i32, i64, vp, sz, vp],
             "sq_w8a8_accumulate_e4m3": [vp, vp, i64, i64, i64, vp, i64, vp, sz, vp],
             "sq_w8a8_linear_scatter": [vp, vp, vp, vp, i64, i64, i64, vp, i32, i32, i64, vp, sz, vp],
+            "sq_quant_act_rotated": [vp, i32, i64, i64, i64, vp, i64, vp, vp, vp, vp],
+            "sq_smooth_quant_weight_rotated": [vp, i32, i64, i64, i64, vp, f32, i64, vp, vp, vp, vp, vp, vp],
         }
         for name, args in sigs.items():
             fn = getattr(L, name)
@@ -177,6 +179,37 @@ def sq_quant_act(x: torch.Tensor, inv_smooth: torch.Tensor, xq=None, x_scale=Non
     _check(lib().sq_quant_act(_ptr(x), _dtype(x, "x"), M, K, x.stride(0), _ptr(inv_smooth), _ptr(xq),
                               _ptr(x_scale), _stream(stream)), "sq_quant_act")
     return xq, x_scale
+
+
+def sq_quant_act_rotated(x: torch.Tensor, inv_smooth: torch.Tensor, n: int, rot_cs: torch.Tensor, xq=None,
+                         x_scale=None, stream=None):
+    """(xq, x_scale) = per-token INT8 of the butterfly rotation (blocks of n,
+    (cos, sin) table rot_cs [log2 n, n/2, 2]) of x * inv_smooth."""
+    _rowmajor(x, "x")
+    M, K = x.shape
+    xq = torch.empty((M, K), dtype=torch.int8, device=x.device) if xq is None else xq
+    x_scale = torch.empty(M, dtype=torch.float32, device=x.device) if x_scale is None else x_scale
+    _check(lib().sq_quant_act_rotated(_ptr(x), _dtype(x, "x"), M, K, x.stride(0), _ptr(inv_smooth), n, _ptr(rot_cs),
+                                      _ptr(xq), _ptr(x_scale), _stream(stream)), "sq_quant_act_rotated")
+    return xq, x_scale
+
+
+def sq_smooth_quant_weight_rotated(w: torch.Tensor, amax: torch.Tensor, alpha: float, n: int, rot_cs: torch.Tensor,
+                                   wq=None, w_scale=None, smooth=None, inv_smooth=None, stream=None):
+    """(wq [N,K] int8, w_scale, s, inv_s) with every output channel's smoothed
+    K-vector rotated like the activations; w is [N, K] (nn.Linear layout)."""
+    _rowmajor(w, "w")
+    N, K = w.shape
+    dev = w.device
+    wq = torch.empty((N, K), dtype=torch.int8, device=dev) if wq is None else wq
+    w_scale = torch.empty(N, dtype=torch.float32, device=dev) if w_scale is None else w_scale
+    smooth = torch.empty(K, dtype=torch.float32, device=dev) if smooth is None else smooth
+    inv_smooth = torch.empty(K, dtype=torch.float32, device=dev) if inv_smooth is None else inv_smooth
+    _check(lib().sq_smooth_quant_weight_rotated(_ptr(w), _dtype(w, "w"), K, N, w.stride(0), _ptr(amax),
+                                                ctypes.c_float(alpha), n, _ptr(rot_cs), _ptr(wq), _ptr(w_scale),
+                                                _ptr(smooth), _ptr(inv_smooth), _stream(stream)),
+           "sq_smooth_quant_weight_rotated")
+    return wq, w_scale, smooth, inv_smooth
 
 
 def sq_fold_smooth_into_norm(gamma: torch.Tensor, inv_smooth: torch.Tensor, gs=None, stream=None) -> torch.Tensor:

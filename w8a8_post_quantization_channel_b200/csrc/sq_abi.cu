@@ -160,6 +160,53 @@ sq_status sq_quant_act(const void *x, sq_dtype xt, int64_t M, int64_t K, int64_t
   return quant_act_impl(x, xt, M, K, ldx, inv_smooth, xq, x_scale, sq::QFmt::I8, stream);
 }
 
+static int log2_exact(int64_t n) {
+  int l = 0;
+  while (l < 62 && ((int64_t)1 << l) < n) ++l;
+  return ((int64_t)1 << l) == n ? l : -1;
+}
+
+static sq_status rot_checks(sq_dtype xt, int64_t K, int64_t n, const float *rot_cs, int *logn) {
+  *logn = log2_exact(n);
+  if (*logn < 1 || K % n != 0 || !valid_vec(rot_cs)) return SQ_ERR_INVALID_ARG;
+  if (n > (xt == SQ_F32 ? 128 : 256) || K > (xt == SQ_F32 ? 8192 : 16384)) return SQ_ERR_UNSUPPORTED;
+  return SQ_OK;
+}
+
+sq_status sq_quant_act_rotated(const void *x, sq_dtype xt, int64_t M, int64_t K, int64_t ldx, const float *inv_smooth,
+                               int64_t n, const float *rot_cs, int8_t *xq, float *x_scale, sq_stream_t stream) {
+  if (!valid_dtype(xt) || K <= 0 || K % 16 != 0 || K >= kMaxDim || M < 0 || M >= kMaxDim) return SQ_ERR_INVALID_ARG;
+  if (ldx < K || (ldx * dsize(xt)) % 16 != 0 || !valid_vec(inv_smooth)) return SQ_ERR_INVALID_ARG;
+  int logn = 0;
+  const sq_status rs = rot_checks(xt, K, n, rot_cs, &logn);
+  if (rs != SQ_OK) return rs;
+  if (M == 0) return SQ_OK;
+  if (!valid_matrix(x, xt, M, K, ldx) || !valid_vec(xq) || !valid_vec(x_scale)) return SQ_ERR_INVALID_ARG;
+  return from_cuda(
+      sq::launch_rot_quant_rows(x, xt, M, K, ldx, inv_smooth, logn, rot_cs, xq, x_scale, (cudaStream_t)stream));
+}
+
+sq_status sq_smooth_quant_weight_rotated(const void *w, sq_dtype wt, int64_t K, int64_t N, int64_t ldw,
+                                         const float *amax, float alpha, int64_t n, const float *rot_cs, int8_t *wq,
+                                         float *w_scale, float *smooth, float *inv_smooth, sq_stream_t stream) {
+  if (!valid_dtype(wt) || K <= 0 || N <= 0 || K % 16 != 0 || N % 16 != 0) return SQ_ERR_INVALID_ARG;
+  if (!(alpha >= 0.0f && alpha <= 1.0f)) return SQ_ERR_INVALID_ARG;
+  if (!valid_matrix(w, wt, N, K, ldw)) return SQ_ERR_INVALID_ARG;
+  if (!valid_vec(amax) || !valid_vec(wq) || !valid_vec(w_scale) || !valid_vec(smooth) || !valid_vec(inv_smooth))
+    return SQ_ERR_INVALID_ARG;
+  int logn = 0;
+  const sq_status rs = rot_checks(wt, K, n, rot_cs, &logn);
+  if (rs != SQ_OK) return rs;
+  cudaStream_t st = (cudaStream_t)stream;
+  // w_j = max_n |W_jn| into `smooth`, then s_j and 1/s_j as without rotation
+  cudaError_t e = sq::launch_zero_fill(smooth, K, st);
+  if (e == cudaSuccess) e = sq::launch_absmax_cols(w, wt, N, K, ldw, nullptr, smooth, true, st);
+  if (e == cudaSuccess) e = sq::launch_smooth_factor(amax, smooth, inv_smooth, K, alpha, st);
+  // rows R(s * w_n), per-output-channel INT8
+  if (e == cudaSuccess) e = sq::launch_rot_quant_rows(w, wt, N, K, ldw, smooth, logn, rot_cs, wq, w_scale, st);
+  return from_cuda(e);
+}
+
 sq_status sq_quant_act_e4m3(const void *x, sq_dtype xt, int64_t M, int64_t K, int64_t ldx, const float *inv_smooth,
                             uint8_t *xq, float *x_scale, sq_stream_t stream) {
   return quant_act_impl(x, xt, M, K, ldx, inv_smooth, reinterpret_cast<int8_t *>(xq), x_scale, sq::QFmt::E4M3,

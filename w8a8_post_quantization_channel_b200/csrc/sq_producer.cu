@@ -300,3 +300,211 @@ cudaError_t launch_quant_static(const void *x, sq_dtype xt, int64_t rows, int64_
 }
 
 }  // namespace sq
+
+// ---------------------------------------------------------------------------
+// Butterfly rotation before quantization ("ButterflyQuant", lifetechia.com:
+// Givens rotations arranged as an FFT butterfly).  Each row v = x * col_scale
+// is rotated block by block (blocks of n = 2^L channels); stage i pairs
+// positions p and p + 2^i (bit i of p clear), pair j = ((p >> (i+1)) << i) |
+// (p mod 2^i), and maps (a, b) to (c a - s b, s a + c b) with (c, s) =
+// cs[i][j].  Then per-row INT8 as quant_rows_kernel.
+// A warp holds 32 consecutive 16-byte vectors (32 V channels, aligned), so a
+// block of n <= 32 V channels lives in one warp, and a lane's channel
+// positions within its block are the same for every vector it holds and
+// every row.  The CTA therefore lays the table out once per lane:
+//   strides below V (both values in one thread), per pair k of the vector:
+//     tin[i][k][lane] = (c, s, -s, c)  ->  (a', b') = (c a, s a) + (-s b, c b)
+//   strides of whole lanes (partner lane ^ (h / V)), per value e:
+//     tsh[i][e / 2][lane] = (c_e, c_e+1, s'_e, s'_e+1)  ->  x' = c x + s' y
+//     with s' = -s in the pair's first position, +s in its second,
+// so a warp reads 512 contiguous bytes per access (no bank conflicts) and
+// the arithmetic runs on the packed fp32 pipe: the same products, negations
+// (exact) and sums as the definition.
+// ---------------------------------------------------------------------------
+namespace sq {
+namespace {
+
+constexpr int kRotMaxStages = 8;  // n <= 256
+
+template <typename T, int kVPT>
+__global__ void __launch_bounds__(kRowMaxThreads)
+    rot_quant_rows_kernel(const T *__restrict__ x, int64_t rows, int64_t nvec, int64_t ld,
+                          const float *__restrict__ col_scale, int logn, const float2 *__restrict__ cs,
+                          int8_t *__restrict__ q, float *__restrict__ row_scale_out) {
+  constexpr int V = Vec<T>::N;
+  constexpr int kLogV = V == 8 ? 3 : 2;
+  extern __shared__ float4 rtab[];  // [logn][V / 2][32]
+  __shared__ float red[2][kRowMaxThreads / 32];
+  const int n = 1 << logn;
+  const int half = n >> 1;
+  pdl_wait();  // the previous kernel's results are visible from here on
+  pdl_trigger();
+  // per-lane table: entry (st, k, l) for k < V / 2
+  for (int idx = threadIdx.x; idx < logn * (V / 2) * 32; idx += blockDim.x) {
+    const int l = idx & 31, k = (idx >> 5) % (V / 2), st = idx / (32 * (V / 2));
+    const int h = 1 << st;
+    const int base = (l * V) & (n - 1);  // this lane's first position in its block
+    float4 t;
+    if (h < V) {
+      // k-th pair of the vector at this stride: lower element e
+      const int e = ((k / h) * 2 * h) + (k % h);
+      const int p = (base + e) & (n - 1);
+      const float2 c = (st < logn) ? cs[st * half + (((p >> (st + 1)) << st) | (p & (h - 1)))] : make_float2(1, 0);
+      t = make_float4(c.x, c.y, -c.y, c.x);
+    } else {
+      float cc[2], ss[2];
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int p = base + 2 * k + u;
+        const bool first = (p & h) == 0;
+        const int pa = first ? p : p - h;
+        const float2 c = cs[st * half + (((pa >> (st + 1)) << st) | (pa & (h - 1)))];
+        cc[u] = c.x;
+        ss[u] = first ? -c.y : c.y;
+      }
+      t = make_float4(cc[0], cc[1], ss[0], ss[1]);
+    }
+    rtab[idx] = t;
+  }
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int nwarps = blockDim.x >> 5;
+  const int64_t K = nvec * V;
+  float sc[kVPT][V];
+#pragma unroll
+  for (int i = 0; i < kVPT; ++i) {
+    const int64_t v = tid + (int64_t)i * blockDim.x;
+#pragma unroll
+    for (int e = 0; e < V; ++e) sc[i][e] = v < nvec ? __ldg(col_scale + v * V + e) : 0.0f;
+  }
+  __syncthreads();
+  const uint64_t policy = policy_evict_first();
+  uint4 cur[kVPT], nxt[kVPT];
+  int64_t r = blockIdx.x;
+#pragma unroll
+  for (int i = 0; i < kVPT; ++i) {
+    const int64_t v = tid + (int64_t)i * blockDim.x;
+    cur[i] = (r < rows && v < nvec) ? ld_policy_v4(x + r * ld + v * V, policy) : make_uint4(0, 0, 0, 0);
+  }
+  int slot = 0;
+  for (; r < rows; r += gridDim.x) {
+    const int64_t rn = r + gridDim.x;
+#pragma unroll
+    for (int i = 0; i < kVPT; ++i) {
+      const int64_t v = tid + (int64_t)i * blockDim.x;
+      nxt[i] = (rn < rows && v < nvec) ? ld_policy_v4(x + rn * ld + v * V, policy) : make_uint4(0, 0, 0, 0);
+    }
+    float val[kVPT][V];
+#pragma unroll
+    for (int i = 0; i < kVPT; ++i) {
+      float f[V];
+      Vec<T>::to_f32(cur[i], f);
+#pragma unroll
+      for (int e = 0; e < V; e += 2) {
+        const float2 p = fmul2_rn(make_float2(f[e], f[e + 1]), make_float2(sc[i][e], sc[i][e + 1]));
+        val[i][e] = p.x;
+        val[i][e + 1] = p.y;
+      }
+    }
+    // strides below V: both values of a pair in this thread
+#pragma unroll
+    for (int st = 0; st < kLogV; ++st) {
+      if (st < logn) {
+        constexpr int kPairs = V / 2;
+#pragma unroll
+        for (int k = 0; k < kPairs; ++k) {
+          const int h = 1 << st;
+          const int e = ((k / h) * 2 * h) + (k % h);
+          const float4 t = rtab[(st * kPairs + k) * 32 + lane];
+#pragma unroll
+          for (int i = 0; i < kVPT; ++i) {
+            const float a = val[i][e], b = val[i][e + h];
+            const float2 p1 = fmul2_rn(make_float2(a, a), make_float2(t.x, t.y));  // (c a, s a)
+            const float2 p2 = fmul2_rn(make_float2(b, b), make_float2(t.z, t.w));  // (-s b, c b)
+            val[i][e] = __fadd_rn(p1.x, p2.x);
+            val[i][e + h] = __fadd_rn(p1.y, p2.y);
+          }
+        }
+      }
+    }
+    // strides of whole lanes: every lane takes part in every shuffle
+#pragma unroll
+    for (int st = kLogV; st < kLogV + 5 && st < kRotMaxStages; ++st) {
+      if (st < logn) {
+        const int lm = (1 << st) / V;
+#pragma unroll
+        for (int e = 0; e < V; e += 2) {
+          const float4 t = rtab[(st * (V / 2) + e / 2) * 32 + lane];
+#pragma unroll
+          for (int i = 0; i < kVPT; ++i) {
+            const float y0 = __shfl_xor_sync(0xffffffffu, val[i][e], lm);
+            const float y1 = __shfl_xor_sync(0xffffffffu, val[i][e + 1], lm);
+            const float2 cx = fmul2_rn(make_float2(val[i][e], val[i][e + 1]), make_float2(t.x, t.y));
+            const float2 sy = fmul2_rn(make_float2(y0, y1), make_float2(t.z, t.w));
+            val[i][e] = __fadd_rn(cx.x, sy.x);
+            val[i][e + 1] = __fadd_rn(cx.y, sy.y);
+          }
+        }
+      }
+    }
+    float m = 0.0f;
+#pragma unroll
+    for (int i = 0; i < kVPT; ++i)
+#pragma unroll
+      for (int e = 0; e < V; e += 2) m = fmax3(m, fabsf(val[i][e]), fabsf(val[i][e + 1]));
+    m = warp_max(m);
+    if (lane == 0) red[slot][warp] = m;
+    __syncthreads();
+    m = 0.0f;
+    for (int w = 0; w < nwarps; ++w) m = fmaxf(m, red[slot][w]);
+    slot ^= 1;
+    const float delta = __fdiv_rn(m, 127.0f);
+    const float rcp = m > 0.0f ? __frcp_rn(delta) : 0.0f;
+    if (tid == 0) row_scale_out[r] = delta;
+    int8_t *qrow = q + r * K;
+#pragma unroll
+    for (int i = 0; i < kVPT; ++i) {
+      const int64_t v = tid + (int64_t)i * blockDim.x;
+      if (v < nvec) {
+        if constexpr (V == 8) {
+          *reinterpret_cast<uint2 *>(qrow + v * V) = codes8(val[i], delta, rcp);
+        } else {
+          *reinterpret_cast<uint32_t *>(qrow + v * V) = codes4(val[i], delta, rcp);
+        }
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < kVPT; ++i) cur[i] = nxt[i];
+  }
+}
+
+template <typename T>
+cudaError_t rot_quant_t(const void *x, int64_t rows, int64_t cols, int64_t ld, const float *col_scale, int logn,
+                        const float *cs, int8_t *q, float *row_scale_out, cudaStream_t st) {
+  constexpr int V = Vec<T>::N;
+  const int64_t nvec = cols / V;
+  if (nvec > 4 * kRowMaxThreads || (1 << logn) > 32 * V) return cudaErrorNotSupported;
+  const int vpt = nvec <= 4 * 32 ? 1 : 4;
+  const int64_t t = (nvec + vpt - 1) / vpt;
+  const int threads = (int)std::max<int64_t>(32, ((t + 31) / 32) * 32);
+  auto kern = vpt == 1 ? rot_quant_rows_kernel<T, 1> : rot_quant_rows_kernel<T, 4>;
+  const size_t smem = (size_t)logn * (V / 2) * 32 * sizeof(float4);
+  int per_sm = 0;
+  cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, smem);
+  if (e != cudaSuccess) return e;
+  const int64_t grid = std::min<int64_t>(rows, (int64_t)std::max(1, per_sm) * num_sms());
+  return launch_pdl(kern, dim3((unsigned)grid), dim3(threads), smem, st, 1, (const T *)x, rows, nvec, ld, col_scale,
+                    logn, reinterpret_cast<const float2 *>(cs), q, row_scale_out);
+}
+
+}  // namespace
+
+cudaError_t launch_rot_quant_rows(const void *x, sq_dtype xt, int64_t rows, int64_t cols, int64_t ld,
+                                  const float *col_scale, int logn, const float *cs, int8_t *q, float *row_scale_out,
+                                  cudaStream_t st) {
+  switch (xt) {
+    case SQ_F32: return rot_quant_t<float>(x, rows, cols, ld, col_scale, logn, cs, q, row_scale_out, st);
+    case SQ_F16: return rot_quant_t<__half>(x, rows, cols, ld, col_scale, logn, cs, q, row_scale_out, st);
+    default: return rot_quant_t<__nv_bfloat16>(x, rows, cols, ld, col_scale, logn, cs, q, row_scale_out, st);
+  }
+}
+}  // namespace sq

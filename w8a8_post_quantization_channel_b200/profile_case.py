@@ -7,7 +7,8 @@ of the workloads' shapes, for profilers and roofline measurements.
 
 --op is calib (T = M tokens), weight (W [N, K]), act, rmsnorm (the fused
 norm producer), static (static-scale quantizer), linear, or the FP8 (E4M3)
-forms act8, weight8 and linear8.  With
+forms act8, weight8 and linear8, or rot (butterfly-rotated act-quant, --N =
+the rotation block size).  With
 --time (implied by --sweep) every iteration is timed with CUDA events on
 the launching stream, a 512 MB buffer is read between iterations so that
 L2 (126 MB) holds none of the operands (a read leaves clean lines behind, so
@@ -54,6 +55,8 @@ SWEEPS = {
     # per-tensor quantizer on 16384-token batches
     "producer": [("rmsnorm", 16384, K, 0, "bf16") for K in (4096, 8192)] + [("rmsnorm", 2048, 4096, 0, "f16")]
                 + [("static", 16384, K, 0, "bf16") for K in (4096, 8192)],
+    # butterfly-rotated activation quantization (N = the rotation's block size n)
+    "rot": [("rot", 16384, 4096, n, "bf16") for n in (16, 64, 256)] + [("rot", 16384, 8192, 256, "bf16")],
     # FP8 (E4M3): activation quantization, weight path, prefill and decode linears
     "fp8": [("act8", 16384, 4096, 0, "bf16"), ("weight8", 0, 8192, 8192, "bf16")]
            + [("linear8", 2048, K, N, "f16") for _, K, N in synth.OPT_6_7B]
@@ -99,6 +102,17 @@ def make_case(op, M, K, N, dtype, dev="cuda"):
         if op == "calib":
             return (lambda: sq.sq_calib_absmax(x, amax)), M * K * ESZ[dtype] + 8 * K, None
         return (lambda: sq.sq_quant_act(x, inv, xq=xq, x_scale=xs)), M * K * (ESZ[dtype] + 1) + 4 * (M + K), None
+    if op == "rot":
+        x = synth.activations(M, K, o, 2, dt, device=dev)
+        inv = torch.rand(K, device=dev) + 0.5
+        n = N or 256
+        L = n.bit_length() - 1
+        theta = torch.rand(L, n // 2, generator=synth.gen(5, dev), device=dev) * 6.2831853
+        cs = torch.stack([torch.cos(theta), torch.sin(theta)], dim=-1).contiguous()
+        xq = torch.empty(M, K, dtype=torch.int8, device=dev)
+        xs = torch.empty(M, device=dev)
+        return (lambda: sq.sq_quant_act_rotated(x, inv, n, cs, xq=xq, x_scale=xs)), M * K * (ESZ[dtype] + 1) + 4 * (
+            M + K), None
     if op == "act8":
         x = synth.activations(M, K, o, 2, dt, device=dev)
         inv = torch.rand(K, device=dev) + 0.5
@@ -179,7 +193,7 @@ def time_case(op, M, K, N, dtype, iters):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--op", choices=["calib", "weight", "act", "linear", "rmsnorm", "static", "act8", "weight8",
-                                     "linear8"])
+                                     "linear8", "rot"])
     ap.add_argument("--sweep", choices=sorted(SWEEPS))
     ap.add_argument("--M", type=int, default=2048)
     ap.add_argument("--K", type=int, default=4096)
