@@ -258,7 +258,7 @@ sq_status sq_smooth_quant_weight_rotated(const void *w, sq_dtype wt, int64_t K,
                                          float *inv_smooth, sq_stream_t stream);
 
 /*
- * FP8 (E4M3) variant.  The survey page "Quantization Calibration
+ * FP8 (E4M3) variant.  The glossary page "Quantization Calibration
  * GPTQ/AWQ/SmoothQuant 2026" (jisaku.com glossary) lists FP8 SmoothQuant:
  * the same smoothing, with FP8 operands.  Both operands are E4M3 codes (1
  * sign, 4 exponent bits of bias 7, 3 mantissa bits, no infinities,

@@ -300,7 +300,7 @@ void or_quant_act_static(const float *x, int64_t M, int64_t K, const float *inv_
 }
 
 /* ---- FP8 (E4M3) variant --------------------------------------------------
- * The survey page "Quantization Calibration GPTQ/AWQ/SmoothQuant 2026"
+ * The glossary page "Quantization Calibration GPTQ/AWQ/SmoothQuant 2026"
  * (jisaku.com glossary) lists FP8 SmoothQuant: the same smoothing with FP8
  * operands (its spec-comparison table: 8-bit weights, FP8 activations).
  * Readings: both operands in E4M3 -- the 8-bit float with 1 sign bit, 4
