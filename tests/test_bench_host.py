@@ -1,0 +1,62 @@
+"""Host-side logic of bench.py, without a GPU: the source-text hash that ties
+the ncu traffic figure to the kernel it was measured on, and the parsing of
+the nvidia-smi clock samples."""
+import importlib.util
+import os
+import sys
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _bench():
+    spec = importlib.util.spec_from_file_location("bench_under_test", os.path.join(ROOT, "bench.py"))
+    mod = importlib.util.module_from_spec(spec)
+    argv = sys.argv
+    sys.argv = ["bench.py"]
+    try:
+        spec.loader.exec_module(mod)
+    finally:
+        sys.argv = argv
+    return mod
+
+
+def test_function_text_finds_definitions_not_calls():
+    b = _bench()
+    src = """
+int helper(int a);
+
+// the kernel
+template <typename T>
+__global__ void kern(const T *x) {
+  if (x) { helper(1); }
+}
+
+void launch() { kern<float><<<1, 1>>>(nullptr); }
+"""
+    t = b.function_text(src, "kern")
+    assert t.startswith("// the kernel") and t.rstrip().endswith("}")
+    assert "launch()" not in t
+    assert b.function_text(src, "launch").startswith("void launch()")
+
+
+def test_traffic_is_reported_only_for_the_measured_source(monkeypatch):
+    b = _bench()
+    entry = dict(b.TRAFFIC["absmax_cols_kernel"])
+    current = b.src_hash(entry["source"], entry["functions"])
+    monkeypatch.setitem(b.TRAFFIC, "absmax_cols_kernel", dict(entry, sha=current))
+    assert b.traffic_for("absmax_cols_kernel", 1e9) == int(round(entry["ratio"] * 1e9))
+    monkeypatch.setitem(b.TRAFFIC, "absmax_cols_kernel", dict(entry, sha="0" * 16))
+    assert b.traffic_for("absmax_cols_kernel", 1e9) is None
+    assert b.traffic_for("no_such_kernel", 1e9) is None
+
+
+def test_clock_summary_keeps_this_gpu_and_collects_reasons():
+    b = _bench()
+    c = b.ClockSampler("0000:1B:00.0")
+    row = lambda bus, mhz, pc: [bus, str(mhz), "1965", "500.0", "0x4", "Not Active", "Not Active", "Not Active", pc]
+    c.rows = [row("00000000:1B:00.0", 1965, "Active"), row("00000000:1B:00.0", 1900, "Not Active"),
+              row("00000000:3A:00.0", 600, "Not Active")]
+    s = c.summary()
+    assert s["samples"] == 2 and s["sm_mhz"] == 1932.5 and s["sm_max_mhz"] == 1965.0
+    assert s["reasons"] == ["sw_power_cap"]
+    assert b.ClockSampler(None).summary()["samples"] == 0
