@@ -239,9 +239,11 @@ sq_status sq_w8a8_linear_scatter(const int8_t *xq, const float *x_scale,
  * both the smoothed activations and the smoothed weights' K-vectors keeps
  * the product while spreading outliers over a block.
  *   rot_cs   [L][n / 2][2] fp32 (cos, sin) pairs, device memory.
- *   n        2 <= n <= 256 (16-bit rows) or 128 (fp32 rows), a power of two
- *            dividing K; K <= 16384 (16-bit) or 8192 (fp32); else
- *            SQ_ERR_UNSUPPORTED / SQ_ERR_INVALID_ARG.
+ *   n        a power of two, 2 <= n, dividing K (n = K rotates the whole
+ *            row); K <= 16384 (16-bit rows) or 8192 (fp32 rows), else
+ *            SQ_ERR_UNSUPPORTED; other n give SQ_ERR_INVALID_ARG.  Blocks
+ *            of up to 256 channels (128 for fp32) rotate in registers;
+ *            wider blocks through a row staged in shared memory (slower).
  * sq_quant_act_rotated: xq, x_scale of R(x * inv_smooth), as sq_quant_act.
  * sq_smooth_quant_weight_rotated: s and 1/s as sq_smooth_quant_weight
  *   (layout SQ_W_NK only), then wq, w_scale of R(s * w_n) per output

@@ -100,8 +100,8 @@ def test_rotation_argument_checks():
     assert f(A16, sq.SQ_BF16, 8, 256, 256, A16, 24, A16, A16, A16, None) == INV                  # n not 2^k
     assert f(A16, sq.SQ_BF16, 8, 256, 256, A16, 1, A16, A16, A16, None) == INV                   # n < 2
     assert f(A16, sq.SQ_BF16, 8, 272, 272, A16, 32, A16, A16, A16, None) == INV                  # K % n
-    assert f(A16, sq.SQ_BF16, 8, 1024, 1024, A16, 512, A16, A16, A16, None) == sq.SQ_ERR_UNSUPPORTED
-    assert f(A16, sq.SQ_F32, 8, 1024, 1024, A16, 256, A16, A16, A16, None) == sq.SQ_ERR_UNSUPPORTED
+    assert f(A16, sq.SQ_BF16, 8, 16400, 16400, A16, 16, A16, A16, A16, None) == sq.SQ_ERR_UNSUPPORTED   # K
+    assert f(A16, sq.SQ_F32, 8, 8208, 8208, A16, 16, A16, A16, A16, None) == sq.SQ_ERR_UNSUPPORTED
     assert f(A16, sq.SQ_BF16, 8, 256, 256, A16, 16, None, A16, A16, None) == INV                 # null table
     g = sq.lib().sq_smooth_quant_weight_rotated
     a = ctypes.c_float(0.5)

@@ -33,7 +33,10 @@ def _table(n, seed, kind="random"):
 
 @pytest.mark.parametrize("dt,K,n", [("bf16", 16, 2), ("bf16", 256, 4), ("bf16", 4096, 256), ("f16", 1040, 16),
                                     ("bf16", 11008, 128), ("f32", 4096, 128), ("f32", 272, 8),
-                                    ("bf16", 16384, 64), ("f16", 2048, 32)])
+                                    ("bf16", 16384, 64), ("f16", 2048, 32),
+                                    # blocks wider than a warp: the shared-memory kernel
+                                    ("bf16", 4096, 4096), ("bf16", 12288, 1024), ("f16", 16384, 16384),
+                                    ("f32", 8192, 8192), ("f32", 768, 256), ("bf16", 1536, 512)])
 @pytest.mark.parametrize("M", [1, 37])
 def test_quant_act_rotated(dt, K, n, M):
     o = synth.outliers(K, frac=0.01, mult=80.0, seed=K)
@@ -68,7 +71,8 @@ def test_special_angles(kind):
         assert float(xs.mean()) < float(xs0.mean())
 
 
-@pytest.mark.parametrize("dt,K,N,n", [("bf16", 1024, 528, 256), ("f32", 272, 64, 16), ("f16", 4096, 256, 128)])
+@pytest.mark.parametrize("dt,K,N,n", [("bf16", 1024, 528, 256), ("f32", 272, 64, 16), ("f16", 4096, 256, 128),
+                                      ("bf16", 4096, 64, 4096)])
 def test_smooth_quant_weight_rotated(dt, K, N, n):
     w = synth.weights(K, N, K + N, TORCH_DT[dt], "nk")
     o = synth.outliers(K, count=max(1, K // 50), seed=K)

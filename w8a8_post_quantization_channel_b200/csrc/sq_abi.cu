@@ -169,7 +169,7 @@ static int log2_exact(int64_t n) {
 static sq_status rot_checks(sq_dtype xt, int64_t K, int64_t n, const float *rot_cs, int *logn) {
   *logn = log2_exact(n);
   if (*logn < 1 || K % n != 0 || !valid_vec(rot_cs)) return SQ_ERR_INVALID_ARG;
-  if (n > (xt == SQ_F32 ? 128 : 256) || K > (xt == SQ_F32 ? 8192 : 16384)) return SQ_ERR_UNSUPPORTED;
+  if (K > (xt == SQ_F32 ? 8192 : 16384)) return SQ_ERR_UNSUPPORTED;
   return SQ_OK;
 }
 

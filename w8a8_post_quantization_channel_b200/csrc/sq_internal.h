@@ -57,8 +57,9 @@ cudaError_t launch_quant_static(const void *x, sq_dtype xt, int64_t rows, int64_
 
 // Rows of x * col_scale rotated per block of n = 2^logn channels by the
 // butterfly with (cos, sin) pairs cs [logn][n / 2][2], then per-row INT8
-// (n <= 32 channels per 16-byte vector x 32: 256 at 16 bits, 128 at 32;
-// K <= 16384 at 16 bits, 8192 at 32; cudaErrorNotSupported beyond).
+// (K <= 16384 at 16 bits, 8192 at 32; cudaErrorNotSupported beyond).  Blocks
+// of up to one warp's channels (256 at 16 bits, 128 at 32) rotate in
+// registers; wider blocks through a row staged in shared memory.
 cudaError_t launch_rot_quant_rows(const void *x, sq_dtype xt, int64_t rows, int64_t cols, int64_t ld,
                                   const float *col_scale, int logn, const float *cs, int8_t *q, float *row_scale_out,
                                   cudaStream_t st);

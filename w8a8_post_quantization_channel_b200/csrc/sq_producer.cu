@@ -324,7 +324,8 @@ cudaError_t launch_quant_static(const void *x, sq_dtype xt, int64_t rows, int64_
 namespace sq {
 namespace {
 
-constexpr int kRotMaxStages = 8;  // n <= 256
+constexpr int kRotMaxStages = 8;  // n <= 256 in the warp-local kernel
+constexpr int kRotSmemThreads = 512;
 
 template <typename T, int kVPT>
 __global__ void __launch_bounds__(kRowMaxThreads)
@@ -477,12 +478,104 @@ __global__ void __launch_bounds__(kRowMaxThreads)
   }
 }
 
+// Blocks wider than a warp's 32 V channels: R rows (R <= 4) are staged in
+// shared memory as fp32 and every stage walks the pairs by index -- pair q
+// of a row is pair j = q mod (n/2) of block q / (n/2), whose first element
+// sits at ((j >> i) << (i + 1)) | (j mod 2^i) -- with (c, s) = cs[i][j] read
+// through L1/L2 once for all R rows; a barrier separates the stages.
+// Persistent over groups of R rows; the codes follow as in the other row
+// quantizers.
+template <typename T>
+__global__ void __launch_bounds__(kRotSmemThreads)
+    rot_quant_rows_smem_kernel(const T *__restrict__ x, int64_t rows, int64_t nvec, int64_t ld,
+                               const float *__restrict__ col_scale, int logn, const float2 *__restrict__ cs, int R,
+                               int8_t *__restrict__ q, float *__restrict__ row_scale_out) {
+  extern __shared__ float rowbuf[];  // [R][K]
+  __shared__ float red[32];
+  constexpr int V = Vec<T>::N;
+  pdl_wait();  // the previous kernel's results are visible from here on
+  pdl_trigger();
+  const int K = (int)(nvec * V);  // <= 16384
+  const int half = 1 << (logn - 1);
+  const int pairs = K / 2;
+  const int64_t groups = (rows + R - 1) / R;
+  for (int64_t g = blockIdx.x; g < groups; g += gridDim.x) {
+    const int64_t r0 = g * R;
+    const int nr = (int)min((int64_t)R, rows - r0);
+    for (int u = 0; u < nr; ++u) {
+      const T *xr = x + (r0 + u) * ld;
+      float *buf = rowbuf + u * K;
+      for (int v = threadIdx.x; v < (int)nvec; v += blockDim.x) {
+        float f[V];
+        Vec<T>::to_f32(ld_nc_v4(xr + (int64_t)v * V), f);
+#pragma unroll
+        for (int e = 0; e < V; ++e) buf[v * V + e] = __fmul_rn(f[e], __ldg(col_scale + v * V + e));
+      }
+    }
+    __syncthreads();
+    for (int st = 0; st < logn; ++st) {
+      const int h = 1 << st;
+      const float2 *ts = cs + (int64_t)st * half;
+      for (int pq = threadIdx.x; pq < pairs; pq += blockDim.x) {
+        const int j = pq & (half - 1);  // pair within its block; the block starts at (pq - j) * 2
+        const int pa = ((pq - j) << 1) + (((j >> st) << (st + 1)) | (j & (h - 1)));
+        const float2 t = __ldg(ts + j);
+        for (int u = 0; u < nr; ++u) {
+          float *buf = rowbuf + u * K;
+          const float a = buf[pa], b = buf[pa + h];
+          buf[pa] = __fsub_rn(__fmul_rn(t.x, a), __fmul_rn(t.y, b));
+          buf[pa + h] = __fadd_rn(__fmul_rn(t.y, a), __fmul_rn(t.x, b));
+        }
+      }
+      __syncthreads();
+    }
+    for (int u = 0; u < nr; ++u) {
+      const float *buf = rowbuf + u * K;
+      float m = 0.0f;
+      for (int k = threadIdx.x; k < K; k += blockDim.x) m = fmaxf(m, fabsf(buf[k]));
+      m = block_max(m, red);
+      const float delta = __fdiv_rn(m, 127.0f);
+      const float rcp = m > 0.0f ? __frcp_rn(delta) : 0.0f;
+      if (threadIdx.x == 0) row_scale_out[r0 + u] = delta;
+      int8_t *qrow = q + (r0 + u) * K;
+      for (int v = threadIdx.x; v < (int)nvec; v += blockDim.x) {
+        float val[V];
+#pragma unroll
+        for (int e = 0; e < V; ++e) val[e] = buf[v * V + e];
+        if constexpr (V == 8) {
+          *reinterpret_cast<uint2 *>(qrow + v * V) = codes8(val, delta, rcp);
+        } else {
+          *reinterpret_cast<uint32_t *>(qrow + v * V) = codes4(val, delta, rcp);
+        }
+      }
+    }
+    __syncthreads();  // the buffers are reused by the next group
+  }
+}
+
 template <typename T>
 cudaError_t rot_quant_t(const void *x, int64_t rows, int64_t cols, int64_t ld, const float *col_scale, int logn,
                         const float *cs, int8_t *q, float *row_scale_out, cudaStream_t st) {
   constexpr int V = Vec<T>::N;
   const int64_t nvec = cols / V;
-  if (nvec > 4 * kRowMaxThreads || (1 << logn) > 32 * V) return cudaErrorNotSupported;
+  if (nvec > 4 * kRowMaxThreads) return cudaErrorNotSupported;
+  if ((1 << logn) > 32 * V) {  // blocks wider than a warp: the shared-memory kernel
+    const size_t row_bytes = (size_t)cols * sizeof(float);
+    const int R = (int)std::max<size_t>(1, std::min<size_t>(4, (200 * 1024) / row_bytes));
+    const size_t smem = R * row_bytes;
+    if (smem > 200 * 1024) return cudaErrorNotSupported;
+    auto kern = rot_quant_rows_smem_kernel<T>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    int per_sm = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kRotSmemThreads, smem);
+    if (e != cudaSuccess) return e;
+    const int64_t grid = std::min<int64_t>(rows, (int64_t)std::max(1, per_sm) * num_sms());
+    const int64_t groups = (rows + R - 1) / R;
+    return launch_pdl(kern, dim3((unsigned)std::min<int64_t>(grid, groups)), dim3(kRotSmemThreads), smem, st, 1,
+                      (const T *)x, rows, nvec, ld, col_scale, logn, reinterpret_cast<const float2 *>(cs), R, q,
+                      row_scale_out);
+  }
   const int vpt = nvec <= 4 * 32 ? 1 : 4;
   const int64_t t = (nvec + vpt - 1) / vpt;
   const int threads = (int)std::max<int64_t>(32, ((t + 31) / 32) * 32);
