@@ -261,7 +261,8 @@ def test_linear_epilogue_cta_pairs(dt):
 # Decode-shaped products (M <= 64 tokens): the weight-streaming kernel,
 # whose CTAs combine partial tiles through the caller's workspace.
 DECODE_SHAPES = [(1, 4096, 4096), (2, 272, 1040), (16, 1024, 8192), (17, 4096, 272), (33, 528, 4096),
-                 (48, 16, 16), (64, 12288, 1040), (64, 1040, 11008), (8, 28672, 8192), (1, 8192, 8192)]
+                 (48, 16, 16), (64, 12288, 1040), (64, 1040, 11008), (8, 28672, 8192), (1, 8192, 8192),
+                 (8, 11008, 4096)]  # 86 tiles of 128 rows: one CTA per tile, no K split
 
 
 @pytest.mark.parametrize("M,N,K", DECODE_SHAPES)
