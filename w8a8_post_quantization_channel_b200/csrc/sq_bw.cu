@@ -21,7 +21,7 @@ namespace {
 
 constexpr int kColThreadsX = 32;  // 16-byte column vectors per CTA slab
 constexpr int kColThreadsY = 8;   // row lanes per CTA
-constexpr int kColUnroll = 4;     // independent row loads in flight per thread
+constexpr int kColUnroll = 8;     // independent row loads in flight per thread
 
 // amax[c] = max(amax[c], max_r |v_rc|), v_rc = x[r][c] (* row_scale[r]).
 // CTA (32 x 8): threadIdx.x picks a 16-byte column vector of a 32-vector
@@ -52,12 +52,15 @@ __global__ void __launch_bounds__(kColThreadsX *kColThreadsY)
 #pragma unroll
       for (int u = 0; u < kColUnroll; ++u) raw[u] = ld_policy_v4(col + (r + u * kColThreadsY) * ld, policy);
 #pragma unroll
-      for (int u = 0; u < kColUnroll; ++u) {
-        float f[V];
-        Vec<T>::to_f32(raw[u], f);
-        const float sc = kScaled ? __ldg(row_scale + r + u * kColThreadsY) : 1.0f;
+      for (int u = 0; u < kColUnroll; u += 2) {
+        float f0[V], f1[V];
+        Vec<T>::to_f32(raw[u], f0);
+        Vec<T>::to_f32(raw[u + 1], f1);
+        const float s0 = kScaled ? __ldg(row_scale + r + u * kColThreadsY) : 1.0f;
+        const float s1 = kScaled ? __ldg(row_scale + r + (u + 1) * kColThreadsY) : 1.0f;
 #pragma unroll
-        for (int e = 0; e < V; ++e) m[e] = fmaxf(m[e], fabsf(kScaled ? __fmul_rn(sc, f[e]) : f[e]));
+        for (int e = 0; e < V; ++e)
+          m[e] = fmax3(m[e], fabsf(kScaled ? __fmul_rn(s0, f0[e]) : f0[e]), fabsf(kScaled ? __fmul_rn(s1, f1[e]) : f1[e]));
       }
     }
     for (; r < r1; r += kColThreadsY) {
