@@ -73,6 +73,8 @@ def _load():
             "or_fold_norm_weight": ([f32p, f32p, i64, f32p], None),
             "or_rmsnorm_quant_act": ([f32p, i64, i64, f32p, ctypes.c_float, i8p, f32p], None),
             "or_rmsnorm_factor": ([f32p, i64, i64, ctypes.c_float, f32p], None),
+            "or_layernorm_quant_act": ([f32p, i64, i64, f32p, f32p, ctypes.c_float, i8p, f32p], None),
+            "or_layernorm_stats": ([f32p, i64, i64, ctypes.c_float, f32p, f32p], None),
             "or_static_act_scale": ([f32p, f32p, i64], ctypes.c_float),
             "or_quant_act_static": ([f32p, i64, i64, f32p, ctypes.c_float, i8p, f32p], None),
             "or_e4m3_decode": ([ctypes.c_uint8], ctypes.c_float),
@@ -255,6 +257,33 @@ def rmsnorm_factor(x, eps: float) -> np.ndarray:
     r = np.zeros(M, np.float32)
     _load().or_rmsnorm_factor(_ptr(x, ctypes.c_float), M, K, ctypes.c_float(eps), _ptr(r, ctypes.c_float))
     return r
+
+
+def layernorm_quant_act(x, gs, bs, eps: float):
+    """(Xq, dx): LayerNorm (epsilon eps) with the folded weight gs and bias
+    bs (None: no bias), then per-token quantization."""
+    x = _f32(x)
+    gs = _f32(gs)
+    M, K = x.shape
+    xq = np.zeros((M, K), np.int8)
+    dx = np.zeros(M, np.float32)
+    bp = None if bs is None else _f32(bs)
+    _load().or_layernorm_quant_act(_ptr(x, ctypes.c_float), M, K, _ptr(gs, ctypes.c_float),
+                                   None if bp is None else _ptr(bp, ctypes.c_float), ctypes.c_float(eps),
+                                   _ptr(xq, ctypes.c_int8), _ptr(dx, ctypes.c_float))
+    return xq, dx
+
+
+def layernorm_stats(x, eps: float):
+    """Per-token (mu_t, r_t): the mean rounded once to fp32, and
+    1 / sqrt(var_t + eps) rounded once to fp32."""
+    x = _f32(x)
+    M, K = x.shape
+    mu = np.zeros(M, np.float32)
+    r = np.zeros(M, np.float32)
+    _load().or_layernorm_stats(_ptr(x, ctypes.c_float), M, K, ctypes.c_float(eps), _ptr(mu, ctypes.c_float),
+                               _ptr(r, ctypes.c_float))
+    return mu, r
 
 
 def static_act_scale(amax, inv_s) -> float:

@@ -274,6 +274,65 @@ void or_rmsnorm_factor(const float *x, int64_t M, int64_t K, float eps, float *r
   }
 }
 
+/* ---- upstream producer: LayerNorm, smoothing and per-token quantization --
+ * The same fold for a layer normalisation with weight gamma and bias beta
+ * (the OPT models of the page's benchmarks use this form):
+ *   gs_j = gamma_j * inv_s_j,  bs_j = beta_j * inv_s_j   (fp32, once per layer)
+ * and for token t
+ *   mu_t  = sum_j x_tj / K                     (double, sequential)
+ *   var_t = sum_j (x_tj - mu_t)^2 / K          (double: each deviation and
+ *                                               its square in double)
+ *   r_t   = (float)(1 / sqrt(var_t + eps))     (double, rounded once)
+ *   muf_t = (float)mu_t
+ *   v_tj  = ((x_tj - muf_t) * r_t) * gs_j + bs_j   (fp32, in that order)
+ * then per-token quantization of v as in or_quant_act.  bs may be NULL (no
+ * bias). */
+static void or_layernorm_row_stats(const float *row, int64_t K, float eps, float *muf, float *r) {
+  double sum = 0.0;
+  for (int64_t j = 0; j < K; ++j) sum += (double)row[j];
+  const double mu = sum / (double)K;
+  double ss = 0.0;
+  for (int64_t j = 0; j < K; ++j) {
+    const double d = (double)row[j] - mu;
+    ss += d * d;
+  }
+  *r = (float)(1.0 / sqrt(ss / (double)K + (double)eps));
+  *muf = (float)mu;
+}
+
+void or_layernorm_stats(const float *x, int64_t M, int64_t K, float eps, float *mu, float *r) {
+  for (int64_t t = 0; t < M; ++t) or_layernorm_row_stats(x + t * K, K, eps, &mu[t], &r[t]);
+}
+
+static float or_layernorm_value(float x, float muf, float r, float g, float b) {
+  const float c = x - muf;
+  const float n = c * r;
+  const float w = n * g;
+  return w + b;
+}
+
+void or_layernorm_quant_act(const float *x, int64_t M, int64_t K, const float *gs, const float *bs, float eps,
+                            int8_t *xq, float *dx) {
+  for (int64_t t = 0; t < M; ++t) {
+    const float *row = x + t * K;
+    float muf, r;
+    or_layernorm_row_stats(row, K, eps, &muf, &r);
+    float m = 0.0f;
+    for (int64_t j = 0; j < K; ++j) {
+      float v = fabsf(or_layernorm_value(row[j], muf, r, gs[j], bs ? bs[j] : 0.0f));
+      if (v > m) m = v;
+    }
+    if (m == 0.0f) {
+      dx[t] = 0.0f;
+      for (int64_t j = 0; j < K; ++j) xq[t * K + j] = 0;
+      continue;
+    }
+    dx[t] = m / 127.0f;
+    for (int64_t j = 0; j < K; ++j)
+      xq[t * K + j] = or_quantize_value(or_layernorm_value(row[j], muf, r, gs[j], bs ? bs[j] : 0.0f), dx[t]);
+  }
+}
+
 /* ---- static per-tensor activation scale --------------------------------
  * The page notes activations change per prompt, which is why the main path
  * quantizes per token at run time; the static alternative fixes one scale

@@ -446,3 +446,112 @@ def test_p7_static_scale_and_saturation():
     xq, dx = oracle.quant_act_static(x, np.ones(x.shape[1], np.float32), float(g["delta"][0]))
     np.testing.assert_array_equal(xq[0], _int(g["xq"]))
     assert dx[0] == np.float32(float(g["delta"][0]))
+
+
+# ---------------------------------------------------------------------------
+# upstream producer: LayerNorm (weight and bias) folded with X diag(s)^-1
+# ---------------------------------------------------------------------------
+
+def test_p10_layernorm_worked_example():
+    g = load("p10_layernorm.txt")
+    x = _fl(g["x"]).astype(np.float32)[None, :]
+    eps = float(g["eps"][0])
+    mu, r = oracle.layernorm_stats(x, eps)
+    assert mu[0] == float(g["mu"][0]) and r[0] == float(g["r"][0])
+    ones = np.ones(4, np.float32)
+    for case, gs, bs in (("a", _fl(g["gs_a"]), None), ("b", _fl(g["gs_b"]), None),
+                         ("c", ones, _fl(g["bs_c"]))):
+        xq, dx = oracle.layernorm_quant_act(x, gs, bs, eps)
+        np.testing.assert_array_equal(xq[0], _int(g["xq_" + case]))
+        assert dx[0] == np.float32(np.float32(float(g["dx_%s_num" % case][0])) / np.float32(127))
+
+
+def test_layernorm_stats_match_library_layer_norm():
+    rng = np.random.default_rng(31)
+    x = (rng.standard_normal((9, 320)) + rng.uniform(-3, 3, (9, 1))).astype(np.float32)
+    x[:, 5] *= 80
+    eps = 1e-5
+    mu, r = oracle.layernorm_stats(x, eps)
+    xt = torch.from_numpy(x.astype(np.float64))
+    normed = torch.nn.functional.layer_norm(xt, (320,), eps=eps).numpy()  # (x - mean) / sqrt(var + eps)
+    mean = xt.mean(dim=1).numpy()
+    assert _ulps(mu, mean).max() <= 0.5
+    j = np.argmax(np.abs(x - mean[:, None]), axis=1)  # the largest deviation in each row
+    rows = np.arange(9)
+    r_lib = normed[rows, j] / (x[rows, j].astype(np.float64) - mean)
+    assert _ulps(r, r_lib).max() <= 1
+
+
+def test_layernorm_on_zero_mean_rows_equals_rmsnorm():
+    # rows made of +-pairs have mean exactly 0, so the variance is the mean
+    # square: LayerNorm without bias must give the RMSNorm producer's codes
+    # and scales bit for bit.  A 1/(K-1) variance or a mean taken of |x|
+    # fails here.
+    rng = np.random.default_rng(32)
+    half = (rng.standard_normal((6, 48)) * 3).astype(np.float32)
+    x = np.concatenate([half, -half], axis=1)[:, rng.permutation(96)]
+    gs = oracle.fold_norm_weight(rng.uniform(0.3, 2, 96), rng.uniform(0.1, 3, 96))
+    eps = 1e-5
+    mu, _ = oracle.layernorm_stats(x, eps)
+    np.testing.assert_array_equal(mu, 0.0)
+    a = oracle.layernorm_quant_act(x, gs, None, eps)
+    b = oracle.rmsnorm_quant_act(x, gs, eps)
+    np.testing.assert_array_equal(a[0], b[0])
+    np.testing.assert_array_equal(a[1], b[1])
+
+
+def test_layernorm_shift_and_scale_invariance():
+    # values on a 1/8 grid, K = 16: the mean is exact, and so is every
+    # deviation, with or without a shift of the whole token by a constant,
+    # so the codes cannot change.  A power-of-two rescale with negligible
+    # eps is absorbed exactly by r.  A producer that skips the mean (RMS of
+    # the raw values) fails the shift.
+    rng = np.random.default_rng(33)
+    x = (rng.integers(-40, 41, (7, 16)) / 8.0).astype(np.float32)
+    gs = oracle.fold_norm_weight(rng.uniform(0.5, 2, 16), rng.uniform(0.2, 3, 16))
+    bs = rng.uniform(-0.5, 0.5, 16).astype(np.float32)
+    eps = 1e-30
+    base = oracle.layernorm_quant_act(x, gs, bs, eps)
+    shifted = oracle.layernorm_quant_act(x + np.float32(37.0), gs, bs, eps)
+    scaled = oracle.layernorm_quant_act(x * np.float32(16.0), gs, bs, eps)
+    for other in (shifted, scaled):
+        np.testing.assert_array_equal(base[0], other[0])
+        np.testing.assert_array_equal(base[1], other[1])
+    assert not np.array_equal(base[0], oracle.rmsnorm_quant_act(x + np.float32(37.0), gs, eps)[0])
+
+
+def test_layernorm_bias_alone():
+    # with gs = 0 every token normalises to v = bs, whatever x is: the codes
+    # are plain quantization of the bias row (its sign and per-column place
+    # fixed by quant_act's own pins)
+    rng = np.random.default_rng(34)
+    x = rng.standard_normal((4, 32)).astype(np.float32)
+    bs = rng.uniform(-2, 2, 32).astype(np.float32)
+    xq, dx = oracle.layernorm_quant_act(x, np.zeros(32, np.float32), bs, 1e-5)
+    bq, bd = oracle.quant_act(bs[None, :], np.ones(32, np.float32))
+    np.testing.assert_array_equal(xq, np.repeat(bq, 4, axis=0))
+    np.testing.assert_array_equal(dx, np.repeat(bd, 4))
+
+
+def test_folded_layernorm_equals_norm_then_smoothing():
+    # with inv_s a power of two per channel, folding it into the weight and
+    # the bias changes no rounding: (n gamma + beta) inv_s == n (gamma inv_s)
+    # + beta inv_s exactly.  So the folded producer must equal the unfolded
+    # sequence: normalise, apply gamma and beta, then X diag(s)^-1 and
+    # per-token quantization.
+    rng = np.random.default_rng(35)
+    K = 64
+    x = (rng.standard_normal((7, K)) + 2.0).astype(np.float32)
+    x[:, 3] *= 40
+    gamma = rng.uniform(0.2, 3.0, K).astype(np.float32)
+    beta = rng.uniform(-1.0, 1.0, K).astype(np.float32)
+    inv_s = np.float32(2.0) ** rng.integers(-6, 7, K).astype(np.float32)
+    eps = 1e-5
+    xq, dx = oracle.layernorm_quant_act(x, oracle.fold_norm_weight(gamma, inv_s),
+                                        oracle.fold_norm_weight(beta, inv_s), eps)
+    mu, r = oracle.layernorm_stats(x, eps)
+    n = ((x - mu[:, None]).astype(np.float32) * r[:, None]).astype(np.float32)
+    normed = ((n * gamma).astype(np.float32) + beta).astype(np.float32)
+    xq_u, dx_u = oracle.quant_act(normed, inv_s)
+    np.testing.assert_array_equal(xq, xq_u)
+    np.testing.assert_array_equal(dx, dx_u)
