@@ -149,6 +149,30 @@ sq_status sq_rmsnorm_quant_act(const void *x, sq_dtype xt, int64_t M, int64_t K,
                                int8_t *xq, float *x_scale, sq_stream_t stream);
 
 /*
+ * Upstream producer for models whose linears are fed by a LayerNorm with a
+ * bias (the OPT models of the page's speed-up and perplexity tables): fold
+ * diag(s)^-1 into both, gs = gamma * inv_smooth and bs = beta * inv_smooth
+ * (sq_fold_smooth_into_norm computes either product), then per token
+ *   mu_t  = sum_j x_tj / K
+ *   var_t = sum_j (x_tj - mu_t)^2 / K
+ *          (both in double precision: each value, deviation and square in
+ *          double, the sums in an unspecified order; mu_t and
+ *          r_t = 1 / sqrt(var_t + eps) each rounded once to fp32)
+ *   v_tj  = ((x_tj - mu_t) * r_t) * gs_j + bs_j   (fp32, in that order)
+ *   then per-token quantization of v exactly as sq_quant_act.
+ *   gs [K] fp32; bs [K] fp32 or NULL (no bias); eps > 0 and finite (a
+ *   constant token has var_t = 0).  Other arguments as sq_quant_act.
+ * As for sq_rmsnorm_quant_act, mu_t and r_t may differ from another
+ * implementation's by one fp32 ulp, which moves a code by one only next to
+ * a rounding boundary.  K <= 16384 for 16-bit x, <= 8192 for fp32 x, else
+ * SQ_ERR_UNSUPPORTED.
+ */
+sq_status sq_layernorm_quant_act(const void *x, sq_dtype xt, int64_t M, int64_t K,
+                                 int64_t ldx, const float *gs, const float *bs,
+                                 float eps, int8_t *xq, float *x_scale,
+                                 sq_stream_t stream);
+
+/*
  * Static per-tensor activation scale, the alternative to per-token scales
  * (the page notes activations change per prompt, which is why the main path
  * measures each token at run time).  After smoothing, channel j's

@@ -126,6 +126,16 @@ def test_producer_argument_checks():
     assert f(A16, sq.SQ_BF16, 8, 24, 24, A16, eps, A16, A16, None) == INV               # K % 16
     assert f(A16, sq.SQ_BF16, 8, 16400, 16400, A16, eps, A16, A16, None) == sq.SQ_ERR_UNSUPPORTED
     assert f(A16, sq.SQ_F32, 8, 8208, 8208, A16, eps, A16, A16, None) == sq.SQ_ERR_UNSUPPORTED
+    ln = L.sq_layernorm_quant_act
+    assert ln(None, sq.SQ_BF16, 0, 256, 256, A16, None, eps, None, None, None) == sq.SQ_OK   # M == 0: no-op
+    assert ln(A16, sq.SQ_BF16, 8, 256, 256, None, A16, eps, A16, A16, None) == INV          # null gs
+    assert ln(A16, sq.SQ_BF16, 8, 256, 256, A16, MIS, eps, A16, A16, None) == INV           # misaligned bs
+    assert ln(A16, sq.SQ_BF16, 8, 256, 256, A16, A16, ctypes.c_float(0.0), A16, A16, None) == INV  # eps = 0
+    assert ln(A16, sq.SQ_BF16, 8, 256, 256, A16, A16, ctypes.c_float(float("nan")), A16, A16, None) == INV
+    assert ln(A16, sq.SQ_BF16, 8, 24, 24, A16, A16, eps, A16, A16, None) == INV             # K % 16
+    assert ln(A16, sq.SQ_BF16, 8, 256, 200, A16, A16, eps, A16, A16, None) == INV           # ldx < K
+    assert ln(A16, sq.SQ_BF16, 8, 16400, 16400, A16, None, eps, A16, A16, None) == sq.SQ_ERR_UNSUPPORTED
+    assert ln(A16, sq.SQ_F32, 8, 8208, 8208, A16, None, eps, A16, A16, None) == sq.SQ_ERR_UNSUPPORTED
     st = L.sq_static_act_scale
     assert st(A16, A16, 256, MIS + 1, None) == INV                                       # delta not 4-B aligned
     assert st(None, A16, 256, A16, None) == INV

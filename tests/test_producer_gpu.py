@@ -9,6 +9,10 @@ everywhere except where the oracle's own pre-rounding value lies within
 1e-4 of a rounding boundary, and there by at most one.  Scales agree within
 two fp32 ulps.
 
+sq_layernorm_quant_act: LayerNorm with the folded weight gs and bias bs +
+per-token INT8; the mean and the variance are double-precision sums in an
+order neither side fixes, with the same tolerance as above.
+
 sq_static_act_scale / sq_quant_act_static: bit-exact, including values
 beyond the calibrated range, which saturate at +-127.
 """
@@ -96,6 +100,79 @@ def test_rmsnorm_quant_feeds_the_linear():
     # the linear is exact given the GPU's own codes and scales
     y_ref = oracle.dequant(oracle.gemm_i8(xq.cpu().numpy(), wq), xs.cpu().numpy(), dw)
     np.testing.assert_array_equal(y.cpu().numpy(), y_ref)
+
+
+def _ln_boundary_mask(x, gs, bs, eps):
+    """As _boundary_mask, for the LayerNorm value ((x - mu) r) gs + bs."""
+    mu, r = oracle.layernorm_stats(x, eps)
+    v = (x - mu[:, None]).astype(np.float32)
+    v = (v * r[:, None]).astype(np.float32)
+    v = (v * gs).astype(np.float32)
+    if bs is not None:
+        v = (v + bs).astype(np.float32)
+    m = np.abs(v).max(axis=1)
+    delta = (m / np.float32(127.0)).astype(np.float32)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        u = np.abs(np.where(delta[:, None] > 0, v / delta[:, None], 0).astype(np.float32)).astype(np.float64)
+    return np.abs(u - np.floor(u) - 0.5) < 1e-4
+
+
+@pytest.mark.parametrize("dt,K", [("bf16", 16), ("bf16", 256), ("f16", 1040), ("bf16", 4096), ("f32", 4096),
+                                  ("f16", 11008), ("bf16", 16384), ("f32", 8192)])
+@pytest.mark.parametrize("M", [1, 7, 300])
+@pytest.mark.parametrize("bias", [True, False])
+def test_layernorm_quant_act(dt, K, M, bias):
+    o = synth.outliers(K, frac=0.01, mult=50.0, seed=K)
+    x = synth.activations(M, K, o, seed=K + M + 11, dtype=TORCH_DT[dt])
+    x += 0.75  # a nonzero mean for the normalisation to remove
+    if M > 3:
+        x[3] = 2.5  # a constant token: variance 0, every value -> the bias
+    g = synth.gen(K + 9)
+    gamma = torch.rand(K, generator=g) * 2.0 + 0.05
+    beta = torch.rand(K, generator=g) - 0.5
+    inv_s = torch.exp(torch.randn(K, generator=g))
+    gs = oracle.fold_norm_weight(gamma.numpy(), inv_s.numpy())
+    bs = oracle.fold_norm_weight(beta.numpy(), inv_s.numpy()) if bias else None
+    eps = 1e-5
+    xq, xs = sq.sq_layernorm_quant_act(x.to(DEV), torch.from_numpy(gs).to(DEV),
+                                       None if bs is None else torch.from_numpy(bs).to(DEV), eps)
+    xf = f32(x)
+    xq_ref, xs_ref = oracle.layernorm_quant_act(xf, gs, bs, eps)
+    xs_g = xs.cpu().numpy()
+    ulp = np.spacing(np.abs(xs_ref).astype(np.float32)).astype(np.float64)
+    assert np.all(np.abs(xs_g.astype(np.float64) - xs_ref) <= 2 * ulp)
+    diff = xq.cpu().numpy().astype(np.int32) - xq_ref.astype(np.int32)
+    near = _ln_boundary_mask(xf, gs, bs, eps)
+    assert np.abs(diff).max() <= 1
+    assert np.all(diff[~near] == 0), f"{int((diff[~near] != 0).sum())} codes differ away from rounding boundaries"
+    if M > 3 and not bias:
+        assert xs_g[3] == 0 and not xq.cpu().numpy()[3].any()
+    assert sq.sq_check_device_error() == sq.SQ_OK
+
+
+def test_layernorm_quant_feeds_the_linear():
+    # OPT-style block: LayerNorm with bias folded with 1/s, then the INT8
+    # linear; the linear is exact given the GPU's own codes and scales
+    M, K, N = 64, 4096, 512
+    o = synth.outliers(K, frac=0.01, mult=60.0, seed=13)
+    x = synth.activations(M, K, o, seed=14, dtype=torch.float16)
+    g = synth.gen(15)
+    gamma = torch.rand(K, generator=g) + 0.5
+    beta = torch.rand(K, generator=g) - 0.5
+    w = synth.weights(K, N, 16, torch.float16, "nk")
+    amax = oracle.calib_absmax(f32(x))
+    s, inv = oracle.smooth_factor(amax, oracle.weight_absmax(f32(w), oracle.LAYOUT_NK), 0.5)
+    wq, dw = oracle.smooth_quant_weight(f32(w), oracle.LAYOUT_NK, s)
+    inv_d = torch.from_numpy(inv).to(DEV)
+    gs = sq.sq_fold_smooth_into_norm(gamma.to(DEV), inv_d)
+    bs = sq.sq_fold_smooth_into_norm(beta.to(DEV), inv_d)
+    xq, xs = sq.sq_layernorm_quant_act(x.to(DEV), gs, bs, 1e-5)
+    y = sq.sq_w8a8_linear(xq, xs, torch.from_numpy(wq).to(DEV), torch.from_numpy(dw).to(DEV), torch.float32)
+    y_ref = oracle.dequant(oracle.gemm_i8(xq.cpu().numpy(), wq), xs.cpu().numpy(), dw)
+    np.testing.assert_array_equal(y.cpu().numpy(), y_ref)
+    # and the codes are the oracle's (up to the boundary tolerance)
+    xq_ref, _ = oracle.layernorm_quant_act(f32(x), gs.cpu().numpy(), bs.cpu().numpy(), 1e-5)
+    assert np.abs(xq.cpu().numpy().astype(np.int32) - xq_ref).max() <= 1
 
 
 @pytest.mark.parametrize("dt,K", [("bf16", 4096), ("f16", 1040), ("f32", 272)])

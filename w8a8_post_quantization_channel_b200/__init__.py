@@ -34,7 +34,8 @@ __all__ = [
     "sq_calib_absmax", "sq_smooth_quant_weight", "sq_quant_act", "sq_w8a8_linear",
     "sq_w8a8_linear_workspace_size", "sq_w8a8_accumulate", "sq_check_device_error", "sq_status_string",
     "sq_w8a8_linear_decode_noalloc", "SQ_DECODE_STATIC_SCRATCH_BYTES", "sq_selftest_wait_timeout",
-    "sq_fold_smooth_into_norm", "sq_rmsnorm_quant_act", "sq_static_act_scale", "sq_quant_act_static",
+    "sq_fold_smooth_into_norm", "sq_rmsnorm_quant_act", "sq_layernorm_quant_act", "sq_static_act_scale",
+    "sq_quant_act_static",
     "sq_smooth_quant_weight_e4m3", "sq_quant_act_e4m3", "sq_w8a8_linear_e4m3", "sq_w8a8_accumulate_e4m3",
     "sq_w8a8_linear_scatter", "sq_quant_act_rotated", "sq_smooth_quant_weight_rotated",
 ]
@@ -85,6 +86,7 @@ def lib() -> ctypes.CDLL:
             "sq_selftest_wait_timeout": [i32, vp],
             "sq_fold_smooth_into_norm": [vp, vp, i64, vp, vp],
             "sq_rmsnorm_quant_act": [vp, i32, i64, i64, i64, vp, f32, vp, vp, vp],
+            "sq_layernorm_quant_act": [vp, i32, i64, i64, i64, vp, vp, f32, vp, vp, vp],
             "sq_static_act_scale": [vp, vp, i64, vp, vp],
             "sq_quant_act_static": [vp, i32, i64, i64, i64, vp, vp, vp, vp, vp],
             "sq_smooth_quant_weight_e4m3": [vp, i32, i32, i64, i64, i64, vp, f32, vp, vp, vp, vp, vp],
@@ -228,6 +230,19 @@ def sq_rmsnorm_quant_act(x: torch.Tensor, gs: torch.Tensor, eps: float, xq=None,
     x_scale = torch.empty(M, dtype=torch.float32, device=x.device) if x_scale is None else x_scale
     _check(lib().sq_rmsnorm_quant_act(_ptr(x), _dtype(x, "x"), M, K, x.stride(0), _ptr(gs), ctypes.c_float(eps),
                                       _ptr(xq), _ptr(x_scale), _stream(stream)), "sq_rmsnorm_quant_act")
+    return xq, x_scale
+
+
+def sq_layernorm_quant_act(x: torch.Tensor, gs: torch.Tensor, bs, eps: float, xq=None, x_scale=None, stream=None):
+    """(xq, x_scale) = per-token INT8 of LayerNorm(x; eps) with the folded
+    weight gs and bias bs (None: no bias)."""
+    _rowmajor(x, "x")
+    M, K = x.shape
+    xq = torch.empty((M, K), dtype=torch.int8, device=x.device) if xq is None else xq
+    x_scale = torch.empty(M, dtype=torch.float32, device=x.device) if x_scale is None else x_scale
+    _check(lib().sq_layernorm_quant_act(_ptr(x), _dtype(x, "x"), M, K, x.stride(0), _ptr(gs),
+                                        None if bs is None else _ptr(bs), ctypes.c_float(eps), _ptr(xq),
+                                        _ptr(x_scale), _stream(stream)), "sq_layernorm_quant_act")
     return xq, x_scale
 
 

@@ -232,6 +232,18 @@ sq_status sq_rmsnorm_quant_act(const void *x, sq_dtype xt, int64_t M, int64_t K,
   return from_cuda(sq::launch_rmsnorm_quant(x, xt, M, K, ldx, gs, eps, xq, x_scale, (cudaStream_t)stream));
 }
 
+sq_status sq_layernorm_quant_act(const void *x, sq_dtype xt, int64_t M, int64_t K, int64_t ldx, const float *gs,
+                                 const float *bs, float eps, int8_t *xq, float *x_scale, sq_stream_t stream) {
+  if (!valid_dtype(xt) || K <= 0 || K % 16 != 0 || K >= kMaxDim || M < 0 || M >= kMaxDim) return SQ_ERR_INVALID_ARG;
+  if (ldx < K || (ldx * dsize(xt)) % 16 != 0) return SQ_ERR_INVALID_ARG;
+  if (!(eps > 0.0f) || eps > 3.0e38f) return SQ_ERR_INVALID_ARG;  // rejects NaN and infinity too
+  if (!valid_vec(gs) || (bs != nullptr && !valid_vec(bs))) return SQ_ERR_INVALID_ARG;
+  if (K > (xt == SQ_F32 ? 8192 : 16384)) return SQ_ERR_UNSUPPORTED;
+  if (M == 0) return SQ_OK;
+  if (!valid_matrix(x, xt, M, K, ldx) || !valid_vec(xq) || !valid_vec(x_scale)) return SQ_ERR_INVALID_ARG;
+  return from_cuda(sq::launch_layernorm_quant(x, xt, M, K, ldx, gs, bs, eps, xq, x_scale, (cudaStream_t)stream));
+}
+
 sq_status sq_static_act_scale(const float *amax, const float *inv_smooth, int64_t K, float *delta,
                               sq_stream_t stream) {
   if (K <= 0 || K >= kMaxDim || !valid_vec(amax) || !valid_vec(inv_smooth)) return SQ_ERR_INVALID_ARG;

@@ -48,6 +48,9 @@ cudaError_t launch_fold_norm_weight(const float *gamma, const float *inv_s, int6
 // 16 bits, 8192 at 32; cudaErrorNotSupported beyond).
 cudaError_t launch_rmsnorm_quant(const void *x, sq_dtype xt, int64_t rows, int64_t cols, int64_t ld,
                                  const float *gs, float eps, int8_t *q, float *row_scale_out, cudaStream_t st);
+cudaError_t launch_layernorm_quant(const void *x, sq_dtype xt, int64_t rows, int64_t cols, int64_t ld,
+                                   const float *gs, const float *bs, float eps, int8_t *q, float *row_scale_out,
+                                   cudaStream_t st);
 // *delta = max_j(amax_j * inv_s_j) / 127.
 cudaError_t launch_static_scale(const float *amax, const float *inv_s, int64_t K, float *delta, cudaStream_t st);
 // Static per-tensor quantization with the device scalar *delta.

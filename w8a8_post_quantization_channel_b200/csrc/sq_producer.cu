@@ -2,11 +2,14 @@
 // (sm_100a).  smooth_lm(alpha) in the usage example of "SmoothQuant
 // (activation smoothing quantization)" (jisaku.com glossary) moves
 // diag(s)^-1 out of the run-time path into the preceding layer; in
-// transformer blocks that layer is an RMS normalisation, whose weight takes
-// it.  Also the static per-tensor activation scale, the alternative to
+// transformer blocks that layer is a normalisation -- RMS (Llama) or a
+// LayerNorm with a bias (the OPT models of the page's tables) -- whose
+// weight and bias take it.  Also the static per-tensor activation scale, the alternative to
 // per-token scales that the same page contrasts with dynamic ones:
 //   fold        gs_j = gamma_j * inv_s_j
 //   producer    r_t = 1 / sqrt(sum_j x_tj^2 / K + eps), v = (x r) gs, INT8
+//   LayerNorm   mu_t = mean_j x_tj, r_t = 1 / sqrt(mean_j (x_tj - mu_t)^2 + eps),
+//               v = ((x - mu) r) gs + bs, INT8 (bs = beta * inv_s)
 //   static      delta = max_j(amax_j inv_s_j) / 127, q = sat(rne(x inv_s / delta))
 #include <algorithm>
 
@@ -35,21 +38,71 @@ __device__ __forceinline__ double sumsq_vec(uint4 raw) {
   return acc;
 }
 
-// RMS normalisation whose weight already carries diag(s)^-1 (gs = gamma *
-// inv_s, folded ahead of time), then per-token INT8.  Persistent like
-// quant_rows_kernel: the folded weight stays in registers across rows and
-// the next row is prefetched while the current one is reduced twice (sum of
-// squares in double, then the absmax of v = (x * r) * gs, recomputed for
-// the codes rather than held).
-template <typename T, int kVPT>
+// Sum of one 16-byte row vector in double (each value converted exactly).
+template <typename T>
+__device__ __forceinline__ double sum_vec(uint4 raw) {
+  constexpr int V = Vec<T>::N;
+  float f[V];
+  Vec<T>::to_f32(raw, f);
+  double acc = 0.0;
+#pragma unroll
+  for (int e = 0; e < V; ++e) acc = __dadd_rn(acc, (double)f[e]);
+  return acc;
+}
+
+// Sum of the squared deviations from mu of one row vector, in double.
+// Lanes past the row end hold x = 0 and must add nothing: `live` is false
+// there.
+template <typename T>
+__device__ __forceinline__ double devsq_vec(uint4 raw, double mu, bool live) {
+  constexpr int V = Vec<T>::N;
+  float f[V];
+  Vec<T>::to_f32(raw, f);
+  double acc = 0.0;
+#pragma unroll
+  for (int e = 0; e < V; ++e) {
+    const double d = __dsub_rn((double)f[e], mu);
+    acc = __fma_rn(d, d, acc);
+  }
+  return live ? acc : 0.0;
+}
+
+// Block-wide double sum of one per-thread partial through red[] (one slot
+// per warp); every thread gets the total.
+__device__ __forceinline__ double block_sum_d(double v, double *red, int lane, int warp, int nwarps) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = __dadd_rn(v, __shfl_xor_sync(0xffffffffu, v, o));
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  v = 0.0;
+  for (int w = 0; w < nwarps; ++w) v = __dadd_rn(v, red[w]);
+  return v;
+}
+
+// x / K in double: an exact scaling when K is a power of two.
+__device__ __forceinline__ double div_by_count(double x, int64_t K) {
+  return (K & (K - 1)) == 0 ? __dmul_rn(x, __drcp_rn((double)K)) : __ddiv_rn(x, (double)K);
+}
+
+// Normalisation whose weight (and bias) already carry diag(s)^-1 (gs =
+// gamma * inv_s, bs = beta * inv_s, folded ahead of time), then per-token
+// INT8.  kLN false: RMS normalisation, v = (x * r) * gs with
+// r = 1/sqrt(mean(x^2) + eps).  kLN true: layer normalisation,
+// v = ((x - mu) * r) * gs + bs with r = 1/sqrt(mean((x - mu)^2) + eps); bs
+// may be null (no bias).  Persistent like quant_rows_kernel: the folded
+// weight stays in registers across rows and the next row is prefetched
+// while the current one is reduced (the statistics in double, then the
+// absmax of v, recomputed for the codes rather than held).
+template <typename T, int kVPT, bool kLN>
 __global__ void __launch_bounds__(kRowMaxThreads)
-    rmsnorm_quant_rows_kernel(const T *__restrict__ x, int64_t rows, int64_t nvec, int64_t ld,
-                              const float *__restrict__ gs, float eps, int8_t *__restrict__ q,
-                              float *__restrict__ row_scale_out) {
+    norm_quant_rows_kernel(const T *__restrict__ x, int64_t rows, int64_t nvec, int64_t ld,
+                           const float *__restrict__ gs, const float *__restrict__ bs, float eps,
+                           int8_t *__restrict__ q, float *__restrict__ row_scale_out) {
   pdl_wait();  // the previous kernel's results are visible from here on
   pdl_trigger();
   constexpr int V = Vec<T>::N;
   __shared__ double red_ss[2][kRowMaxThreads / 32];
+  __shared__ double red_mu[kLN ? 2 : 1][kRowMaxThreads / 32];
   __shared__ float red_m[2][kRowMaxThreads / 32];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int nwarps = blockDim.x >> 5;
@@ -75,6 +128,13 @@ __global__ void __launch_bounds__(kRowMaxThreads)
     const int64_t v = tid + (int64_t)i * blockDim.x;
     cur[i] = (r < rows && v < nvec) ? ld_policy_v4(x + r * ld + v * V, policy) : make_uint4(0, 0, 0, 0);
   }
+  // the bias is read through L1 in each pass (held in registers next to gs
+  // it would spill); vectors past the row end, or no bias, read zeros
+  auto bias = [&](int i, int e) -> float2 {
+    const int64_t v = tid + (int64_t)i * blockDim.x;
+    if (bs == nullptr || v >= nvec) return make_float2(0.0f, 0.0f);
+    return __ldg(reinterpret_cast<const float2 *>(bs + v * V + e));
+  };
   int slot = 0;
   for (; r < rows; r += gridDim.x) {
     const int64_t rn = r + gridDim.x;
@@ -83,27 +143,34 @@ __global__ void __launch_bounds__(kRowMaxThreads)
       const int64_t v = tid + (int64_t)i * blockDim.x;
       nxt[i] = (rn < rows && v < nvec) ? ld_policy_v4(x + rn * ld + v * V, policy) : make_uint4(0, 0, 0, 0);
     }
-    // sum of squares in double (each square exact): one partial per
-    // vector, then a tree -- the order of this sum is left open by the
-    // definition
+    // the statistics in double, one partial per vector, then a tree -- the
+    // order of these sums is left open by the definition
+    double mu = 0.0;
+    float muf = 0.0f;
     double part[kVPT];
+    if constexpr (kLN) {
 #pragma unroll
-    for (int i = 0; i < kVPT; ++i) part[i] = sumsq_vec<T>(cur[i]);
+      for (int i = 0; i < kVPT; ++i) part[i] = sum_vec<T>(cur[i]);
+#pragma unroll
+      for (int w = kVPT / 2; w > 0; w >>= 1)
+#pragma unroll
+        for (int i = 0; i < w; ++i) part[i] = __dadd_rn(part[i], part[i + w]);
+      mu = div_by_count(block_sum_d(part[0], red_mu[slot], lane, warp, nwarps), K);
+      muf = __double2float_rn(mu);
+#pragma unroll
+      for (int i = 0; i < kVPT; ++i) part[i] = devsq_vec<T>(cur[i], mu, tid + (int64_t)i * blockDim.x < nvec);
+    } else {
+#pragma unroll
+      for (int i = 0; i < kVPT; ++i) part[i] = sumsq_vec<T>(cur[i]);
+    }
 #pragma unroll
     for (int w = kVPT / 2; w > 0; w >>= 1)
 #pragma unroll
       for (int i = 0; i < w; ++i) part[i] = __dadd_rn(part[i], part[i + w]);
-    double ss = part[0];
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) ss = __dadd_rn(ss, __shfl_xor_sync(0xffffffffu, ss, o));
-    if (lane == 0) red_ss[slot][warp] = ss;
-    __syncthreads();
-    ss = 0.0;
-    for (int w = 0; w < nwarps; ++w) ss = __dadd_rn(ss, red_ss[slot][w]);
-    // ss / K: an exact scaling when K is a power of two
-    const double mean = (K & (K - 1)) == 0 ? __dmul_rn(ss, __drcp_rn((double)K)) : __ddiv_rn(ss, (double)K);
-    const float rt = __double2float_rn(__ddiv_rn(1.0, __dsqrt_rn(__dadd_rn(mean, (double)eps))));
-    // absmax of v = (x * r) * gs (lanes past the row end hold x = gs = 0)
+    const double ms = div_by_count(block_sum_d(part[0], red_ss[slot], lane, warp, nwarps), K);
+    const float rt = __double2float_rn(__ddiv_rn(1.0, __dsqrt_rn(__dadd_rn(ms, (double)eps))));
+    // absmax of v (lanes past the row end hold x = gs = bs = 0 and give
+    // v = 0, or -muf * r * 0 = +-0)
     float m = 0.0f;
 #pragma unroll
     for (int i = 0; i < kVPT; ++i) {
@@ -111,8 +178,13 @@ __global__ void __launch_bounds__(kRowMaxThreads)
       Vec<T>::to_f32(cur[i], f);
 #pragma unroll
       for (int e = 0; e < V; e += 2) {
-        const float2 p = fmul2_rn(fmul2_rn(make_float2(f[e], f[e + 1]), make_float2(rt, rt)),
-                                  make_float2(g[i][e], g[i][e + 1]));
+        float2 c = make_float2(f[e], f[e + 1]);
+        if constexpr (kLN) c = fsub2_rn(c, make_float2(muf, muf));
+        float2 p = fmul2_rn(fmul2_rn(c, make_float2(rt, rt)), make_float2(g[i][e], g[i][e + 1]));
+        if constexpr (kLN) {
+          const float2 bb = bias(i, e);
+          p = make_float2(__fadd_rn(p.x, bb.x), __fadd_rn(p.y, bb.y));
+        }
         m = fmax3(m, fabsf(p.x), fabsf(p.y));
       }
     }
@@ -135,8 +207,13 @@ __global__ void __launch_bounds__(kRowMaxThreads)
         float val[V];
 #pragma unroll
         for (int e = 0; e < V; e += 2) {
-          const float2 p = fmul2_rn(fmul2_rn(make_float2(f[e], f[e + 1]), make_float2(rt, rt)),
-                                    make_float2(g[i][e], g[i][e + 1]));
+          float2 c = make_float2(f[e], f[e + 1]);
+          if constexpr (kLN) c = fsub2_rn(c, make_float2(muf, muf));
+          float2 p = fmul2_rn(fmul2_rn(c, make_float2(rt, rt)), make_float2(g[i][e], g[i][e + 1]));
+          if constexpr (kLN) {
+            const float2 bb = bias(i, e);
+            p = make_float2(__fadd_rn(p.x, bb.x), __fadd_rn(p.y, bb.y));
+          }
           val[e] = p.x;
           val[e + 1] = p.y;
         }
@@ -236,9 +313,9 @@ __global__ void __launch_bounds__(256) quant_static_kernel(const T *__restrict__
   }
 }
 
-template <typename T>
-cudaError_t rmsnorm_quant_t(const void *x, int64_t rows, int64_t cols, int64_t ld, const float *gs, float eps,
-                            int8_t *q, float *row_scale_out, cudaStream_t st) {
+template <typename T, bool kLN>
+cudaError_t norm_quant_t(const void *x, int64_t rows, int64_t cols, int64_t ld, const float *gs, const float *bs,
+                         float eps, int8_t *q, float *row_scale_out, cudaStream_t st) {
   constexpr int V = Vec<T>::N;
   const int64_t nvec = cols / V;
   if (nvec > 4 * kRowMaxThreads) return cudaErrorNotSupported;
@@ -246,13 +323,13 @@ cudaError_t rmsnorm_quant_t(const void *x, int64_t rows, int64_t cols, int64_t l
   const int vpt = nvec <= 4 * 32 ? 1 : 4;
   int64_t t = (nvec + vpt - 1) / vpt;
   const int threads = (int)std::max<int64_t>(32, ((t + 31) / 32) * 32);
-  auto kern = vpt == 1 ? rmsnorm_quant_rows_kernel<T, 1> : rmsnorm_quant_rows_kernel<T, 4>;
+  auto kern = vpt == 1 ? norm_quant_rows_kernel<T, 1, kLN> : norm_quant_rows_kernel<T, 4, kLN>;
   int per_sm = 0;
   cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, 0);
   if (e != cudaSuccess) return e;
   const int64_t grid = std::min<int64_t>(rows, (int64_t)std::max(1, per_sm) * num_sms());
-  return launch_pdl(kern, dim3((unsigned)grid), dim3(threads), 0, st, 1, (const T *)x, rows, nvec, ld, gs, eps, q,
-                    row_scale_out);
+  return launch_pdl(kern, dim3((unsigned)grid), dim3(threads), 0, st, 1, (const T *)x, rows, nvec, ld, gs, bs, eps,
+                    q, row_scale_out);
 }
 
 template <typename T>
@@ -273,9 +350,19 @@ cudaError_t quant_static_t(const void *x, int64_t rows, int64_t cols, int64_t ld
 cudaError_t launch_rmsnorm_quant(const void *x, sq_dtype xt, int64_t rows, int64_t cols, int64_t ld,
                                  const float *gs, float eps, int8_t *q, float *row_scale_out, cudaStream_t st) {
   switch (xt) {
-    case SQ_F32: return rmsnorm_quant_t<float>(x, rows, cols, ld, gs, eps, q, row_scale_out, st);
-    case SQ_F16: return rmsnorm_quant_t<__half>(x, rows, cols, ld, gs, eps, q, row_scale_out, st);
-    default: return rmsnorm_quant_t<__nv_bfloat16>(x, rows, cols, ld, gs, eps, q, row_scale_out, st);
+    case SQ_F32: return norm_quant_t<float, false>(x, rows, cols, ld, gs, nullptr, eps, q, row_scale_out, st);
+    case SQ_F16: return norm_quant_t<__half, false>(x, rows, cols, ld, gs, nullptr, eps, q, row_scale_out, st);
+    default: return norm_quant_t<__nv_bfloat16, false>(x, rows, cols, ld, gs, nullptr, eps, q, row_scale_out, st);
+  }
+}
+
+cudaError_t launch_layernorm_quant(const void *x, sq_dtype xt, int64_t rows, int64_t cols, int64_t ld,
+                                   const float *gs, const float *bs, float eps, int8_t *q, float *row_scale_out,
+                                   cudaStream_t st) {
+  switch (xt) {
+    case SQ_F32: return norm_quant_t<float, true>(x, rows, cols, ld, gs, bs, eps, q, row_scale_out, st);
+    case SQ_F16: return norm_quant_t<__half, true>(x, rows, cols, ld, gs, bs, eps, q, row_scale_out, st);
+    default: return norm_quant_t<__nv_bfloat16, true>(x, rows, cols, ld, gs, bs, eps, q, row_scale_out, st);
   }
 }
 

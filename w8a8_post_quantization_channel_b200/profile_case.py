@@ -5,8 +5,8 @@ of the workloads' shapes, for profilers and roofline measurements.
       --M 2048 --K 4096 --N 16384 --dtype f16 --iters 3
   python -m w8a8_post_quantization_channel_b200.profile_case --sweep decode
 
---op is calib (T = M tokens), weight (W [N, K]), act, rmsnorm (the fused
-norm producer), static (static-scale quantizer), linear, or the FP8 (E4M3)
+--op is calib (T = M tokens), weight (W [N, K]), act, rmsnorm and
+layernorm (the fused norm producers), static (static-scale quantizer), linear, or the FP8 (E4M3)
 forms act8, weight8 and linear8, or rot (butterfly-rotated act-quant, --N =
 the rotation block size).  With
 --time (implied by --sweep) every iteration is timed with CUDA events on
@@ -51,9 +51,11 @@ SWEEPS = {
     # smoothing + weight quantization, [K, K] and the OPT shapes
     "weight": [("weight", 0, K, K, "bf16") for K in (4096, 7168, 8192, 28672)] + [("weight", 0, 4096, 12288, "f16"),
                                                                                      ("weight", 0, 16384, 4096, "f16")],
-    # upstream producer (RMSNorm + smoothing + per-token INT8) and the static
-    # per-tensor quantizer on 16384-token batches
+    # upstream producers (RMSNorm or LayerNorm + smoothing + per-token INT8)
+    # and the static per-tensor quantizer on 16384-token batches
     "producer": [("rmsnorm", 16384, K, 0, "bf16") for K in (4096, 8192)] + [("rmsnorm", 2048, 4096, 0, "f16")]
+                + [("layernorm", 16384, K, 0, "bf16") for K in (4096, 8192)]
+                + [("layernorm", 2048, 4096, 0, "f16"), ("layernorm", 16384, 4096, 0, "f16")]
                 + [("static", 16384, K, 0, "bf16") for K in (4096, 8192)],
     # butterfly-rotated activation quantization (N = the rotation's block size n)
     "rot": [("rot", 16384, 4096, n, "bf16") for n in (16, 64, 256, 4096)] + [("rot", 16384, 8192, 256, "bf16")],
@@ -81,7 +83,7 @@ def peaks():
 def make_case(op, M, K, N, dtype, dev="cuda"):
     dt = DT[dtype]
     o = synth.outliers(K, frac=0.01, mult=100.0, seed=1)
-    if op in ("rmsnorm", "static"):
+    if op in ("rmsnorm", "layernorm", "static"):
         x = synth.activations(M, K, o, 2, dt, device=dev)
         inv = torch.rand(K, device=dev) + 0.5
         gamma = torch.rand(K, device=dev) + 0.5
@@ -92,6 +94,10 @@ def make_case(op, M, K, N, dtype, dev="cuda"):
         if op == "rmsnorm":
             gs = sq.sq_fold_smooth_into_norm(gamma, inv)
             return (lambda: sq.sq_rmsnorm_quant_act(x, gs, 1e-5, xq=xq, x_scale=xs)), nbytes, None
+        if op == "layernorm":
+            gs = sq.sq_fold_smooth_into_norm(gamma, inv)
+            bs = sq.sq_fold_smooth_into_norm(torch.rand(K, device=dev) - 0.5, inv)
+            return (lambda: sq.sq_layernorm_quant_act(x, gs, bs, 1e-5, xq=xq, x_scale=xs)), nbytes + 4 * K, None
         return (lambda: sq.sq_quant_act_static(x, inv, delta, xq=xq, x_scale=xs)), nbytes, None
     if op in ("calib", "act"):
         x = synth.activations(M, K, o, 2, dt, device=dev)
@@ -192,8 +198,8 @@ def time_case(op, M, K, N, dtype, iters):
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--op", choices=["calib", "weight", "act", "linear", "rmsnorm", "static", "act8", "weight8",
-                                     "linear8", "rot"])
+    ap.add_argument("--op", choices=["calib", "weight", "act", "linear", "rmsnorm", "layernorm", "static", "act8",
+                                     "weight8", "linear8", "rot"])
     ap.add_argument("--sweep", choices=sorted(SWEEPS))
     ap.add_argument("--M", type=int, default=2048)
     ap.add_argument("--K", type=int, default=4096)
