@@ -284,7 +284,9 @@ void or_rmsnorm_factor(const float *x, int64_t M, int64_t K, float eps, float *r
  *                                               its square in double)
  *   r_t   = (float)(1 / sqrt(var_t + eps))     (double, rounded once)
  *   muf_t = (float)mu_t
- *   v_tj  = ((x_tj - muf_t) * r_t) * gs_j + bs_j   (fp32, in that order)
+ *   n_tj  = (x_tj - muf_t) * r_t                   (fp32, in that order)
+ *   v_tj  = fma(n_tj, gs_j, bs_j)                  (the affine step of the
+ *                                                   norm, rounded once)
  * then per-token quantization of v as in or_quant_act.  bs may be NULL (no
  * bias). */
 static void or_layernorm_row_stats(const float *row, int64_t K, float eps, float *muf, float *r) {
@@ -307,8 +309,7 @@ void or_layernorm_stats(const float *x, int64_t M, int64_t K, float eps, float *
 static float or_layernorm_value(float x, float muf, float r, float g, float b) {
   const float c = x - muf;
   const float n = c * r;
-  const float w = n * g;
-  return w + b;
+  return fmaf(n, g, b); /* the affine step n * g + b, rounded once */
 }
 
 void or_layernorm_quant_act(const float *x, int64_t M, int64_t K, const float *gs, const float *bs, float eps,

@@ -12,6 +12,7 @@ mathematics fix, never against the oracle itself.
 - brute-force integer matrix products and library reductions/conversions.
 """
 from decimal import Decimal, getcontext
+from fractions import Fraction
 
 import numpy as np
 import pytest
@@ -35,6 +36,17 @@ def _int(rows):
     if rows and isinstance(rows[0], list):
         return np.array([[int(v) for v in r] for r in rows], np.int64)
     return np.array([int(v) for v in rows], np.int64)
+
+
+def _round_f32(fr: Fraction) -> np.float32:
+    """The fp32 nearest to the rational fr, ties to even."""
+    f = np.float32(float(fr))
+    best = f
+    for c in (np.nextafter(f, np.float32(-np.inf)), np.nextafter(f, np.float32(np.inf))):
+        d_c, d_b = abs(Fraction(float(c)) - fr), abs(Fraction(float(best)) - fr)
+        if d_c < d_b or (d_c == d_b and (int(c.view(np.uint32)) & 1) == 0):
+            best = c
+    return best
 
 
 def _ulps(got, exact):
@@ -551,7 +563,10 @@ def test_folded_layernorm_equals_norm_then_smoothing():
                                         oracle.fold_norm_weight(beta, inv_s), eps)
     mu, r = oracle.layernorm_stats(x, eps)
     n = ((x - mu[:, None]).astype(np.float32) * r[:, None]).astype(np.float32)
-    normed = ((n * gamma).astype(np.float32) + beta).astype(np.float32)
+    # the affine step n * gamma + beta, taken exactly in rationals and
+    # rounded once to fp32
+    normed = np.array([[_round_f32(Fraction(float(n[t, j])) * Fraction(float(gamma[j])) + Fraction(float(beta[j])))
+                        for j in range(K)] for t in range(n.shape[0])], np.float32)
     xq_u, dx_u = oracle.quant_act(normed, inv_s)
     np.testing.assert_array_equal(xq, xq_u)
     np.testing.assert_array_equal(dx, dx_u)
