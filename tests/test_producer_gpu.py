@@ -127,6 +127,11 @@ def test_layernorm_quant_act(dt, K, M, bias):
     x += 0.75  # a nonzero mean for the normalisation to remove
     if M > 3:
         x[3] = 2.5  # a constant token: variance 0, every value -> the bias
+    if M > 6:
+        # a token with a large mean and a small spread (mean^2 / var ~ 1e5),
+        # and one whose first value is an outlier
+        x[5] = 1000.0 + 4.0 * torch.randint(-1, 2, (K,), generator=synth.gen(K + 10)).to(x.dtype)
+        x[6, 0] = 3000.0
     g = synth.gen(K + 9)
     gamma = torch.rand(K, generator=g) * 2.0 + 0.05
     beta = torch.rand(K, generator=g) - 0.5

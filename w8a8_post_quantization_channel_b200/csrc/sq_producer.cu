@@ -9,7 +9,7 @@
 //   fold        gs_j = gamma_j * inv_s_j
 //   producer    r_t = 1 / sqrt(sum_j x_tj^2 / K + eps), v = (x r) gs, INT8
 //   LayerNorm   mu_t = mean_j x_tj, r_t = 1 / sqrt(mean_j (x_tj - mu_t)^2 + eps),
-//               v = ((x - mu) r) gs + bs, INT8 (bs = beta * inv_s)
+//               v = fma((x - mu) r, gs, bs), INT8 (bs = beta * inv_s)
 //   static      delta = max_j(amax_j inv_s_j) / 127, q = sat(rne(x inv_s / delta))
 #include <algorithm>
 
@@ -38,33 +38,29 @@ __device__ __forceinline__ double sumsq_vec(uint4 raw) {
   return acc;
 }
 
-// Sum of one 16-byte row vector in double (each value converted exactly).
+// Shifted sums of one 16-byte row vector in double: s += sum_e (x_e - c),
+// q += sum_e (x_e - c)^2, each value converted exactly, in two chains per
+// sum.  Lanes past the row end hold x = 0 and must add nothing: `live` is
+// false there.
 template <typename T>
-__device__ __forceinline__ double sum_vec(uint4 raw) {
+__device__ __forceinline__ void shifted_sums_vec(uint4 raw, double c, bool live, double &s, double &q) {
   constexpr int V = Vec<T>::N;
   float f[V];
   Vec<T>::to_f32(raw, f);
-  double acc = 0.0;
+  double s0 = 0.0, s1 = 0.0, q0 = 0.0, q1 = 0.0;
 #pragma unroll
-  for (int e = 0; e < V; ++e) acc = __dadd_rn(acc, (double)f[e]);
-  return acc;
-}
-
-// Sum of the squared deviations from mu of one row vector, in double.
-// Lanes past the row end hold x = 0 and must add nothing: `live` is false
-// there.
-template <typename T>
-__device__ __forceinline__ double devsq_vec(uint4 raw, double mu, bool live) {
-  constexpr int V = Vec<T>::N;
-  float f[V];
-  Vec<T>::to_f32(raw, f);
-  double acc = 0.0;
-#pragma unroll
-  for (int e = 0; e < V; ++e) {
-    const double d = __dsub_rn((double)f[e], mu);
-    acc = __fma_rn(d, d, acc);
+  for (int e = 0; e < V; e += 2) {
+    const double d0 = __dsub_rn((double)f[e], c);
+    const double d1 = __dsub_rn((double)f[e + 1], c);
+    s0 = __dadd_rn(s0, d0);
+    s1 = __dadd_rn(s1, d1);
+    q0 = __fma_rn(d0, d0, q0);
+    q1 = __fma_rn(d1, d1, q1);
   }
-  return live ? acc : 0.0;
+  if (live) {
+    s = __dadd_rn(s, __dadd_rn(s0, s1));
+    q = __dadd_rn(q, __dadd_rn(q0, q1));
+  }
 }
 
 // Block-wide double sum of one per-thread partial through red[] (one slot
@@ -79,6 +75,28 @@ __device__ __forceinline__ double block_sum_d(double v, double *red, int lane, i
   return v;
 }
 
+// Block-wide double sums of two per-thread partials through red[] (two
+// slots per warp); every thread gets both totals.
+__device__ __forceinline__ void block_sum_d2(double &a, double &b, double (*red)[2], int lane, int warp,
+                                             int nwarps) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    a = __dadd_rn(a, __shfl_xor_sync(0xffffffffu, a, o));
+    b = __dadd_rn(b, __shfl_xor_sync(0xffffffffu, b, o));
+  }
+  if (lane == 0) {
+    red[warp][0] = a;
+    red[warp][1] = b;
+  }
+  __syncthreads();
+  a = 0.0;
+  b = 0.0;
+  for (int w = 0; w < nwarps; ++w) {
+    a = __dadd_rn(a, red[w][0]);
+    b = __dadd_rn(b, red[w][1]);
+  }
+}
+
 // x / K in double: an exact scaling when K is a power of two.
 __device__ __forceinline__ double div_by_count(double x, int64_t K) {
   return (K & (K - 1)) == 0 ? __dmul_rn(x, __drcp_rn((double)K)) : __ddiv_rn(x, (double)K);
@@ -88,8 +106,8 @@ __device__ __forceinline__ double div_by_count(double x, int64_t K) {
 // gamma * inv_s, bs = beta * inv_s, folded ahead of time), then per-token
 // INT8.  kLN false: RMS normalisation, v = (x * r) * gs with
 // r = 1/sqrt(mean(x^2) + eps).  kLN true: layer normalisation,
-// v = ((x - mu) * r) * gs + bs with r = 1/sqrt(mean((x - mu)^2) + eps); bs
-// may be null (no bias).  Persistent like quant_rows_kernel: the folded
+// v = fma((x - mu) * r, gs, bs) with r = 1/sqrt(mean((x - mu)^2) + eps),
+// the mean and variance from one shifted pass; bs may be null (no bias).  Persistent like quant_rows_kernel: the folded
 // weight stays in registers across rows and the next row is prefetched
 // while the current one is reduced (the statistics in double, then the
 // absmax of v, recomputed for the codes rather than held).
@@ -102,13 +120,14 @@ __global__ void __launch_bounds__(kRowMaxThreads)
   pdl_trigger();
   constexpr int V = Vec<T>::N;
   __shared__ double red_ss[2][kRowMaxThreads / 32];
-  __shared__ double red_mu[kLN ? 2 : 1][kRowMaxThreads / 32];
+  __shared__ double red_sq[kLN ? 2 : 1][kRowMaxThreads / 32][2];
   __shared__ float red_m[2][kRowMaxThreads / 32];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int nwarps = blockDim.x >> 5;
   const int64_t K = nvec * V;
   const uint64_t policy = policy_evict_first();
   float g[kVPT][V];
+  float b[kLN ? kVPT : 1][V];
 #pragma unroll
   for (int i = 0; i < kVPT; ++i) {
     const int64_t v = tid + (int64_t)i * blockDim.x;
@@ -119,6 +138,14 @@ __global__ void __launch_bounds__(kRowMaxThreads)
       g[i][4 * e4 + 1] = gv.y;
       g[i][4 * e4 + 2] = gv.z;
       g[i][4 * e4 + 3] = gv.w;
+      if constexpr (kLN) {
+        const float4 bv = (v < nvec && bs != nullptr) ? __ldg(reinterpret_cast<const float4 *>(bs + v * V) + e4)
+                                                      : make_float4(0, 0, 0, 0);
+        b[i][4 * e4 + 0] = bv.x;
+        b[i][4 * e4 + 1] = bv.y;
+        b[i][4 * e4 + 2] = bv.z;
+        b[i][4 * e4 + 3] = bv.w;
+      }
     }
   }
   uint4 cur[kVPT], nxt[kVPT];
@@ -128,13 +155,9 @@ __global__ void __launch_bounds__(kRowMaxThreads)
     const int64_t v = tid + (int64_t)i * blockDim.x;
     cur[i] = (r < rows && v < nvec) ? ld_policy_v4(x + r * ld + v * V, policy) : make_uint4(0, 0, 0, 0);
   }
-  // the bias is read through L1 in each pass (held in registers next to gs
-  // it would spill); vectors past the row end, or no bias, read zeros
-  auto bias = [&](int i, int e) -> float2 {
-    const int64_t v = tid + (int64_t)i * blockDim.x;
-    if (bs == nullptr || v >= nvec) return make_float2(0.0f, 0.0f);
-    return __ldg(reinterpret_cast<const float2 *>(bs + v * V + e));
-  };
+  // LayerNorm: the row's first value, the shift of its one-pass statistics
+  double c_cur = 0.0, c_nxt = 0.0;
+  if constexpr (kLN) c_cur = r < rows ? (double)Vec<T>::one(x + r * ld) : 0.0;
   int slot = 0;
   for (; r < rows; r += gridDim.x) {
     const int64_t rn = r + gridDim.x;
@@ -143,32 +166,48 @@ __global__ void __launch_bounds__(kRowMaxThreads)
       const int64_t v = tid + (int64_t)i * blockDim.x;
       nxt[i] = (rn < rows && v < nvec) ? ld_policy_v4(x + rn * ld + v * V, policy) : make_uint4(0, 0, 0, 0);
     }
-    // the statistics in double, one partial per vector, then a tree -- the
-    // order of these sums is left open by the definition
-    double mu = 0.0;
+    if constexpr (kLN) c_nxt = rn < rows ? (double)Vec<T>::one(x + rn * ld) : 0.0;
+    // the statistics in double -- the order of these sums is left open by
+    // the definition
+    double ms;  // the mean square under the root: mean(x^2), or var
     float muf = 0.0f;
-    double part[kVPT];
     if constexpr (kLN) {
+      // One pass over the deviations d = x - c from the row's first value
+      // c: with S = sum d and Q = sum d^2, mu = c + S/K and
+      // var = Q/K - (S/K)^2.  As c is one of the row's values,
+      // (mu - c)^2 <= K var, so the subtraction loses at most log2(K + 1)
+      // bits of the double's 53: var and r stay within 2^-34 (relative) of
+      // the two-pass values, far inside one fp32 ulp.
+      double sh = 0.0, q = 0.0;
 #pragma unroll
-      for (int i = 0; i < kVPT; ++i) part[i] = sum_vec<T>(cur[i]);
+      for (int i = 0; i < kVPT; ++i)
+        shifted_sums_vec<T>(cur[i], c_cur, tid + (int64_t)i * blockDim.x < nvec, sh, q);
+      block_sum_d2(sh, q, red_sq[slot], lane, warp, nwarps);
+      const double m1 = div_by_count(sh, K);
+      ms = fmax(__fma_rn(-m1, m1, div_by_count(q, K)), 0.0);
+      muf = __double2float_rn(__dadd_rn(c_cur, m1));
+      c_cur = c_nxt;
+    } else {
+      double part[kVPT];
+#pragma unroll
+      for (int i = 0; i < kVPT; ++i) part[i] = sumsq_vec<T>(cur[i]);
 #pragma unroll
       for (int w = kVPT / 2; w > 0; w >>= 1)
 #pragma unroll
         for (int i = 0; i < w; ++i) part[i] = __dadd_rn(part[i], part[i + w]);
-      mu = div_by_count(block_sum_d(part[0], red_mu[slot], lane, warp, nwarps), K);
-      muf = __double2float_rn(mu);
-#pragma unroll
-      for (int i = 0; i < kVPT; ++i) part[i] = devsq_vec<T>(cur[i], mu, tid + (int64_t)i * blockDim.x < nvec);
-    } else {
-#pragma unroll
-      for (int i = 0; i < kVPT; ++i) part[i] = sumsq_vec<T>(cur[i]);
+      ms = div_by_count(block_sum_d(part[0], red_ss[slot], lane, warp, nwarps), K);
     }
-#pragma unroll
-    for (int w = kVPT / 2; w > 0; w >>= 1)
-#pragma unroll
-      for (int i = 0; i < w; ++i) part[i] = __dadd_rn(part[i], part[i + w]);
-    const double ms = div_by_count(block_sum_d(part[0], red_ss[slot], lane, warp, nwarps), K);
     const float rt = __double2float_rn(__ddiv_rn(1.0, __dsqrt_rn(__dadd_rn(ms, (double)eps))));
+    // v for values e, e+1 of vector i: (x * r) * gs, or for LayerNorm
+    // fma((x - mu) * r, gs, bs), the affine step rounded once
+    auto value2 = [&](const float (&f)[V], int i, int e) -> float2 {
+      if constexpr (kLN) {
+        const float2 n = fmul2_rn(fsub2_rn(make_float2(f[e], f[e + 1]), make_float2(muf, muf)), make_float2(rt, rt));
+        return ffma2_rn(n, make_float2(g[i][e], g[i][e + 1]), make_float2(b[i][e], b[i][e + 1]));
+      } else {
+        return fmul2_rn(fmul2_rn(make_float2(f[e], f[e + 1]), make_float2(rt, rt)), make_float2(g[i][e], g[i][e + 1]));
+      }
+    };
     // absmax of v (lanes past the row end hold x = gs = bs = 0 and give
     // v = 0, or -muf * r * 0 = +-0)
     float m = 0.0f;
@@ -178,13 +217,7 @@ __global__ void __launch_bounds__(kRowMaxThreads)
       Vec<T>::to_f32(cur[i], f);
 #pragma unroll
       for (int e = 0; e < V; e += 2) {
-        float2 c = make_float2(f[e], f[e + 1]);
-        if constexpr (kLN) c = fsub2_rn(c, make_float2(muf, muf));
-        float2 p = fmul2_rn(fmul2_rn(c, make_float2(rt, rt)), make_float2(g[i][e], g[i][e + 1]));
-        if constexpr (kLN) {
-          const float2 bb = bias(i, e);
-          p = make_float2(__fadd_rn(p.x, bb.x), __fadd_rn(p.y, bb.y));
-        }
+        const float2 p = value2(f, i, e);
         m = fmax3(m, fabsf(p.x), fabsf(p.y));
       }
     }
@@ -207,13 +240,7 @@ __global__ void __launch_bounds__(kRowMaxThreads)
         float val[V];
 #pragma unroll
         for (int e = 0; e < V; e += 2) {
-          float2 c = make_float2(f[e], f[e + 1]);
-          if constexpr (kLN) c = fsub2_rn(c, make_float2(muf, muf));
-          float2 p = fmul2_rn(fmul2_rn(c, make_float2(rt, rt)), make_float2(g[i][e], g[i][e + 1]));
-          if constexpr (kLN) {
-            const float2 bb = bias(i, e);
-            p = make_float2(__fadd_rn(p.x, bb.x), __fadd_rn(p.y, bb.y));
-          }
+          const float2 p = value2(f, i, e);
           val[e] = p.x;
           val[e + 1] = p.y;
         }
