@@ -321,11 +321,6 @@ struct FmtE4M3 {
   }
 };
 
-__device__ __forceinline__ uint32_t pack4_i8(int a, int b, int c, int d) {
-  return (uint32_t)(a & 0xff) | ((uint32_t)(b & 0xff) << 8) | ((uint32_t)(c & 0xff) << 16) |
-         ((uint32_t)(d & 0xff) << 24);
-}
-
 // Max over a warp; values are non-negative floats.
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
