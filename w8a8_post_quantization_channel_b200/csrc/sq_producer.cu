@@ -593,60 +593,164 @@ __global__ void __launch_bounds__(kRowMaxThreads)
 }
 
 // Blocks wider than a warp's 32 V channels: R rows (R <= 4) are staged in
-// shared memory as fp32 and every stage walks the pairs by index -- pair q
-// of a row is pair j = q mod (n/2) of block q / (n/2), whose first element
-// sits at ((j >> i) << (i + 1)) | (j mod 2^i) -- with (c, s) = cs[i][j] read
-// through L1/L2 once for all R rows; a barrier separates the stages.
-// Persistent over groups of R rows; the codes follow as in the other row
-// quantizers.
+// shared memory as fp32, and the stages run in radix-8 passes.  A pass
+// takes stages i0, i0+1 and i0+2 at once on groups of 8 values at positions
+// p0 + k 2^i0 (k < 8; p0 with bits i0..i0+2 clear): each thread loads a
+// group, applies the three stages in registers -- stage i0+s pairs k and
+// k + 2^s -- and stores it back, so a pass costs one barrier and one
+// shared-memory round trip for three stages.  The first pass (stages 0-2,
+// 8 contiguous values) runs as the rows are loaded.  The group's angles,
+// cs[i][j] with j = ((p >> (i+1)) << i) | (p mod 2^i) for the pair's first
+// position p, are read once for all R rows.  Shared-memory slots are padded
+// by one word per 32 (slot p + p / 32), which spreads the stride-8 accesses
+// of the first pass over all 32 banks.  Persistent over groups of R rows;
+// the codes follow as in the other row quantizers.
+__device__ __forceinline__ int rot_slot(int p) { return p + (p >> 5); }
+
+// Angles of r stages starting at i0 for the group whose first value sits at
+// block position pb (bits i0..i0+r-1 clear): t[s][m] for pair m of stage
+// i = i0 + s.  Pair m's first position is pb + k 2^i0 with k = m with a
+// zero bit inserted at s; dropping bit i of it gives j = jb + m 2^i0, where
+// jb drops bit i of pb.
+template <int r>
+__device__ __forceinline__ void group_angles(const float2 *__restrict__ cs, int half, int i0, int pb,
+                                             float2 (&t)[r][1 << (r - 1)]) {
+#pragma unroll
+  for (int s = 0; s < r; ++s) {
+    const int i = i0 + s;
+    const float2 *row = cs + (int64_t)i * half + (((pb >> (i + 1)) << i) | (pb & ((1 << i) - 1)));
+#pragma unroll
+    for (int m = 0; m < (1 << (r - 1)); ++m) t[s][m] = __ldg(row + (m << i0));
+  }
+}
+
+// r stages on the 2^r values of a group: (a, b) -> (c a - s b, s a + c b),
+// every product and sum rounded as the definition states.  With t = (c, s)
+// and ts = (s, c): (a, b) * t = (c a, s b) and (a, b) * ts = (s a, c b), so
+// a butterfly is two packed products and two scalar sums.
+template <int r>
+__device__ __forceinline__ void group_stages(float (&v)[1 << r], const float2 (&t)[r][1 << (r - 1)],
+                                             const float2 (&ts)[r][1 << (r - 1)]) {
+#pragma unroll
+  for (int s = 0; s < r; ++s) {
+#pragma unroll
+    for (int m = 0; m < (1 << (r - 1)); ++m) {
+      const int k = ((m >> s) << (s + 1)) | (m & ((1 << s) - 1));
+      const float2 ab = make_float2(v[k], v[k + (1 << s)]);
+      const float2 p = fmul2_rn(ab, t[s][m]);   // (c a, s b)
+      const float2 q = fmul2_rn(ab, ts[s][m]);  // (s a, c b)
+      v[k] = __fsub_rn(p.x, p.y);
+      v[k + (1 << s)] = __fadd_rn(q.x, q.y);
+    }
+  }
+}
+
+template <int r>
+__device__ __forceinline__ void swap_angles(const float2 (&t)[r][1 << (r - 1)], float2 (&ts)[r][1 << (r - 1)]) {
+#pragma unroll
+  for (int s = 0; s < r; ++s)
+#pragma unroll
+    for (int m = 0; m < (1 << (r - 1)); ++m) ts[s][m] = make_float2(t[s][m].y, t[s][m].x);
+}
+
+// One pass of r stages from i0 over nr staged rows of K values.  For
+// i0 >= 5 the group's slots are evenly spaced, slot(p0) + k (2^i0 +
+// 2^(i0-5)); i0 = 3 takes the slot of each position.  The last pass also
+// returns each row's largest magnitude over this thread's groups (mx).
+template <int r, bool kLast>
+__device__ __forceinline__ void rot_pass(float *rowbuf, int Kp, int nr, int K, int n, int i0,
+                                         const float2 *__restrict__ cs, float (&mx)[4]) {
+  const int half = n >> 1;
+  const int step = i0 >= 5 ? (1 << i0) + (1 << (i0 - 5)) : 0;
+  for (int gi = threadIdx.x; gi < (K >> r); gi += blockDim.x) {
+    const int p0 = ((gi >> i0) << (i0 + r)) | (gi & ((1 << i0) - 1));
+    float2 t[r][1 << (r - 1)], ts[r][1 << (r - 1)];
+    group_angles<r>(cs, half, i0, p0 & (n - 1), t);
+    swap_angles<r>(t, ts);
+    int slot[1 << r];
+#pragma unroll
+    for (int k = 0; k < (1 << r); ++k) slot[k] = step ? rot_slot(p0) + k * step : rot_slot(p0 + (k << i0));
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {  // nr <= 4 rows; unrolled so that mx[u] stays in registers
+      if (u >= nr) break;
+      float *buf = rowbuf + u * Kp;
+      float v[1 << r];
+#pragma unroll
+      for (int k = 0; k < (1 << r); ++k) v[k] = buf[slot[k]];
+      group_stages<r>(v, t, ts);
+#pragma unroll
+      for (int k = 0; k < (1 << r); ++k) buf[slot[k]] = v[k];
+      if constexpr (kLast) {
+#pragma unroll
+        for (int k = 0; k < (1 << r); k += 2) mx[u] = fmax3(mx[u], fabsf(v[k]), fabsf(v[k + 1]));
+      }
+    }
+  }
+}
+
 template <typename T>
-__global__ void __launch_bounds__(kRotSmemThreads)
+__global__ void __launch_bounds__(kRotSmemThreads, 2)
     rot_quant_rows_smem_kernel(const T *__restrict__ x, int64_t rows, int64_t nvec, int64_t ld,
                                const float *__restrict__ col_scale, int logn, const float2 *__restrict__ cs, int R,
                                int8_t *__restrict__ q, float *__restrict__ row_scale_out) {
-  extern __shared__ float rowbuf[];  // [R][K]
+  extern __shared__ float rowbuf[];  // [R][Kp]: value p of row u in slot u * Kp + rot_slot(p)
   __shared__ float red[32];
   constexpr int V = Vec<T>::N;
+  constexpr int kVecs = 8 / V;  // 16-byte vectors per group of 8 values
   pdl_wait();  // the previous kernel's results are visible from here on
   pdl_trigger();
-  const int K = (int)(nvec * V);  // <= 16384
-  const int half = 1 << (logn - 1);
-  const int pairs = K / 2;
+  const int K = (int)(nvec * V);  // <= 16384, a multiple of n >= 512
+  const int Kp = rot_slot(K);
+  const int n = 1 << logn;
   const int64_t groups = (rows + R - 1) / R;
   for (int64_t g = blockIdx.x; g < groups; g += gridDim.x) {
     const int64_t r0 = g * R;
     const int nr = (int)min((int64_t)R, rows - r0);
-    for (int u = 0; u < nr; ++u) {
-      const T *xr = x + (r0 + u) * ld;
-      float *buf = rowbuf + u * K;
-      for (int v = threadIdx.x; v < (int)nvec; v += blockDim.x) {
-        float f[V];
-        Vec<T>::to_f32(ld_nc_v4(xr + (int64_t)v * V), f);
+    // load, scale and stages 0-2 on groups of 8 contiguous values
+    for (int gi = threadIdx.x; gi < (K >> 3); gi += blockDim.x) {
+      const int p0 = gi << 3;
+      float2 t[3][4], ts[3][4];
+      group_angles<3>(cs, n >> 1, 0, p0 & (n - 1), t);
+      swap_angles<3>(t, ts);
+      float sc[8];
 #pragma unroll
-        for (int e = 0; e < V; ++e) buf[v * V + e] = __fmul_rn(f[e], __ldg(col_scale + v * V + e));
+      for (int k = 0; k < 8; ++k) sc[k] = __ldg(col_scale + p0 + k);
+      for (int u = 0; u < nr; ++u) {
+        const T *xr = x + (r0 + u) * ld + p0;
+        float v[8];
+#pragma unroll
+        for (int w = 0; w < kVecs; ++w) {
+          float f[V];
+          Vec<T>::to_f32(ld_nc_v4(xr + w * V), f);
+#pragma unroll
+          for (int e = 0; e < V; ++e) v[w * V + e] = __fmul_rn(f[e], sc[w * V + e]);
+        }
+        group_stages<3>(v, t, ts);
+        float *buf = rowbuf + u * Kp;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) buf[rot_slot(p0 + k)] = v[k];
       }
     }
     __syncthreads();
-    for (int st = 0; st < logn; ++st) {
-      const int h = 1 << st;
-      const float2 *ts = cs + (int64_t)st * half;
-      for (int pq = threadIdx.x; pq < pairs; pq += blockDim.x) {
-        const int j = pq & (half - 1);  // pair within its block; the block starts at (pq - j) * 2
-        const int pa = ((pq - j) << 1) + (((j >> st) << (st + 1)) | (j & (h - 1)));
-        const float2 t = __ldg(ts + j);
-        for (int u = 0; u < nr; ++u) {
-          float *buf = rowbuf + u * K;
-          const float a = buf[pa], b = buf[pa + h];
-          buf[pa] = __fsub_rn(__fmul_rn(t.x, a), __fmul_rn(t.y, b));
-          buf[pa + h] = __fadd_rn(__fmul_rn(t.y, a), __fmul_rn(t.x, b));
-        }
+    float mx[4] = {0.0f, 0.0f, 0.0f, 0.0f};  // per staged row (R <= 4)
+    for (int i0 = 3; i0 < logn; i0 += 3) {
+      const int left = logn - i0;
+      if (left > 3) {
+        rot_pass<3, false>(rowbuf, Kp, nr, K, n, i0, cs, mx);
+      } else if (left == 3) {
+        rot_pass<3, true>(rowbuf, Kp, nr, K, n, i0, cs, mx);
+      } else if (left == 2) {
+        rot_pass<2, true>(rowbuf, Kp, nr, K, n, i0, cs, mx);
+      } else {
+        rot_pass<1, true>(rowbuf, Kp, nr, K, n, i0, cs, mx);
       }
       __syncthreads();
     }
     for (int u = 0; u < nr; ++u) {
-      const float *buf = rowbuf + u * K;
+      const float *buf = rowbuf + u * Kp;
       float m = 0.0f;
-      for (int k = threadIdx.x; k < K; k += blockDim.x) m = fmaxf(m, fabsf(buf[k]));
+#pragma unroll
+      for (int w = 0; w < 4; ++w) m = w == u ? mx[w] : m;  // mx[u] without a runtime index
       m = block_max(m, red);
       const float delta = __fdiv_rn(m, 127.0f);
       const float rcp = m > 0.0f ? __frcp_rn(delta) : 0.0f;
@@ -655,7 +759,7 @@ __global__ void __launch_bounds__(kRotSmemThreads)
       for (int v = threadIdx.x; v < (int)nvec; v += blockDim.x) {
         float val[V];
 #pragma unroll
-        for (int e = 0; e < V; ++e) val[e] = buf[v * V + e];
+        for (int e = 0; e < V; ++e) val[e] = buf[rot_slot(v * V + e)];
         if constexpr (V == 8) {
           *reinterpret_cast<uint2 *>(qrow + v * V) = codes8(val, delta, rcp);
         } else {
@@ -674,7 +778,7 @@ cudaError_t rot_quant_t(const void *x, int64_t rows, int64_t cols, int64_t ld, c
   const int64_t nvec = cols / V;
   if (nvec > 4 * kRowMaxThreads) return cudaErrorNotSupported;
   if ((1 << logn) > 32 * V) {  // blocks wider than a warp: the shared-memory kernel
-    const size_t row_bytes = (size_t)cols * sizeof(float);
+    const size_t row_bytes = (size_t)(cols + cols / 32) * sizeof(float);  // padded slots
     const int R = (int)std::max<size_t>(1, std::min<size_t>(4, (200 * 1024) / row_bytes));
     const size_t smem = R * row_bytes;
     if (smem > 200 * 1024) return cudaErrorNotSupported;

@@ -58,7 +58,8 @@ SWEEPS = {
                 + [("layernorm", 2048, 4096, 0, "f16"), ("layernorm", 16384, 4096, 0, "f16")]
                 + [("static", 16384, K, 0, "bf16") for K in (4096, 8192)],
     # butterfly-rotated activation quantization (N = the rotation's block size n)
-    "rot": [("rot", 16384, 4096, n, "bf16") for n in (16, 64, 256, 4096)] + [("rot", 16384, 8192, 256, "bf16")],
+    "rot": [("rot", 16384, 4096, n, "bf16") for n in (16, 64, 256, 1024, 4096)] + [("rot", 16384, 8192, 256, "bf16"),
+                                                                                    ("rot", 16384, 8192, 8192, "bf16")],
     # FP8 (E4M3): activation quantization, weight path, prefill and decode linears
     "fp8": [("act8", 16384, 4096, 0, "bf16"), ("weight8", 0, 8192, 8192, "bf16")]
            + [("linear8", 2048, K, N, "f16") for _, K, N in synth.OPT_6_7B]
