@@ -603,7 +603,8 @@ __global__ void __launch_bounds__(kRowMaxThreads)
 // cs[i][j] with j = ((p >> (i+1)) << i) | (p mod 2^i) for the pair's first
 // position p, are read once for all R rows.  Shared-memory slots are padded
 // by one word per 32 (slot p + p / 32), which spreads the stride-8 accesses
-// of the first pass over all 32 banks.  Persistent over groups of R rows;
+// of the first pass over all 32 banks; the 2^3-stride pass takes its groups
+// in a permuted order for the same effect.  Persistent over groups of R rows;
 // the codes follow as in the other row quantizers.
 __device__ __forceinline__ int rot_slot(int p) { return p + (p >> 5); }
 
@@ -662,7 +663,19 @@ __device__ __forceinline__ void rot_pass(float *rowbuf, int Kp, int nr, int K, i
                                          const float2 *__restrict__ cs, float (&mx)[4]) {
   const int half = n >> 1;
   const int step = i0 >= 5 ? (1 << i0) + (1 << (i0 - 5)) : 0;
-  for (int gi = threadIdx.x; gi < (K >> r); gi += blockDim.x) {
+  // The 2^3-stride pass with groups in order would put lanes 8 apart on the
+  // same banks.  Taking a group's upper index a = gi >> 3 as
+  // 16 (h >> 2) + 4 ((t >> 3) & 3) + (h & 3), h = t >> 5, gives a warp's
+  // lanes a values 4 apart: slot banks b + 2a + 8k then differ across all
+  // 32 lanes (t is the loop index idx, b = idx & 7).  A bijection of
+  // [0, K/8) when K/8 is a multiple of 128.
+  const bool permute = i0 == 3 && r == 3 && ((K >> 3) & 127) == 0;
+  for (int idx = threadIdx.x; idx < (K >> r); idx += blockDim.x) {
+    int gi = idx;
+    if (permute) {
+      const int h = idx >> 5;
+      gi = (idx & 7) | ((((h >> 2) << 4) | (((idx >> 3) & 3) << 2) | (h & 3)) << 3);
+    }
     const int p0 = ((gi >> i0) << (i0 + r)) | (gi & ((1 << i0) - 1));
     float2 t[r][1 << (r - 1)], ts[r][1 << (r - 1)];
     group_angles<r>(cs, half, i0, p0 & (n - 1), t);
