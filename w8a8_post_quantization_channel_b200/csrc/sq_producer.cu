@@ -664,11 +664,11 @@ __device__ __forceinline__ void rot_pass(float *rowbuf, int Kp, int nr, int K, i
   const int half = n >> 1;
   const int step = i0 >= 5 ? (1 << i0) + (1 << (i0 - 5)) : 0;
   // The 2^3-stride pass with groups in order would put lanes 8 apart on the
-  // same banks.  Taking a group's upper index a = gi >> 3 as
-  // 16 (h >> 2) + 4 ((t >> 3) & 3) + (h & 3), h = t >> 5, gives a warp's
-  // lanes a values 4 apart: slot banks b + 2a + 8k then differ across all
-  // 32 lanes (t is the loop index idx, b = idx & 7).  A bijection of
-  // [0, K/8) when K/8 is a multiple of 128.
+  // same banks.  For loop index idx, taking the group gi = b + 8 a with
+  // b = idx & 7, h = idx >> 5 and a = 16 (h >> 2) + 4 ((idx >> 3) & 3) +
+  // (h & 3) gives a warp's lanes a values 4 apart: slot banks b + 2a + 8k
+  // then differ across all 32 lanes.  A bijection of [0, K/8) when K/8 is a
+  // multiple of 128.
   const bool permute = i0 == 3 && r == 3 && ((K >> 3) & 127) == 0;
   for (int idx = threadIdx.x; idx < (K >> r); idx += blockDim.x) {
     int gi = idx;
