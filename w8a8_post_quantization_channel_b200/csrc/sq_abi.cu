@@ -88,6 +88,7 @@ const char *sq_status_string(sq_status s) {
 
 sq_status sq_calib_absmax(const void *x, sq_dtype xt, int64_t T, int64_t K, int64_t ldx, float *amax,
                           sq_stream_t stream) {
+  SQ_TRACE_CALL();
   if (!valid_dtype(xt) || K <= 0 || K % 16 != 0 || K >= kMaxDim || T < 0 || T >= kMaxDim) return SQ_ERR_INVALID_ARG;
   if (!valid_vec(amax)) return SQ_ERR_INVALID_ARG;
   if (ldx < K || (ldx * dsize(xt)) % 16 != 0) return SQ_ERR_INVALID_ARG;
@@ -133,6 +134,7 @@ static sq_status smooth_quant_weight_impl(const void *w, sq_dtype wt, sq_wlayout
 sq_status sq_smooth_quant_weight(const void *w, sq_dtype wt, sq_wlayout layout, int64_t K, int64_t N, int64_t ldw,
                                  const float *amax, float alpha, int8_t *wq, float *w_scale, float *smooth,
                                  float *inv_smooth, sq_stream_t stream) {
+  SQ_TRACE_CALL();
   return smooth_quant_weight_impl(w, wt, layout, K, N, ldw, amax, alpha, wq, w_scale, smooth, inv_smooth,
                                   sq::QFmt::I8, stream);
 }
@@ -140,6 +142,7 @@ sq_status sq_smooth_quant_weight(const void *w, sq_dtype wt, sq_wlayout layout, 
 sq_status sq_smooth_quant_weight_e4m3(const void *w, sq_dtype wt, sq_wlayout layout, int64_t K, int64_t N,
                                       int64_t ldw, const float *amax, float alpha, uint8_t *wq, float *w_scale,
                                       float *smooth, float *inv_smooth, sq_stream_t stream) {
+  SQ_TRACE_CALL();
   return smooth_quant_weight_impl(w, wt, layout, K, N, ldw, amax, alpha, reinterpret_cast<int8_t *>(wq), w_scale,
                                   smooth, inv_smooth, sq::QFmt::E4M3, stream);
 }
@@ -157,6 +160,7 @@ static sq_status quant_act_impl(const void *x, sq_dtype xt, int64_t M, int64_t K
 
 sq_status sq_quant_act(const void *x, sq_dtype xt, int64_t M, int64_t K, int64_t ldx, const float *inv_smooth,
                        int8_t *xq, float *x_scale, sq_stream_t stream) {
+  SQ_TRACE_CALL();
   return quant_act_impl(x, xt, M, K, ldx, inv_smooth, xq, x_scale, sq::QFmt::I8, stream);
 }
 
@@ -175,6 +179,7 @@ static sq_status rot_checks(sq_dtype xt, int64_t K, int64_t n, const float *rot_
 
 sq_status sq_quant_act_rotated(const void *x, sq_dtype xt, int64_t M, int64_t K, int64_t ldx, const float *inv_smooth,
                                int64_t n, const float *rot_cs, int8_t *xq, float *x_scale, sq_stream_t stream) {
+  SQ_TRACE_CALL();
   if (!valid_dtype(xt) || K <= 0 || K % 16 != 0 || K >= kMaxDim || M < 0 || M >= kMaxDim) return SQ_ERR_INVALID_ARG;
   if (ldx < K || (ldx * dsize(xt)) % 16 != 0 || !valid_vec(inv_smooth)) return SQ_ERR_INVALID_ARG;
   int logn = 0;
@@ -189,6 +194,7 @@ sq_status sq_quant_act_rotated(const void *x, sq_dtype xt, int64_t M, int64_t K,
 sq_status sq_smooth_quant_weight_rotated(const void *w, sq_dtype wt, int64_t K, int64_t N, int64_t ldw,
                                          const float *amax, float alpha, int64_t n, const float *rot_cs, int8_t *wq,
                                          float *w_scale, float *smooth, float *inv_smooth, sq_stream_t stream) {
+  SQ_TRACE_CALL();
   if (!valid_dtype(wt) || K <= 0 || N <= 0 || K % 16 != 0 || N % 16 != 0) return SQ_ERR_INVALID_ARG;
   if (!(alpha >= 0.0f && alpha <= 1.0f)) return SQ_ERR_INVALID_ARG;
   if (!valid_matrix(w, wt, N, K, ldw)) return SQ_ERR_INVALID_ARG;
@@ -209,12 +215,14 @@ sq_status sq_smooth_quant_weight_rotated(const void *w, sq_dtype wt, int64_t K, 
 
 sq_status sq_quant_act_e4m3(const void *x, sq_dtype xt, int64_t M, int64_t K, int64_t ldx, const float *inv_smooth,
                             uint8_t *xq, float *x_scale, sq_stream_t stream) {
+  SQ_TRACE_CALL();
   return quant_act_impl(x, xt, M, K, ldx, inv_smooth, reinterpret_cast<int8_t *>(xq), x_scale, sq::QFmt::E4M3,
                         stream);
 }
 
 sq_status sq_fold_smooth_into_norm(const float *gamma, const float *inv_smooth, int64_t K, float *gs,
                                    sq_stream_t stream) {
+  SQ_TRACE_CALL();
   if (K <= 0 || K >= kMaxDim || !valid_vec(gamma) || !valid_vec(inv_smooth) || !valid_vec(gs))
     return SQ_ERR_INVALID_ARG;
   return from_cuda(sq::launch_fold_norm_weight(gamma, inv_smooth, K, gs, (cudaStream_t)stream));
@@ -222,6 +230,7 @@ sq_status sq_fold_smooth_into_norm(const float *gamma, const float *inv_smooth, 
 
 sq_status sq_rmsnorm_quant_act(const void *x, sq_dtype xt, int64_t M, int64_t K, int64_t ldx, const float *gs,
                                float eps, int8_t *xq, float *x_scale, sq_stream_t stream) {
+  SQ_TRACE_CALL();
   if (!valid_dtype(xt) || K <= 0 || K % 16 != 0 || K >= kMaxDim || M < 0 || M >= kMaxDim) return SQ_ERR_INVALID_ARG;
   if (ldx < K || (ldx * dsize(xt)) % 16 != 0) return SQ_ERR_INVALID_ARG;
   if (!(eps >= 0.0f) || eps > 3.0e38f) return SQ_ERR_INVALID_ARG;  // rejects NaN and infinity too
@@ -234,6 +243,7 @@ sq_status sq_rmsnorm_quant_act(const void *x, sq_dtype xt, int64_t M, int64_t K,
 
 sq_status sq_layernorm_quant_act(const void *x, sq_dtype xt, int64_t M, int64_t K, int64_t ldx, const float *gs,
                                  const float *bs, float eps, int8_t *xq, float *x_scale, sq_stream_t stream) {
+  SQ_TRACE_CALL();
   if (!valid_dtype(xt) || K <= 0 || K % 16 != 0 || K >= kMaxDim || M < 0 || M >= kMaxDim) return SQ_ERR_INVALID_ARG;
   if (ldx < K || (ldx * dsize(xt)) % 16 != 0) return SQ_ERR_INVALID_ARG;
   if (!(eps > 0.0f) || eps > 3.0e38f) return SQ_ERR_INVALID_ARG;  // rejects NaN and infinity too
@@ -246,6 +256,7 @@ sq_status sq_layernorm_quant_act(const void *x, sq_dtype xt, int64_t M, int64_t 
 
 sq_status sq_static_act_scale(const float *amax, const float *inv_smooth, int64_t K, float *delta,
                               sq_stream_t stream) {
+  SQ_TRACE_CALL();
   if (K <= 0 || K >= kMaxDim || !valid_vec(amax) || !valid_vec(inv_smooth)) return SQ_ERR_INVALID_ARG;
   if (delta == nullptr || (reinterpret_cast<uintptr_t>(delta) & 3u) != 0) return SQ_ERR_INVALID_ARG;
   return from_cuda(sq::launch_static_scale(amax, inv_smooth, K, delta, (cudaStream_t)stream));
@@ -253,6 +264,7 @@ sq_status sq_static_act_scale(const float *amax, const float *inv_smooth, int64_
 
 sq_status sq_quant_act_static(const void *x, sq_dtype xt, int64_t M, int64_t K, int64_t ldx, const float *inv_smooth,
                               const float *delta, int8_t *xq, float *x_scale, sq_stream_t stream) {
+  SQ_TRACE_CALL();
   if (!valid_dtype(xt) || K <= 0 || K % 16 != 0 || K >= kMaxDim || M < 0 || M >= kMaxDim) return SQ_ERR_INVALID_ARG;
   if (ldx < K || (ldx * dsize(xt)) % 16 != 0) return SQ_ERR_INVALID_ARG;
   if (!valid_vec(inv_smooth) || delta == nullptr || (reinterpret_cast<uintptr_t>(delta) & 3u) != 0)
@@ -301,6 +313,7 @@ static sq_status accumulate_impl(const int8_t *xq, const int8_t *wq, int64_t M, 
 sq_status sq_w8a8_linear(const int8_t *xq, const float *x_scale, const int8_t *wq, const float *w_scale, int64_t M,
                          int64_t N, int64_t K, void *y, sq_dtype yt, int64_t ldy, void *workspace,
                          size_t workspace_bytes, sq_stream_t stream) {
+  SQ_TRACE_CALL();
   return linear_impl(xq, x_scale, wq, w_scale, M, N, K, y, yt, ldy, workspace, workspace_bytes, sq::QFmt::I8,
                      stream);
 }
@@ -308,6 +321,7 @@ sq_status sq_w8a8_linear(const int8_t *xq, const float *x_scale, const int8_t *w
 sq_status sq_w8a8_linear_e4m3(const uint8_t *xq, const float *x_scale, const uint8_t *wq, const float *w_scale,
                               int64_t M, int64_t N, int64_t K, void *y, sq_dtype yt, int64_t ldy, void *workspace,
                               size_t workspace_bytes, sq_stream_t stream) {
+  SQ_TRACE_CALL();
   return linear_impl(reinterpret_cast<const int8_t *>(xq), x_scale, reinterpret_cast<const int8_t *>(wq), w_scale,
                      M, N, K, y, yt, ldy, workspace, workspace_bytes, sq::QFmt::E4M3, stream);
 }
@@ -315,6 +329,7 @@ sq_status sq_w8a8_linear_e4m3(const uint8_t *xq, const float *x_scale, const uin
 sq_status sq_w8a8_linear_scatter(const int8_t *xq, const float *x_scale, const int8_t *wq, const float *w_scale,
                                  int64_t M, int64_t N, int64_t K, void *const *y_dst, int n_dst, sq_dtype yt,
                                  int64_t ldy, void *workspace, size_t workspace_bytes, sq_stream_t stream) {
+  SQ_TRACE_CALL();
   if (!valid_dtype(yt) || !valid_vec(w_scale)) return SQ_ERR_INVALID_ARG;
   if (y_dst == nullptr || n_dst < 1 || n_dst > sq::kMaxDest) return SQ_ERR_INVALID_ARG;
   sq::YDest dst{};
@@ -338,21 +353,25 @@ size_t sq_w8a8_linear_workspace_size(int64_t M, int64_t N, int64_t K) {
 
 sq_status sq_w8a8_accumulate(const int8_t *xq, const int8_t *wq, int64_t M, int64_t N, int64_t K, int32_t *acc,
                              int64_t ldacc, void *workspace, size_t workspace_bytes, sq_stream_t stream) {
+  SQ_TRACE_CALL();
   return accumulate_impl(xq, wq, M, N, K, acc, ldacc, workspace, workspace_bytes, sq::QFmt::I8, stream);
 }
 
 sq_status sq_w8a8_accumulate_e4m3(const uint8_t *xq, const uint8_t *wq, int64_t M, int64_t N, int64_t K, float *acc,
                                   int64_t ldacc, void *workspace, size_t workspace_bytes, sq_stream_t stream) {
+  SQ_TRACE_CALL();
   return accumulate_impl(reinterpret_cast<const int8_t *>(xq), reinterpret_cast<const int8_t *>(wq), M, N, K, acc,
                          ldacc, workspace, workspace_bytes, sq::QFmt::E4M3, stream);
 }
 
 sq_status sq_selftest_wait_timeout(int limit_ms, sq_stream_t stream) {
+  SQ_TRACE_CALL();
   if (limit_ms < 1 || limit_ms > 5000) return SQ_ERR_INVALID_ARG;
   return from_cuda(sq::launch_wait_timeout_selftest((unsigned long long)limit_ms * 1000000ull, (cudaStream_t)stream));
 }
 
 sq_status sq_check_device_error(sq_stream_t stream) {
+  SQ_TRACE_CALL();
   if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return SQ_ERR_CUDA;
   unsigned *word = sq::device_error_word();
   if (word == nullptr) return SQ_ERR_CUDA;

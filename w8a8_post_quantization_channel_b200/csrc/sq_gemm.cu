@@ -1209,6 +1209,7 @@ bool is_aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u)
 extern "C" sq_status sq_w8a8_linear_decode_noalloc(const int8_t *xq, const float *x_scale, const int8_t *wq,
                                                    const float *w_scale, int64_t M, int64_t N, int64_t K, void *y,
                                                    sq_dtype yt, int64_t ldy, sq_stream_t stream) {
+  SQ_TRACE_CALL();
   if (yt != SQ_F32 && yt != SQ_F16 && yt != SQ_BF16) return SQ_ERR_INVALID_ARG;
   const int64_t ysize = yt == SQ_F32 ? 4 : 2;
   if (M < 0 || N <= 0 || K <= 0 || N % 16 != 0 || K % 16 != 0 || N >= ((int64_t)1 << 31) ||

@@ -2,12 +2,25 @@
 #pragma once
 
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 #include <stddef.h>
 #include <stdint.h>
 
 #include "sq.h"
 
 namespace sq {
+
+// An NVTX range named after the ABI call, open for the call's host-side
+// duration (validation and launches), so a profiler's timeline shows which
+// call enqueued which kernels.  Without a profiler attached NVTX calls
+// return at once and allocate nothing.
+struct TraceRange {
+  explicit TraceRange(const char *name) { nvtxRangePushA(name); }
+  ~TraceRange() { nvtxRangePop(); }
+  TraceRange(const TraceRange &) = delete;
+  TraceRange &operator=(const TraceRange &) = delete;
+};
+#define SQ_TRACE_CALL() const sq::TraceRange sq_trace_range_(__func__)
 
 // Number of SMs of the current device (cached per device).
 int num_sms();
