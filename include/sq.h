@@ -155,10 +155,11 @@ sq_status sq_rmsnorm_quant_act(const void *x, sq_dtype xt, int64_t M, int64_t K,
  * (sq_fold_smooth_into_norm computes either product), then per token
  *   mu_t  = sum_j x_tj / K
  *   var_t = sum_j (x_tj - mu_t)^2 / K
- *          (both in double precision, within 2^-34 relative of their exact
- *          values: this library takes one pass over the deviations from
- *          the token's first value, in an unspecified order; mu_t and
- *          r_t = 1 / sqrt(var_t + eps) each rounded once to fp32)
+ *          (both in double precision: this library takes one pass over
+ *          the deviations from the token's first value, in an unspecified
+ *          order, which keeps var_t within 2^-31 (relative) and mu_t within
+ *          2^-40 standard deviations of their exact values for K <= 16384;
+ *          mu_t and r_t = 1 / sqrt(var_t + eps) each rounded once to fp32)
  *   n_tj  = (x_tj - mu_t) * r_t              (fp32, in that order)
  *   v_tj  = fma(n_tj, gs_j, bs_j)            (one rounding)
  *   then per-token quantization of v exactly as sq_quant_act.

@@ -175,9 +175,10 @@ __global__ void __launch_bounds__(kRowMaxThreads)
       // One pass over the deviations d = x - c from the row's first value
       // c: with S = sum d and Q = sum d^2, mu = c + S/K and
       // var = Q/K - (S/K)^2.  As c is one of the row's values,
-      // (mu - c)^2 <= K var, so the subtraction loses at most log2(K + 1)
-      // bits of the double's 53: var and r stay within 2^-34 (relative) of
-      // the two-pass values, far inside one fp32 ulp.
+      // (mu - c)^2 <= K var, so Q/K <= (K + 1) var: with about 44 rounding
+      // steps per term in each double sum, var stays within ~132 (K + 1)
+      // 2^-53 (relative; 2^-31 at K = 16384) of its exact value and mu
+      // within 2^-40 standard deviations, far inside one fp32 ulp of r.
       double sh = 0.0, q = 0.0;
 #pragma unroll
       for (int i = 0; i < kVPT; ++i)
