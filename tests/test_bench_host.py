@@ -1,6 +1,7 @@
-"""Host-side logic of bench.py, without a GPU: the source-text hash that ties
-the ncu traffic figure to the kernel it was measured on, and the parsing of
-the nvidia-smi clock samples."""
+"""Host-side logic of bench.py and profile_case.py, without a GPU: the
+source-text hash that ties the ncu traffic figure to the kernel it was
+measured on, the parsing of the nvidia-smi clock samples, the algorithmic
+bytes and ops per row, and the sweep definitions."""
 import importlib.util
 import os
 import sys
@@ -60,3 +61,31 @@ def test_clock_summary_keeps_this_gpu_and_collects_reasons():
     assert s["samples"] == 2 and s["sm_mhz"] == 1932.5 and s["sm_max_mhz"] == 1965.0
     assert s["reasons"] == ["sw_power_cap"]
     assert b.ClockSampler(None).summary()["samples"] == 0
+
+
+def test_row_work_counts_the_algorithmic_bytes():
+    # one OPT-shaped linear: the per-row bytes and ops the bench divides by
+    b = _bench()
+
+    class L:
+        M, K, N = 2048, 4096, 12288
+        calib = type("T", (), {"shape": (65536, 4096)})()
+
+    w = b.row_work([L])
+    assert w["calib"] == 65536 * 4096 * 2 + 8 * 4096
+    assert w["weight"] == 2 * 12288 * 4096 * 2 + 12288 * 4096 + 4 * 12288 + 16 * 4096  # 2 reads + int8 write
+    assert w["act"] == 2048 * 4096 * 3 + 4 * 2048 + 4 * 4096  # 2 B read + 1 B write per element
+    assert w["linear_ops"] == 2 * 2048 * 12288 * 4096
+
+
+def test_profile_sweeps_name_known_ops():
+    from w8a8_post_quantization_channel_b200 import profile_case as pc
+    known = {"calib", "weight", "act", "linear", "rmsnorm", "layernorm", "static", "act8", "weight8", "linear8",
+             "rot"}
+    for name, cases in pc.SWEEPS.items():
+        assert cases, name
+        for op, M, K, N, dt in cases:
+            assert op in known, (name, op)
+            assert dt in pc.DT and K % 16 == 0, (name, op, K, dt)
+            if op == "rot":
+                assert N & (N - 1) == 0 and K % N == 0, (name, K, N)
