@@ -197,3 +197,39 @@ def test_static_scale_and_quantization(dt, K):
     np.testing.assert_array_equal(xs.cpu().numpy(), xs_ref)
     assert (np.abs(xq_ref[7]) == 127).sum() > 0
     assert sq.sq_check_device_error() == sq.SQ_OK
+
+
+@pytest.mark.parametrize("dt", ["bf16", "f32"])
+def test_producers_on_strided_rows(dt):
+    # rows K = 1024 wide inside a buffer with leading dimension K + 64: every
+    # producer reads only its row's K values
+    M, K = 19, 1024
+    base = synth.activations(M, K + 64, synth.outliers(K + 64, frac=0.01, mult=40.0, seed=5), seed=6,
+                             dtype=TORCH_DT[dt])
+    base[:, K:] = 1.0e4  # beyond the row: would dominate every maximum if read
+    x = base.to(DEV)[:, :K]
+    xf = f32(base[:, :K])
+    g = synth.gen(7)
+    gamma = torch.rand(K, generator=g) + 0.5
+    beta = torch.rand(K, generator=g) - 0.5
+    inv_s = torch.exp(torch.randn(K, generator=g) * 0.5)
+    gs = oracle.fold_norm_weight(gamma.numpy(), inv_s.numpy())
+    bs = oracle.fold_norm_weight(beta.numpy(), inv_s.numpy())
+    eps = 1e-5
+    xq, xs = sq.sq_rmsnorm_quant_act(x, torch.from_numpy(gs).to(DEV), eps)
+    xq_ref, xs_ref = oracle.rmsnorm_quant_act(xf, gs, eps)
+    diff = xq.cpu().numpy().astype(np.int32) - xq_ref
+    assert np.abs(diff).max() <= 1 and np.all(diff[~_boundary_mask(xf, gs, eps)] == 0)
+    assert np.all(np.abs(xs.cpu().numpy().astype(np.float64) - xs_ref) <= 2 * np.spacing(xs_ref))
+    xq, xs = sq.sq_layernorm_quant_act(x, torch.from_numpy(gs).to(DEV), torch.from_numpy(bs).to(DEV), eps)
+    xq_ref, xs_ref = oracle.layernorm_quant_act(xf, gs, bs, eps)
+    diff = xq.cpu().numpy().astype(np.int32) - xq_ref
+    assert np.abs(diff).max() <= 1 and np.all(diff[~_ln_boundary_mask(xf, gs, bs, eps)] == 0)
+    assert np.all(np.abs(xs.cpu().numpy().astype(np.float64) - xs_ref) <= 2 * np.spacing(xs_ref))
+    amax = oracle.calib_absmax(xf)
+    delta = sq.sq_static_act_scale(torch.from_numpy(amax).to(DEV), inv_s.to(DEV))
+    xq, xs = sq.sq_quant_act_static(x, inv_s.to(DEV), delta)
+    xq_ref, xs_ref = oracle.quant_act_static(xf, inv_s.numpy(), oracle.static_act_scale(amax, inv_s.numpy()))
+    np.testing.assert_array_equal(xq.cpu().numpy(), xq_ref)
+    np.testing.assert_array_equal(xs.cpu().numpy(), xs_ref)
+    assert sq.sq_check_device_error() == sq.SQ_OK

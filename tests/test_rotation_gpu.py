@@ -102,3 +102,19 @@ def test_rotated_linear_matches_the_unrotated_product():
     exact = f32(x).astype(np.float64) @ f32(w).astype(np.float64).T
     err = np.abs(y - exact).max() / np.abs(exact).max()
     assert err < 0.02, err
+
+
+@pytest.mark.parametrize("n", [64, 1024])
+def test_quant_act_rotated_strided_rows(n):
+    # rows K wide inside a buffer with leading dimension K + 64
+    M, K = 13, 2048
+    base = synth.activations(M, K + 64, synth.outliers(K + 64, frac=0.01, mult=40.0, seed=8), seed=9,
+                             dtype=torch.bfloat16)
+    base[:, K:] = 1.0e4  # beyond the row: would dominate every maximum if read
+    inv = torch.exp(torch.randn(K, generator=synth.gen(10)) * 0.5)
+    c, s, cs = _table(n, n + 3)
+    xq, xs = sq.sq_quant_act_rotated(base.to(DEV)[:, :K], inv.to(DEV), n, cs)
+    xq_ref, xs_ref = oracle.quant_act_rotated(f32(base[:, :K]), inv.numpy(), n, c, s)
+    np.testing.assert_array_equal(xs.cpu().numpy(), xs_ref)
+    np.testing.assert_array_equal(xq.cpu().numpy(), xq_ref)
+
