@@ -381,6 +381,20 @@ def test_output_rounding_matches_library_conversions():
 # upstream producer: RMSNorm folded with X diag(s)^-1, and the static scale
 # ---------------------------------------------------------------------------
 
+def test_p11_rmsnorm_worked_example():
+    g = load("p11_rmsnorm.txt")
+    x = _fl(g["x"]).astype(np.float32)[None, :]
+    eps = float(g["eps"][0])
+    r = oracle.rmsnorm_factor(x, eps)
+    assert r[0] == np.float32(1.0 / float(g["r_inv"][0]))
+    for case in ("a", "b"):
+        gs = _fl(g["gs_" + case]).astype(np.float32)
+        xq, dx = oracle.rmsnorm_quant_act(x, gs, eps)
+        np.testing.assert_array_equal(xq[0], _int(g["xq_" + case]))
+        v = ((x[0] * r[0]).astype(np.float32) * gs).astype(np.float32)
+        assert dx[0] == np.float32(np.abs(v).max() / np.float32(127))
+
+
 def test_rmsnorm_factor_matches_library_rms_norm():
     rng = np.random.default_rng(21)
     x = rng.standard_normal((9, 320)).astype(np.float32)
