@@ -478,7 +478,9 @@ def bench_reference(args, rank, world):
     return {"impl": "reference", "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "i8", "data": "synthetic",
-            "config": {"workload": WORKLOAD, "global_batch": 2048, "seq_len": None, "parallelism": "dp1"},
+            # the same workload description as this bench's own arm at this N
+            "config": {"workload": WORKLOAD, "global_batch": 2048 * world, "seq_len": None,
+                       "parallelism": f"dp{world}"},
             "cpu_baseline": {"value": value, "unit": "TOPS", "cores": 1, "kind": "oracle", "sample": desc},
             "e2e": {"value": value, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
