@@ -11,7 +11,6 @@ mathematics fix, never against the oracle itself.
 - the defining property of round-to-nearest quantization on a uniform grid;
 - brute-force integer matrix products and library reductions/conversions.
 """
-from decimal import Decimal, getcontext
 from fractions import Fraction
 
 import numpy as np
@@ -21,7 +20,6 @@ import torch
 import oracle
 from tests.golden.load import load
 
-getcontext().prec = 40
 KN, NK = oracle.LAYOUT_KN, oracle.LAYOUT_NK
 F32_EPS = float(np.finfo(np.float32).eps)  # 2^-23
 
