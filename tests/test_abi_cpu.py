@@ -169,6 +169,37 @@ def test_linear_argument_checks():
     assert acc(A16, A16, 4, 256, 256, A16, 100, None, 0, None) == INV
 
 
+def test_fp8_argument_checks():
+    L = sq.lib()
+    qa = L.sq_quant_act_e4m3
+    assert qa(None, sq.SQ_BF16, 0, 256, 256, A16, None, None, None) == sq.SQ_OK     # M == 0: no-op
+    assert qa(A16, sq.SQ_BF16, 8, 256, 256, None, A16, A16, None) == INV            # null inv_s
+    assert qa(A16, sq.SQ_BF16, 8, 24, 24, A16, A16, A16, None) == INV               # K % 16
+    w = L.sq_smooth_quant_weight_e4m3
+    assert w(A16, sq.SQ_F16, sq.SQ_W_NK, 256, 512, 256, A16, ctypes.c_float(2.0), A16, A16, A16, A16, None) == INV
+    assert w(A16, sq.SQ_F16, sq.SQ_W_NK, 256, 512, 256, None, ctypes.c_float(0.5), A16, A16, A16, A16, None) == INV
+    lin = L.sq_w8a8_linear_e4m3
+    assert lin(A16, A16, A16, A16, 0, 256, 256, A16, sq.SQ_BF16, 256, None, 0, None) == sq.SQ_OK
+    assert lin(A16, A16, A16, A16, 64, 40, 256, A16, sq.SQ_BF16, 256, None, 0, None) == INV   # N % 16
+    assert lin(None, A16, A16, A16, 64, 256, 256, A16, sq.SQ_BF16, 256, None, 0, None) == INV
+    acc = L.sq_w8a8_accumulate_e4m3
+    assert acc(A16, A16, 4, 256, 256, A16, 100, None, 0, None) == INV                  # ldacc < N
+
+
+def test_decode_noalloc_and_selftest_argument_checks():
+    L = sq.lib()
+    f = L.sq_w8a8_linear_decode_noalloc
+    assert f(A16, A16, A16, A16, 0, 256, 256, A16, sq.SQ_BF16, 256, None) == sq.SQ_OK   # M == 0: no-op
+    assert f(A16, A16, A16, A16, 65, 256, 256, A16, sq.SQ_BF16, 256, None) == sq.SQ_ERR_UNSUPPORTED
+    assert f(A16, A16, A16, A16, 8, 256, 256, A16, 9, 256, None) == INV                 # output dtype
+    assert f(A16, A16, A16, A16, 8, 256, 256, A16, sq.SQ_BF16, 128, None) == INV        # ldy < N
+    assert f(A16, A16, None, A16, 8, 256, 256, A16, sq.SQ_BF16, 256, None) == INV       # null wq
+    assert f(A16, A16, A16, A16, 8, 256, 256, MIS, sq.SQ_BF16, 256, None) == INV        # misaligned y
+    t = L.sq_selftest_wait_timeout
+    assert t(0, None) == INV
+    assert t(6000, None) == INV
+
+
 def test_workspace_size_is_defined_for_all_shapes():
     for M in (0, 1, 8, 64, 128, 2048):
         for N, K in ((256, 256), (4096, 4096), (28672, 8192)):
