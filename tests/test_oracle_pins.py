@@ -36,17 +36,6 @@ def _int(rows):
     return np.array([int(v) for v in rows], np.int64)
 
 
-def _round_f32(fr: Fraction) -> np.float32:
-    """The fp32 nearest to the rational fr, ties to even."""
-    f = np.float32(float(fr))
-    best = f
-    for c in (np.nextafter(f, np.float32(-np.inf)), np.nextafter(f, np.float32(np.inf))):
-        d_c, d_b = abs(Fraction(float(c)) - fr), abs(Fraction(float(best)) - fr)
-        if d_c < d_b or (d_c == d_b and (int(c.view(np.uint32)) & 1) == 0):
-            best = c
-    return best
-
-
 def _ulps(got, exact):
     """Distance of fp32 'got' from the exact value, in fp32 ulps of exact."""
     got = np.asarray(got, np.float64)
@@ -579,8 +568,9 @@ def test_folded_layernorm_equals_norm_then_smoothing():
     n = ((x - mu[:, None]).astype(np.float32) * r[:, None]).astype(np.float32)
     # the affine step n * gamma + beta, taken exactly in rationals and
     # rounded once to fp32
-    normed = np.array([[_round_f32(Fraction(float(n[t, j])) * Fraction(float(gamma[j])) + Fraction(float(beta[j])))
-                        for j in range(K)] for t in range(n.shape[0])], np.float32)
+    normed = np.array([[float(_fp32_round(Fraction(float(n[t, j])) * Fraction(float(gamma[j]))
+                                          + Fraction(float(beta[j])))) for j in range(K)]
+                       for t in range(n.shape[0])], np.float32)
     xq_u, dx_u = oracle.quant_act(normed, inv_s)
     np.testing.assert_array_equal(xq, xq_u)
     np.testing.assert_array_equal(dx, dx_u)
