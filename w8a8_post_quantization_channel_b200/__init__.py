@@ -59,6 +59,7 @@ class SqError(RuntimeError):
 
 
 def library_path() -> str:
+    """Path of the in-tree libsq.so this binding loads."""
     return _LIB_PATH
 
 
@@ -118,6 +119,7 @@ def header_functions() -> list[str]:
 
 
 def sq_status_string(status: int) -> str:
+    """The library's description of a status code."""
     return lib().sq_status_string(int(status)).decode()
 
 
@@ -267,6 +269,7 @@ def sq_quant_act_static(x: torch.Tensor, inv_smooth: torch.Tensor, delta: torch.
 
 
 def sq_w8a8_linear_workspace_size(M: int, N: int, K: int) -> int:
+    """Workspace bytes sq_w8a8_linear needs for this shape (0 outside decode shapes)."""
     return int(lib().sq_w8a8_linear_workspace_size(M, N, K))
 
 
