@@ -75,6 +75,7 @@ def _load():
             "or_rmsnorm_factor": ([f32p, i64, i64, ctypes.c_float, f32p], None),
             "or_layernorm_quant_act": ([f32p, i64, i64, f32p, f32p, ctypes.c_float, i8p, f32p], None),
             "or_layernorm_stats": ([f32p, i64, i64, ctypes.c_float, f32p, f32p], None),
+            "or_layernorm_values": ([f32p, i64, i64, f32p, f32p, ctypes.c_float, f32p], None),
             "or_static_act_scale": ([f32p, f32p, i64], ctypes.c_float),
             "or_quant_act_static": ([f32p, i64, i64, f32p, ctypes.c_float, i8p, f32p], None),
             "or_e4m3_decode": ([ctypes.c_uint8], ctypes.c_float),
@@ -284,6 +285,19 @@ def layernorm_stats(x, eps: float):
     _load().or_layernorm_stats(_ptr(x, ctypes.c_float), M, K, ctypes.c_float(eps), _ptr(mu, ctypes.c_float),
                                _ptr(r, ctypes.c_float))
     return mu, r
+
+
+def layernorm_values(x, gs, bs, eps: float) -> np.ndarray:
+    """The folded LayerNorm values v [M,K] that layernorm_quant_act quantizes."""
+    x = _f32(x)
+    gs = _f32(gs)
+    M, K = x.shape
+    v = np.zeros((M, K), np.float32)
+    bp = None if bs is None else _f32(bs)
+    _load().or_layernorm_values(_ptr(x, ctypes.c_float), M, K, _ptr(gs, ctypes.c_float),
+                                None if bp is None else _ptr(bp, ctypes.c_float), ctypes.c_float(eps),
+                                _ptr(v, ctypes.c_float))
+    return v
 
 
 def static_act_scale(amax, inv_s) -> float:

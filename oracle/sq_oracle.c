@@ -312,6 +312,19 @@ static float or_layernorm_value(float x, float muf, float r, float g, float b) {
   return fmaf(n, g, b); /* the affine step n * g + b, rounded once */
 }
 
+/* The normalised, folded values v_tj of or_layernorm_quant_act before
+ * quantization (exposed so tests can see how close v / delta lies to a
+ * rounding boundary). */
+void or_layernorm_values(const float *x, int64_t M, int64_t K, const float *gs, const float *bs, float eps,
+                         float *v) {
+  for (int64_t t = 0; t < M; ++t) {
+    const float *row = x + t * K;
+    float muf, r;
+    or_layernorm_row_stats(row, K, eps, &muf, &r);
+    for (int64_t j = 0; j < K; ++j) v[t * K + j] = or_layernorm_value(row[j], muf, r, gs[j], bs ? bs[j] : 0.0f);
+  }
+}
+
 void or_layernorm_quant_act(const float *x, int64_t M, int64_t K, const float *gs, const float *bs, float eps,
                             int8_t *xq, float *dx) {
   for (int64_t t = 0; t < M; ++t) {

@@ -175,6 +175,56 @@ def test_smooth_factor_floor_on_empty_channels():
     np.testing.assert_allclose(s, np.sqrt([1e-5 / 0.2, 3.0 / 1e-5, 1.0]), rtol=1e-6)
 
 
+def _alternative_sequences(alpha, a, w):
+    """Other plausible fp32 evaluations of a^alpha / w^(1-alpha) (numpy fp32:
+    IEEE-correct sqrt, product and division)."""
+    f = np.float32
+    sq = lambda v: f(np.sqrt(f(v)))  # noqa: E731
+    once = f(np.float64(a) ** alpha / np.float64(w) ** (1.0 - alpha))
+    if alpha == 0.5:
+        return [sq(f(a / w)), f(sq(a) * f(f(1) / sq(w))), once]
+    if alpha == 0.25:
+        w3 = f(f(w * w) * w)
+        return [sq(sq(f(a / w3))), f(sq(sq(a)) / sq(sq(w3))), f(sq(sq(a)) / sq(f(w * sq(w)))), once]
+    a3 = f(f(a * a) * a)
+    return [sq(sq(f(a3 / w))), f(sq(sq(a3)) / sq(sq(w))), once]
+
+
+def _reciprocal_formula(alpha, a, w):
+    """inv_s as w^(1-alpha) / a^alpha by the mirrored sqrt sequence, in place of 1/s."""
+    f = np.float32
+    sq = lambda v: f(np.sqrt(f(v)))  # noqa: E731
+    if alpha == 0.5:
+        return f(sq(w) / sq(a))
+    if alpha == 0.25:
+        return f(f(sq(w) * sq(sq(w))) / sq(sq(a)))
+    return f(sq(sq(w)) / f(sq(a) * sq(sq(a))))
+
+
+def test_p12_smooth_factor_fp32_sequence():
+    """s and 1/s bit for bit against the hand-derived table
+    (tests/golden/p12_smooth_factor_sequences.txt: the reading's sequence of
+    square roots, one product and one division, worked in exact rationals).
+    Each case also shows that the alternative sequences give a different
+    float, so an oracle that evaluated the power another way fails here.
+    (inv_s computed in double and rounded to fp32 is not a distinct
+    alternative: double rounding of a quotient of fp32 values is innocuous,
+    53 >= 2*24 + 2, so it equals the fp32 division on every input.)"""
+    g = load("p12_smooth_factor_sequences.txt")
+    assert len(g) == 11
+    for key in sorted(g):
+        alpha, ah, wh, sh, ih = g[key]
+        alpha = float(alpha)
+        a, w = np.float32(float.fromhex(ah)), np.float32(float.fromhex(wh))
+        s, inv = oracle.smooth_factor(np.array([a]), np.array([w]), alpha)
+        assert s[0] == np.float32(float.fromhex(sh)), key
+        assert inv[0] == np.float32(float.fromhex(ih)), key
+        if alpha in (0.25, 0.5, 0.75):
+            for alt in _alternative_sequences(alpha, a, w):
+                assert alt != s[0], key
+            assert _reciprocal_formula(alpha, a, w) != inv[0], key
+
+
 # ---------------------------------------------------------------------------
 # reductions against library routines
 # ---------------------------------------------------------------------------
@@ -336,18 +386,48 @@ def test_dequant_exact_on_power_of_two_scales():
     np.testing.assert_array_equal(y, acc.astype(np.float64) * dx[:, None] * dw[None, :])
 
 
+# (acc, dx, dw) triples where the three ways of forming acc * dx * dw in fp32
+# give three different floats: ((float)acc * dx) * dw (the reading),
+# (float)acc * (dx * dw), and the exact product rounded once (an fma or a
+# double-precision product).  Found by a random search over the configs'
+# scale ranges; the expected values are worked below in exact rationals.
+DEQUANT_ORDER_CASES = [
+    (205907, 0.0008812682353891432, 0.019935712218284607),
+    (58144, 0.004028223920613527, 0.015843471512198448),
+    (-219780, 0.004683542996644974, 0.000896687270142138),
+    (-46418, 0.0029101360123604536, 0.013552580028772354),
+]
+
+
 def test_dequant_order_of_rounding():
-    # (float)acc * dx is rounded before * dw: values chosen so the two
-    # groupings differ in fp32
-    acc = np.array([[16777217]], np.int32)  # 2^24 + 1 -> rounds to 2^24 (even)
-    dx = np.array([1.0], np.float32)
-    dw = np.array([1.0], np.float32)
-    assert oracle.dequant(acc, dx, dw)[0, 0] == np.float32(16777216.0)
-    acc = np.array([[3]], np.int32)
-    dx = np.array([np.float32(1.0) / np.float32(3.0)], np.float32)
-    dw = np.array([3.0], np.float32)
-    left = (np.float32(3.0) * dx[0]) * np.float32(3.0)
-    assert oracle.dequant(acc, dx, dw)[0, 0] == left
+    """y = ((float)acc * dx) * dw: each product rounded to fp32 in that order
+    (the reading of the epilogue; the page states only Y = X~ W~).  The
+    expected values are worked in exact rational arithmetic with explicit
+    round-to-nearest-even, and the test checks that the other groupings give
+    a different float on every case, so a re-grouped oracle fails here."""
+    # (float)acc rounds to nearest even beyond 2^24
+    for acc, want in ((16777217, 16777216.0), (16777219, 16777220.0), (-16777221, -16777220.0)):
+        y = oracle.dequant(np.array([[acc]], np.int32), np.ones(1, np.float32), np.ones(1, np.float32))
+        assert y[0, 0] == np.float32(want)
+    for acc, dx, dw in DEQUANT_ORDER_CASES:
+        dx32, dw32 = np.float32(dx), np.float32(dw)
+        A, DX, DW = _fp32_round(Fraction(acc)), Fraction(float(dx32)), Fraction(float(dw32))
+        reading = _fp32_round(_fp32_round(A * DX) * DW)
+        regrouped = _fp32_round(A * _fp32_round(DX * DW))
+        once = _fp32_round(Fraction(acc) * DX * DW)
+        assert len({reading, regrouped, once}) == 3
+        y = oracle.dequant(np.array([[acc]], np.int32), np.array([dx32]), np.array([dw32]))
+        assert Fraction(float(y[0, 0])) == reading
+    # the same cases as one [M, N] call: row t takes dx[t], column n takes dw[n]
+    accs = np.array([[c[0] for c in DEQUANT_ORDER_CASES]], np.int32).repeat(2, 0)
+    dxs = np.array([DEQUANT_ORDER_CASES[0][1], 1.0], np.float32)
+    dws = np.array([c[2] for c in DEQUANT_ORDER_CASES], np.float32)
+    y = oracle.dequant(accs, dxs, dws)
+    for t in range(2):
+        for n in range(len(DEQUANT_ORDER_CASES)):
+            want = _fp32_round(_fp32_round(_fp32_round(Fraction(int(accs[t, n]))) * Fraction(float(dxs[t])))
+                               * Fraction(float(dws[n])))
+            assert Fraction(float(y[t, n])) == want
 
 
 def test_output_rounding_matches_library_conversions():
@@ -439,6 +519,22 @@ def test_folded_norm_equals_norm_then_smoothing():
     np.testing.assert_array_equal(xq, xq_u)
     np.testing.assert_array_equal(dx, dx_u)
     assert not np.array_equal(xq, oracle.rmsnorm_quant_act(x, oracle.fold_norm_weight(gamma, 1 / inv_s), eps)[0])
+
+
+def test_fold_is_one_fp32_product():
+    """gs_j = fl(gamma_j * inv_s_j): the fold multiplies the stored
+    reciprocal, as diag(s)^-1 is applied to X (a single fp32 product, worked
+    here in exact rationals).  On these inputs dividing by s, or by the
+    re-inverted 1/inv_s, gives a different float for some channel."""
+    rng = np.random.default_rng(31)
+    gamma = rng.uniform(0.2, 3.0, 256).astype(np.float32)
+    inv_s = np.exp(rng.uniform(-4, 4, 256)).astype(np.float32)
+    s = (np.float32(1) / inv_s).astype(np.float32)
+    gs = oracle.fold_norm_weight(gamma, inv_s)
+    for j in range(256):
+        assert Fraction(float(gs[j])) == _fp32_round(Fraction(float(gamma[j])) * Fraction(float(inv_s[j])))
+    assert np.any((gamma / s).astype(np.float32) != gs)
+    assert np.any((gamma / (np.float32(1) / inv_s)).astype(np.float32) != gs)
 
 
 def test_rmsnorm_quant_scale_invariance():
@@ -533,6 +629,21 @@ def test_layernorm_shift_and_scale_invariance():
         np.testing.assert_array_equal(base[0], other[0])
         np.testing.assert_array_equal(base[1], other[1])
     assert not np.array_equal(base[0], oracle.rmsnorm_quant_act(x + np.float32(37.0), gs, eps)[0])
+
+
+def test_layernorm_values_are_what_is_quantized():
+    # the exposed values v (used by the GPU tests to find rounding
+    # boundaries) quantize per token to the producer's own codes and scales
+    rng = np.random.default_rng(35)
+    x = (rng.standard_normal((6, 48)) + 0.5).astype(np.float32)
+    gs = rng.uniform(0.2, 3.0, 48).astype(np.float32)
+    bs = rng.uniform(-1, 1, 48).astype(np.float32)
+    for b in (bs, None):
+        v = oracle.layernorm_values(x, gs, b, 1e-5)
+        xq, dx = oracle.layernorm_quant_act(x, gs, b, 1e-5)
+        vq, vd = oracle.quant_act(v, np.ones(48, np.float32))
+        np.testing.assert_array_equal(xq, vq)
+        np.testing.assert_array_equal(dx, vd)
 
 
 def test_layernorm_bias_alone():

@@ -103,13 +103,8 @@ def test_rmsnorm_quant_feeds_the_linear():
 
 
 def _ln_boundary_mask(x, gs, bs, eps):
-    """As _boundary_mask, for the LayerNorm value ((x - mu) r) gs + bs."""
-    mu, r = oracle.layernorm_stats(x, eps)
-    v = (x - mu[:, None]).astype(np.float32)
-    v = (v * r[:, None]).astype(np.float32)
-    v = (v * gs).astype(np.float32)
-    if bs is not None:
-        v = (v + bs).astype(np.float32)
+    """As _boundary_mask, for the oracle's LayerNorm value fma((x - mu) r, gs, bs)."""
+    v = oracle.layernorm_values(x, gs, bs, eps)
     m = np.abs(v).max(axis=1)
     delta = (m / np.float32(127.0)).astype(np.float32)
     with np.errstate(divide="ignore", invalid="ignore"):
