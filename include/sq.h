@@ -209,6 +209,12 @@ sq_status sq_quant_act_static(const void *x, sq_dtype xt, int64_t M, int64_t K,
  *         call ends.  May be NULL when that size is 0.  Calls that share a
  *         workspace must be stream-ordered.
  * M == 0 is a no-op.  K % 16 == 0, N % 16 == 0, ldy >= N.
+ * Decode-shaped calls (1 <= M <= 64) stream Wq over the SMs.  With at most
+ * 32 tokens and more 128-row tiles of Wq than SMs, a stream-K kernel shares
+ * the (tile, k-block) items evenly over all SMs and adds the partial sums
+ * of split tiles in the workspace.  Every other decode shape runs on
+ * clusters of CTAs that split tiles' K ranges and add their partials
+ * through distributed shared memory, with no workspace.
  */
 sq_status sq_w8a8_linear(const int8_t *xq, const float *x_scale,
                          const int8_t *wq, const float *w_scale, int64_t M,
@@ -216,7 +222,10 @@ sq_status sq_w8a8_linear(const int8_t *xq, const float *x_scale,
                          int64_t ldy, void *workspace, size_t workspace_bytes,
                          sq_stream_t stream);
 
-/* Bytes of workspace sq_w8a8_linear needs for this shape (0 if none). */
+/* Bytes of workspace sq_w8a8_linear needs for this shape on the current
+ * device: the stream-K decode kernel's partial sums and tile counters where
+ * that kernel runs (see sq_w8a8_linear), 0 for every other shape.  Where no
+ * device can be queried, the stream-K kernel's need for any 1 <= M <= 64. */
 size_t sq_w8a8_linear_workspace_size(int64_t M, int64_t N, int64_t K);
 
 /*
@@ -338,7 +347,9 @@ sq_status sq_w8a8_accumulate_e4m3(const uint8_t *xq, const uint8_t *wq, int64_t 
  * and forbids side allocations, latency-critical loops that cannot accept
  * cudaMalloc's implicit device-wide synchronisation, and code running inside
  * an allocator's own callbacks.  sq_w8a8_linear needs a caller-provided
- * workspace for 1 <= M <= 64; this entry point instead uses a scratch array
+ * workspace for the decode shapes that take its stream-K kernel (at most 32
+ * tokens, more 128-row tiles of Wq than SMs); this entry point instead uses
+ * a scratch array
  * of SQ_DECODE_STATIC_SCRATCH_BYTES compiled into the library (a static
  * device array that every GPU which loads the library holds until the
  * process exits).  It allocates nothing and calls no allocating routine.
@@ -347,16 +358,22 @@ sq_status sq_w8a8_accumulate_e4m3(const uint8_t *xq, const uint8_t *wq, int64_t 
  * workspace); the results are identical.
  *   - 1 <= M <= 64 and sq_w8a8_linear_workspace_size(M, N, K) <=
  *     SQ_DECODE_STATIC_SCRATCH_BYTES, else SQ_ERR_UNSUPPORTED (nothing is
- *     enqueued).  M == 0 is a no-op.
- *   - The first call on a device looks up the scratch array's device
- *     address (once per device, with that device current); make that first
- *     call outside any stream capture.
- *   - Every call on a device shares the one scratch array and clears the
- *     part it uses on `stream` before using it.  Calls whose work overlaps
- *     on the GPU (different streams without ordering, or several host
- *     threads) race on the scratch and give wrong results: serialise them.
+ *     enqueued).  M == 0 is a no-op.  A shape whose size query is 0 runs
+ *     without touching the scratch.
+ *   - The first call on a device that needs the scratch looks up the
+ *     array's device address (once per device, with that device current);
+ *     make that first call outside any stream capture.
+ *   - Every call on a device shares the one scratch array.  A shape whose
+ *     product takes the stream-K kernel (see sq_w8a8_linear) clears the part
+ *     it uses on `stream` before using it; any other shape uses no scratch
+ *     and clears nothing.  Calls whose work overlaps on the GPU (different
+ *     streams without ordering, or several host threads) race on the
+ *     scratch and give wrong results: serialise them.
  */
 #define SQ_DECODE_STATIC_SCRATCH_BYTES ((size_t)8 << 20) /* 8 MiB */
+/* The size of that scratch array as built into this library, for bindings
+ * that cannot read the macro. */
+size_t sq_decode_static_scratch_bytes(void);
 sq_status sq_w8a8_linear_decode_noalloc(const int8_t *xq, const float *x_scale,
                                         const int8_t *wq, const float *w_scale,
                                         int64_t M, int64_t N, int64_t K,

@@ -200,6 +200,19 @@ def test_decode_noalloc_and_selftest_argument_checks():
     assert t(6000, None) == INV
 
 
+def test_decode_scratch_size_agrees_everywhere():
+    # the header's macro, the value built into the library and the binding's
+    # constant must be one number
+    import os
+    import re
+    hdr = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "sq.h")
+    with open(hdr) as f:
+        m = re.search(r"#define SQ_DECODE_STATIC_SCRATCH_BYTES \(\(size_t\)(\d+) << (\d+)\)", f.read())
+    assert m is not None
+    macro = int(m.group(1)) << int(m.group(2))
+    assert sq.sq_decode_static_scratch_bytes() == macro == sq.SQ_DECODE_STATIC_SCRATCH_BYTES
+
+
 def test_workspace_size_is_defined_for_all_shapes():
     for M in (0, 1, 8, 64, 128, 2048):
         for N, K in ((256, 256), (4096, 4096), (28672, 8192)):

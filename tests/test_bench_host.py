@@ -1,4 +1,4 @@
-"""Host-side logic of bench.py and profile_case.py, without a GPU: the
+"""Host-side logic of bench.py, without a GPU: the
 source-text hash that ties the ncu traffic figure to the kernel it was
 measured on, the parsing of the nvidia-smi clock samples, the algorithmic
 bytes and ops per row, and the sweep definitions."""
@@ -79,10 +79,10 @@ def test_row_work_counts_the_algorithmic_bytes():
 
 
 def test_profile_sweeps_name_known_ops():
-    from w8a8_post_quantization_channel_b200 import profile_case as pc
+    pc = _bench()
     known = {"calib", "weight", "act", "linear", "rmsnorm", "layernorm", "static", "act8", "weight8", "linear8",
              "rot"}
-    for name, cases in pc.SWEEPS.items():
+    for name, cases in pc.sweeps().items():
         assert cases, name
         for op, M, K, N, dt in cases:
             assert op in known, (name, op)

@@ -33,7 +33,8 @@ __all__ = [
     "lib", "library_path", "header_functions",
     "sq_calib_absmax", "sq_smooth_quant_weight", "sq_quant_act", "sq_w8a8_linear",
     "sq_w8a8_linear_workspace_size", "sq_w8a8_accumulate", "sq_check_device_error", "sq_status_string",
-    "sq_w8a8_linear_decode_noalloc", "SQ_DECODE_STATIC_SCRATCH_BYTES", "sq_selftest_wait_timeout",
+    "sq_w8a8_linear_decode_noalloc", "SQ_DECODE_STATIC_SCRATCH_BYTES", "sq_decode_static_scratch_bytes",
+    "sq_selftest_wait_timeout",
     "sq_fold_smooth_into_norm", "sq_rmsnorm_quant_act", "sq_layernorm_quant_act", "sq_static_act_scale",
     "sq_quant_act_static",
     "sq_smooth_quant_weight_e4m3", "sq_quant_act_e4m3", "sq_w8a8_linear_e4m3", "sq_w8a8_accumulate_e4m3",
@@ -102,6 +103,8 @@ def lib() -> ctypes.CDLL:
             fn = getattr(L, name)
             fn.argtypes = args
             fn.restype = ctypes.c_int
+        L.sq_decode_static_scratch_bytes.argtypes = []
+        L.sq_decode_static_scratch_bytes.restype = sz
         L.sq_w8a8_linear_workspace_size.argtypes = [i64, i64, i64]
         L.sq_w8a8_linear_workspace_size.restype = sz
         L.sq_status_string.argtypes = [ctypes.c_int]
@@ -394,8 +397,14 @@ def sq_w8a8_accumulate_e4m3(xq: torch.Tensor, wq: torch.Tensor, acc=None, worksp
 
 
 # Size of the scratch array compiled into libsq.so for the allocation-free
-# decode entry point (SQ_DECODE_STATIC_SCRATCH_BYTES in include/sq.h).
+# decode entry point (SQ_DECODE_STATIC_SCRATCH_BYTES in include/sq.h; the
+# library reports the value it was built with, sq_decode_static_scratch_bytes).
 SQ_DECODE_STATIC_SCRATCH_BYTES = 8 << 20
+
+
+def sq_decode_static_scratch_bytes() -> int:
+    """The scratch size as built into the loaded library."""
+    return int(lib().sq_decode_static_scratch_bytes())
 
 
 def sq_w8a8_linear_decode_noalloc(xq: torch.Tensor, x_scale: torch.Tensor, wq: torch.Tensor,

@@ -251,6 +251,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
 
+  // stores into other GPUs' memory (the column-parallel scatter) are made
+  // visible system-wide before the kernel ends, so that the stream-ordered
+  // collective that follows cannot overtake them
+  if (dst.n > 1) __threadfence_system();
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -439,6 +443,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
 
+  // stores into other GPUs' memory (the column-parallel scatter) are made
+  // visible system-wide before the kernel ends, so that the stream-ordered
+  // collective that follows cannot overtake them
+  if (dst.n > 1) __threadfence_system();
   tc_fence_before();
   __syncthreads();
   cluster_sync();  // the peer's shared memory and TMEM stay live until the leader is done
@@ -542,6 +550,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tmW);
     prefetch_tmap(&tmX);
+    // the first ring's worth of this CTA's Wq boxes, into L2 while the
+    // previous kernel may still run (L2 stays coherent if it writes them)
+    for (int64_t w = w0; w < w1 && w < w0 + L::kStages; ++w)
+      tma_prefetch_l2_2d(&tmW, (int)(w % nk) * kBK, (int)(w / nk) * kDecRows);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, L::kTmemCols);
@@ -708,6 +720,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
 
+  // stores into other GPUs' memory (the column-parallel scatter) are made
+  // visible system-wide before the kernel ends, so that the stream-ordered
+  // collective that follows cannot overtake them
+  if (dst.n > 1) __threadfence_system();
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -717,46 +733,126 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ---------------------------------------------------------------------------
-// Decode-shaped linear, cluster split: for at most one wave of 128-row Wq
-// tiles.  A cluster of S CTAs owns one tile; CTA c of the cluster streams
-// k-blocks [c nk / S, (c+1) nk / S) into its TMEM accumulator (Wq rows on
-// the MMA's M side, tokens on N, as in the stream-K kernel).  The S int32
-// partials are then exchanged through distributed shared memory: each CTA
-// parks its partial in its own shared memory, the cluster synchronises,
-// and CTA c sums rows [c 128 / S, (c+1) 128 / S) over all S partials and
-// dequantizes them.  No workspace, no global atomics, no fences.
+// Decode-shaped linear, cluster split.  C clusters of S CTAs.  Cluster c
+// owns the 128-row Wq tiles [nt c / C, nt (c+1) / C); its (tile, k-block)
+// items, in tile-major order, are split evenly over its S CTAs.  A CTA's
+// share is thus one or more segments: runs of k-blocks of one tile.  Each
+// segment accumulates in its own TMEM columns (Wq rows on the MMA's M side,
+// tokens on N, as in the stream-K kernel).  A segment that covers a whole
+// tile is dequantized straight from TMEM.  A partial segment is parked in
+// shared memory; after a cluster barrier, every CTA that contributed to a
+// split tile sums its share of that tile's rows over all contributors'
+// partials through distributed shared memory (int32 sums: exact; E4M3: f32
+// sums taken in rank order) and dequantizes them.  No workspace, no global
+// atomics.  The scales are read into shared memory while the weights stream.
 // ---------------------------------------------------------------------------
+constexpr int kDecMaxSegs = 16;   // segments per CTA (scale slots in shared memory)
+constexpr int kDecMaxPeers = 8;   // CTAs per cluster
+
+// A split tile's reduction, worked out once per CTA while the weights
+// stream: the tile's contributors (ranks ra .. ra + cnt - 1), this CTA's
+// share of its rows (4-row units [u0, u1) of 32), and where in each
+// contributor's parked partials the tile's segment lies (word offsets).
+struct DecSplit {
+  int g, ra, cnt, u0, u1;
+  uint32_t off[kDecMaxPeers];
+};
+
+// Segments that fit one CTA: TMEM columns (MP each, 512 in all), parking
+// space in the drained ring (MP x 128 int32 each) and the scale slots.
+template <int MP>
+constexpr int dec_max_segs() {
+  constexpr int by_tmem = 512 / MP;
+  constexpr int by_smem = (int)(DecSmem<MP>::kRing / (MP * kDecRows * 4));
+  constexpr int m = by_tmem < by_smem ? by_tmem : by_smem;
+  return m < kDecMaxSegs ? m : kDecMaxSegs;
+}
+
+template <int MP>
+struct DecClusterSmem {
+  static constexpr uint32_t kRing = DecSmem<MP>::kRing;
+  static constexpr uint32_t kBars = DecSmem<MP>::kBars;
+  static constexpr uint32_t kScales = (kDecMaxSegs * kDecRows + MP) * 4;  // dw per segment row, dx per token
+  static constexpr uint32_t kSplits = 2 * sizeof(DecSplit) + 16;           // at most two split tiles per CTA
+  static constexpr uint32_t kTotal = kRing + kBars + kScales + kSplits + 1024;
+};
+
+// Item range [i0, i1) of CTA `rank` among S sharing I items.
+__device__ __forceinline__ void dec_share(int I, int S, int rank, int &i0, int &i1) {
+  i0 = (int)((int64_t)I * rank / S);
+  i1 = (int)((int64_t)I * (rank + 1) / S);
+}
+
+template <OutKind KIND, bool F8>
+__device__ __forceinline__ void store_four(const YDest &dst, int64_t ldy, int t, int n, const uint32_t (&acc)[4],
+                                           float dx, const float *dw) {
+  // four consecutive columns n..n+3 of row t (n % 4 == 0, so 8- or 16-byte aligned)
+  const int64_t i = (int64_t)t * ldy + n;
+  if constexpr (KIND == OutKind::I32) {
+    const uint4 v = make_uint4(acc[0], acc[1], acc[2], acc[3]);
+#pragma unroll 1
+    for (int d = 0; d < dst.n; ++d) *reinterpret_cast<uint4 *>(static_cast<uint32_t *>(dst.p[d]) + i) = v;
+  } else {
+    float v[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) v[k] = __fmul_rn(__fmul_rn(acc_value<F8>(acc[k]), dx), dw[k]);
+    if constexpr (KIND == OutKind::F32) {
+      const float4 f = make_float4(v[0], v[1], v[2], v[3]);
+#pragma unroll 1
+      for (int d = 0; d < dst.n; ++d) *reinterpret_cast<float4 *>(static_cast<float *>(dst.p[d]) + i) = f;
+    } else {
+      uint2 u;
+      if constexpr (KIND == OutKind::BF16) {
+        __nv_bfloat162 a = __floats2bfloat162_rn(v[0], v[1]), b = __floats2bfloat162_rn(v[2], v[3]);
+        u = make_uint2(*reinterpret_cast<uint32_t *>(&a), *reinterpret_cast<uint32_t *>(&b));
+      } else {
+        __half2 a = __floats2half2_rn(v[0], v[1]), b = __floats2half2_rn(v[2], v[3]);
+        u = make_uint2(*reinterpret_cast<uint32_t *>(&a), *reinterpret_cast<uint32_t *>(&b));
+      }
+#pragma unroll 1
+      for (int d = 0; d < dst.n; ++d) *reinterpret_cast<uint2 *>(static_cast<uint16_t *>(dst.p[d]) + i) = u;
+    }
+  }
+}
+
 template <int MP, OutKind KIND, bool F8>
 __global__ void __launch_bounds__(kThreads, 1)
     w8a8_gemm_decode_cluster_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                                     const float *__restrict__ x_scale, const float *__restrict__ w_scale,
-                                    const YDest dst, int64_t ldy, int M, int N, int K, int S, unsigned *err) {
-  using L = DecSmem<MP>;
+                                    const YDest dst, int64_t ldy, int M, int N, int K, int S, int C, uint32_t tcols,
+                                    unsigned *err) {
+  using L = DecClusterSmem<MP>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + L::kRing);
-  uint64_t *empty = full + L::kStages;
-  uint64_t *tfull = empty + L::kStages;
+  uint64_t *empty = full + DecSmem<MP>::kStages;
+  uint64_t *tfull = empty + DecSmem<MP>::kStages;
   uint64_t *drain = tfull + 1;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-  // after the MMAs have drained the ring, it holds this CTA's partial sums
-  // as part[t][row] (t < MP, row < 128)
+  float *dws = reinterpret_cast<float *>(smem + L::kRing + L::kBars);  // [segment][128]
+  float *dxs = dws + kDecMaxSegs * kDecRows;                            // [MP]
+  DecSplit *splits = reinterpret_cast<DecSplit *>(dxs + MP);            // [2]
+  int *nsplit = reinterpret_cast<int *>(splits + 2);
+  // after the MMAs have drained the ring, it holds this CTA's partial
+  // segments as part[segment][t][row] (t < MP, row < 128)
   uint32_t *part = reinterpret_cast<uint32_t *>(smem);
+  constexpr int kStages = DecSmem<MP>::kStages;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t rank = cluster_ctarank();
-  const int tile = blockIdx.x / S;
+  const int rank = S > 1 ? (int)cluster_ctarank() : 0;
+  const int cid = blockIdx.x / S;
+  const int nt = (N + kDecRows - 1) / kDecRows;
   const int nk = (K + kBK - 1) / kBK;
-  const int kb0 = (int)((int64_t)nk * rank / S), kb1 = (int)((int64_t)nk * (rank + 1) / S);
-  // Tiles start their k-walk at different k-blocks so that the CTAs of the
-  // grid do not all fetch the same Xq tile from L2 at the same moment (the
-  // int32 sum does not depend on the order).
-  const int cnt = kb1 - kb0;
-  const int rot = cnt > 0 ? tile % cnt : 0;
+  const int tile0 = (int)((int64_t)nt * cid / C);  // the cluster's first tile
+  const int I = ((int)((int64_t)nt * (cid + 1) / C) - tile0) * nk;
+  int i0, i1;
+  dec_share(I, S, rank, i0, i1);
+  const int lt_first = i0 / nk;  // local index of the first tile this CTA touches
+  const int nseg = i1 > i0 ? (i1 - 1) / nk - lt_first + 1 : 0;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < L::kStages; ++s) {
+    for (int s = 0; s < kStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
@@ -768,9 +864,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tmW);
     prefetch_tmap(&tmX);
+    // the first ring's worth of this CTA's Wq boxes, into L2 while the
+    // previous kernel may still run (weights do not depend on it, and L2
+    // stays coherent if it does write them)
+    int n = 0;
+    for (int g = 0; g < nseg && n < kStages; ++g) {
+      const int lt = lt_first + g;
+      const int a = max(i0, lt * nk) - lt * nk, b = min(i1, (lt + 1) * nk) - lt * nk;
+      const int len = b - a, rot = (tile0 + lt) % len;
+      for (int j = 0; j < len && n < kStages; ++j, ++n)
+        tma_prefetch_l2_2d(&tmW, (a + (j + rot) % len) * kBK, (tile0 + lt) * kDecRows);
+    }
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, L::kTmemCols);
+    tmem_alloc(tmem_slot, tcols);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -782,47 +889,67 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     if (lane == 0) {
+      // ---------------- TMA producer ----------------
       uint32_t stage = 0, phase = 0, armed = 0, armed_parity = 0;
       bool ok = true;
-      for (int i = 0; i < cnt; ++i) {
-        const int kb = kb0 + (i + rot) % cnt;
-        if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, err)) {
-          ok = false;
-          break;
-        }
-        uint8_t *st = smem + stage * L::kStage;
-        mbar_arrive_expect_tx(&full[stage], L::kStage);
-        tma_load_2d(&tmW, &full[stage], st, kb * kBK, tile * kDecRows);
-        tma_load_2d(&tmX, &full[stage], st + L::kW, kb * kBK, 0);
-        armed |= 1u << stage;
-        armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
-        if (++stage == L::kStages) {
-          stage = 0;
-          phase ^= 1;
+      for (int g = 0; g < nseg && ok; ++g) {
+        const int lt = lt_first + g;
+        const int a = max(i0, lt * nk) - lt * nk, b = min(i1, (lt + 1) * nk) - lt * nk;  // k-blocks [a, b)
+        const int len = b - a;
+        // tiles start their k-walk at different k-blocks so that the CTAs
+        // of the grid do not all fetch the same Xq tile from L2 at once
+        // (the segment's sum does not depend on the order)
+        const int rot = (tile0 + lt) % len;
+        for (int j = 0; j < len; ++j) {
+          const int kb = a + (j + rot) % len;
+          if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, err)) {
+            ok = false;
+            break;
+          }
+          uint8_t *st = smem + stage * DecSmem<MP>::kStage;
+          mbar_arrive_expect_tx(&full[stage], DecSmem<MP>::kStage);
+          tma_load_2d(&tmW, &full[stage], st, kb * kBK, (tile0 + lt) * kDecRows);
+          tma_load_2d(&tmX, &full[stage], st + DecSmem<MP>::kW, kb * kBK, 0);
+          armed |= 1u << stage;
+          armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
+          if (++stage == kStages) {
+            stage = 0;
+            phase ^= 1;
+          }
         }
       }
       if (!ok) {
-        for (int s = 0; s < L::kStages; ++s)
+        for (int s = 0; s < kStages; ++s)
           if (armed & (1u << s)) mbar_wait(&full[s], (armed_parity >> s) & 1u, nullptr, err);
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
+      // ---------------- MMA issuer: one accumulator per segment ----------------
       constexpr uint32_t idesc = idesc8<F8>(kDecRows, MP);
       uint32_t stage = 0, phase = 0;
-      for (int i = 0; i < cnt; ++i) {
-        if (!mbar_wait(&full[stage], phase, abort_flag, err)) break;
-        tc_fence_after();
-        uint8_t *st = smem + stage * L::kStage;
-        const uint64_t a0 = desc_sw128_kmajor(smem_u32(st));
-        const uint64_t b0 = desc_sw128_kmajor(smem_u32(st + L::kW));
+      bool ok = true;
+      for (int g = 0; g < nseg && ok; ++g) {
+        const int lt = lt_first + g;
+        const int len = min(i1, (lt + 1) * nk) - max(i0, lt * nk);
+        const uint32_t d = tmem_base + (uint32_t)(g * MP);
+        for (int j = 0; j < len; ++j) {
+          if (!mbar_wait(&full[stage], phase, abort_flag, err)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          uint8_t *st = smem + stage * DecSmem<MP>::kStage;
+          const uint64_t a0 = desc_sw128_kmajor(smem_u32(st));
+          const uint64_t b0 = desc_sw128_kmajor(smem_u32(st + DecSmem<MP>::kW));
 #pragma unroll
-        for (int k = 0; k < kBK / 32; ++k)
-          umma8<F8>(tmem_base, a0 + 2 * k, b0 + 2 * k, idesc, (i != 0 || k != 0) ? 1u : 0u);
-        umma_commit(&empty[stage]);
-        if (++stage == L::kStages) {
-          stage = 0;
-          phase ^= 1;
+          for (int k = 0; k < kBK / 32; ++k)
+            umma8<F8>(d, a0 + 2 * k, b0 + 2 * k, idesc, (j != 0 || k != 0) ? 1u : 0u);
+          umma_commit(&empty[stage]);
+          if (++stage == kStages) {
+            stage = 0;
+            phase ^= 1;
+          }
         }
       }
       umma_commit(tfull);  // also arrives when no MMA was issued
@@ -830,96 +957,138 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_wait(drain, 0, nullptr, err);
     }
     __syncwarp();
+  } else {
+    // ---- epilogue warps, while the weights stream: the scales this CTA
+    // will need, into shared memory, and the layout of its split tiles ----
+    const int e = threadIdx.x - 64;  // 0..127
+    if (KIND != OutKind::I32) {
+      for (int g = 0; g < nseg; ++g) {
+        const int n = (tile0 + lt_first + g) * kDecRows + e;
+        dws[g * kDecRows + e] = n < N ? __ldg(w_scale + n) : 0.0f;
+      }
+      if (e < M) dxs[e] = __ldg(x_scale + e);
+    }
+    if (e == 0) {
+      // only a CTA's first and last segments can be parts of a tile
+      int ns = 0;
+      for (int g = 0; g < nseg; g += (nseg > 1 ? nseg - 1 : 1)) {
+        const int lt = lt_first + g;
+        if (min(i1, (lt + 1) * nk) - max(i0, lt * nk) == nk) continue;  // a whole tile
+        DecSplit &sp = splits[ns++];
+        sp.g = g;
+        sp.ra = -1;
+        int rb = -1;
+        for (int r = 0; r < S; ++r) {  // the CTAs whose item ranges meet the tile
+          int a, b;
+          dec_share(I, S, r, a, b);
+          if (a < b && a < (lt + 1) * nk && b > lt * nk) {
+            if (sp.ra < 0) sp.ra = r;
+            rb = r;
+            sp.off[rb - sp.ra] = (uint32_t)((lt - a / nk) * MP * kDecRows);
+          }
+        }
+        sp.cnt = rb - sp.ra + 1;
+        sp.u0 = (rank - sp.ra) * (kDecRows / 4) / sp.cnt;
+        sp.u1 = (rank - sp.ra + 1) * (kDecRows / 4) / sp.cnt;
+      }
+      *nsplit = ns;
+    }
   }
 
-  // ---- epilogue: accumulator -> registers -> (shared memory) ----
+  // ---- epilogue: accumulators -> output (whole tiles) or shared memory ----
   const bool epi = warp >= 2;
   const int q = warp & 3;
   const int row = q * 32 + lane;  // 0..127 for the epilogue warps
   bool ok = true;
   if (epi) ok = mbar_wait(tfull, 0, abort_flag, err);
-  ok = __syncthreads_and(ok);  // every thread of the CTA takes the same path
-  const bool whole = S == 1;
+  ok = __syncthreads_and(ok);  // every thread of the CTA takes the same path; scales visible
   if (ok && epi) {
     tc_fence_after();
-    const int n = tile * kDecRows + row;
-    const bool n_ok = n < N;
-    const float dw = (KIND != OutKind::I32 && n_ok) ? __ldg(w_scale + n) : 0.0f;
-    const bool have = kb1 > kb0;  // a CTA without k-blocks contributes zeros
+    for (int g = 0; g < nseg; ++g) {
+      const int lt = lt_first + g;
+      const bool whole = min(i1, (lt + 1) * nk) - max(i0, lt * nk) == nk;
+      const int n = (tile0 + lt) * kDecRows + row;
+      const float dw = dws[g * kDecRows + row];
 #pragma unroll
-    for (int c = 0; c < MP / 16; ++c) {
-      uint32_t r[16];
-      tmem_ld16(tmem_base + ((uint32_t)(q * 32) << 16) + c * 16, r);
-      tmem_ld_wait();
+      for (int c = 0; c < MP / 16; ++c) {
+        uint32_t r[16];
+        tmem_ld16(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(g * MP + c * 16), r);
+        tmem_ld_wait();
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        const int t = c * 16 + j;
-        const uint32_t v = have ? r[j] : 0u;
-        if (whole) {
-          if (t < M && n_ok) {
-            const float dx = KIND != OutKind::I32 ? __ldg(x_scale + t) : 0.0f;
-            store_one<KIND, F8>(dst, ldy, t, n, v, dx, dw);
+        for (int j = 0; j < 16; ++j) {
+          const int t = c * 16 + j;
+          if (whole) {
+            if (t < M && n < N) store_one<KIND, F8>(dst, ldy, t, n, r[j], dxs[t], dw);
+          } else if (t < M) {
+            part[(g * MP + t) * kDecRows + row] = r[j];
           }
-        } else {
-          part[t * kDecRows + row] = v;
         }
       }
     }
   }
-  if (!whole) {
-    // partials of all S CTAs in place (and visible cluster-wide)
+  if (S > 1) {
+    // every CTA's partials in place (and visible cluster-wide)
     cluster_sync();
     if (ok && epi) {
-      const int rows_per = kDecRows / S;
-      const int items = rows_per * M;
+      const int e = threadIdx.x - 64;
       const uint32_t part_addr = smem_u32(part);
-      // 4 (token, row) items per round: their remote loads for each peer are
-      // issued together, so a round costs about one latency per peer
-      for (int base = threadIdx.x - 64; base < items; base += 4 * 128) {
-        uint32_t off[4];
-        // int32 sums, or (E4M3) f32 sums taken in peer order
-        uint32_t sum[4] = {0u, 0u, 0u, 0u};
+      for (int si = 0; si < *nsplit; ++si) {
+        const DecSplit &sp = splits[si];
+        const int lt = lt_first + sp.g, units = sp.u1 - sp.u0, total = units * M;
+        // two (token, 4-row) items per thread and round: all their
+        // contributors' partials are requested before any is summed
+        for (int i0r = e; i0r < total; i0r += 256) {
+          uint4 v[2][kDecMaxPeers];
 #pragma unroll
-        for (int b = 0; b < 4; ++b) {
-          const int idx = base + b * 128;
-          const int t = idx / rows_per, rr = (int)rank * rows_per + idx % rows_per;
-          off[b] = part_addr + (uint32_t)(t * kDecRows + rr) * 4u;
-        }
-#pragma unroll 1
-        for (int p = 0; p < S; ++p) {
+          for (int b = 0; b < 2; ++b) {
+            const int idx = i0r + b * 128;
+            if (idx < total) {
+              const int t = idx / units, rr = (sp.u0 + idx % units) * 4;
 #pragma unroll
-          for (int b = 0; b < 4; ++b)
-            if (base + b * 128 < items) {
-              const uint32_t pv = ld_shared_cluster_u32(mapa_shared(off[b], (uint32_t)p));
-              if constexpr (F8) {
-                sum[b] = __float_as_uint(__fadd_rn(__uint_as_float(sum[b]), __uint_as_float(pv)));
-              } else {
-                sum[b] += pv;
-              }
+              for (int p = 0; p < kDecMaxPeers; ++p)
+                if (p < sp.cnt)
+                  v[b][p] = ld_shared_cluster_v4(
+                      mapa_shared(part_addr + (sp.off[p] + (uint32_t)(t * kDecRows + rr)) * 4u, (uint32_t)(sp.ra + p)));
             }
-        }
+          }
 #pragma unroll
-        for (int b = 0; b < 4; ++b) {
-          const int idx = base + b * 128;
-          if (idx < items) {
-            const int t = idx / rows_per, rr = (int)rank * rows_per + idx % rows_per;
-            const int n = tile * kDecRows + rr;
-            if (n < N) {
-              const float dx = KIND != OutKind::I32 ? __ldg(x_scale + t) : 0.0f;
-              const float dw = KIND != OutKind::I32 ? __ldg(w_scale + n) : 0.0f;
-              store_one<KIND, F8>(dst, ldy, t, n, sum[b], dx, dw);
+          for (int b = 0; b < 2; ++b) {
+            const int idx = i0r + b * 128;
+            if (idx < total) {
+              const int t = idx / units, rr = (sp.u0 + idx % units) * 4;
+              // int32 sums, or (E4M3) f32 sums taken in rank order
+              uint32_t sum[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+              for (int p = 0; p < kDecMaxPeers; ++p)
+                if (p < sp.cnt) {
+                  const uint32_t w4[4] = {v[b][p].x, v[b][p].y, v[b][p].z, v[b][p].w};
+#pragma unroll
+                  for (int k = 0; k < 4; ++k) {
+                    if constexpr (F8) {
+                      sum[k] = __float_as_uint(__fadd_rn(__uint_as_float(sum[k]), __uint_as_float(w4[k])));
+                    } else {
+                      sum[k] += w4[k];
+                    }
+                  }
+                }
+              const int n = (tile0 + lt) * kDecRows + rr;
+              if (n < N) store_four<KIND, F8>(dst, ldy, t, n, sum, dxs[t], dws + sp.g * kDecRows + rr);
             }
           }
         }
       }
     }
-    cluster_sync();  // no CTA leaves while a peer still reads its partial
+    cluster_sync();  // no CTA leaves while a peer still reads its partials
   }
+  // stores into other GPUs' memory (the column-parallel scatter) are made
+  // visible system-wide before the kernel ends, so that the stream-ordered
+  // collective that follows cannot overtake them
+  if (dst.n > 1) __threadfence_system();
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, L::kTmemCols);
+    tmem_dealloc(tmem_base, tcols);
   }
 }
 
@@ -1018,7 +1187,7 @@ constexpr int kPairStages = 7;
 
 template <int MP, OutKind KIND, bool F8>
 void prepare_decode_cluster_kernel() {
-  using L = DecSmem<MP>;
+  using L = DecClusterSmem<MP>;
   static bool done[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -1034,13 +1203,12 @@ void prepare_decode_cluster_kernel() {
 // be resident at once (0 if none or the query fails).
 template <int MP, OutKind KIND, bool F8>
 int cluster_capacity(int S) {
-  using L = DecSmem<MP>;
-  static int cache[64][5] = {};  // [device][log2 S]
+  using L = DecClusterSmem<MP>;
+  if (S == 1) return num_sms();
+  static int cache[64][kDecMaxPeers + 1] = {};  // [device][S]
   int dev = 0;
   cudaGetDevice(&dev);
-  int lg = 0;
-  while ((1 << lg) < S) ++lg;
-  int &c = cache[dev & 63][lg];
+  int &c = cache[dev & 63][S];
   if (c == 0) {
     prepare_decode_cluster_kernel<MP, KIND, F8>();
     cudaLaunchConfig_t cfg = {};
@@ -1064,20 +1232,85 @@ int cluster_capacity(int S) {
   return c > 0 ? c : 0;
 }
 
-template <int MP, OutKind KIND, bool F8>
-cudaError_t launch_decode_cluster(const CUtensorMap &tmW, const CUtensorMap &tmX, const float *x_scale,
-                                  const float *w_scale, int M, int N, int K, const YDest &dst, int64_t ldy, int nt,
-                                  int S,
-                                  cudaStream_t st) {
-  using L = DecSmem<MP>;
-  prepare_decode_cluster_kernel<MP, KIND, F8>();
-  return launch_pdl(w8a8_gemm_decode_cluster_kernel<MP, KIND, F8>, dim3(nt * S), dim3(kThreads), L::kTotal, st,
-                    (unsigned)S, tmW, tmX, x_scale, w_scale, dst, ldy, M, N, K, S, device_error_word());
+// How a decode-shaped product is laid over the SMs: C clusters of S CTAs
+// (cluster split, no workspace), or the stream-K kernel over the workspace.
+struct DecodePlan {
+  bool cluster = false;
+  int S = 1, C = 0;
+  uint32_t tcols = 32;  // TMEM columns per CTA of the cluster kernel
+};
+
+// Extra cost of a split tile (cluster barriers, partials through distributed
+// shared memory), in k-blocks streamed by one CTA.
+constexpr int kDecSplitCost = 6;
+
+// The plan for a decode-shaped product of M tokens on the current device.
+//  - More tiles than SMs and at most 32 tokens: the stream-K kernel.  Every
+//    CTA's share then spans at least one tile's k-blocks, so a split tile
+//    has at most two contributors: their int32 partials, and E4M3 (f32)
+//    ones too, add to the same value in either order.
+//  - Otherwise the cluster split with the least cost: the k-blocks its
+//    busiest CTA streams, plus kDecSplitCost when tiles are split (ties:
+//    fewer CTAs per cluster), among the splits whose segments fit one CTA;
+//    the stream-K kernel if none fits and tiles outnumber the SMs.
+// Residency is taken from one instantiation of the cluster kernel: all of
+// them use the same shared memory and one CTA per SM, and a plan that named
+// more clusters than fit would still be correct (clusters do not wait for
+// one another), only slower.
+template <int MP>
+DecodePlan plan_decode(int M, int N, int K) {
+  const int nt = (N + kDecRows - 1) / kDecRows, nk = (K + kBK - 1) / kBK, sms = num_sms();
+  DecodePlan best;
+  if (nt > sms && M <= 32) return best;
+  int64_t best_cost = INT64_MAX;
+  for (int S = 1; S <= kDecMaxPeers; ++S) {
+    const int cap = cluster_capacity<MP, OutKind::BF16, false>(S);
+    int C = nt < sms / S ? nt : sms / S;
+    if (cap < C) C = cap;
+    if (C <= 0) continue;
+    const int64_t tmax = (nt + C - 1) / C;              // tiles of the largest cluster
+    const int64_t items = (tmax * nk + S - 1) / S;       // k-blocks of its busiest CTA
+    int64_t segs = items == 0 ? 0 : (items + nk - 1) / nk + 1;
+    if (segs > tmax) segs = tmax;
+    if (segs > dec_max_segs<MP>()) continue;
+    const int64_t cost = items + (S > 1 ? kDecSplitCost : 0);
+    if (cost < best_cost) {
+      best_cost = cost;
+      best.cluster = true;
+      best.S = S;
+      best.C = C;
+      uint32_t need = (uint32_t)(segs * MP), cols = 32;
+      while (cols < need) cols *= 2;
+      best.tcols = cols;
+    }
+  }
+  // (with no fitting split and no more tiles than SMs, S = 1 always fits:
+  // one tile per CTA is one segment)
+  return best;
+}
+
+// Whether the decode-shaped product takes the stream-K kernel (and so the
+// workspace) on the current device.
+bool decode_plan_uses_workspace(int M, int N, int K) {
+  if (M <= 16) return !plan_decode<16>(M, N, K).cluster;
+  if (M <= 32) return !plan_decode<32>(M, N, K).cluster;
+  if (M <= 48) return !plan_decode<48>(M, N, K).cluster;
+  return !plan_decode<64>(M, N, K).cluster;
 }
 
 template <int MP, OutKind KIND, bool F8>
 cudaError_t launch_decode(const int8_t *xq, const float *x_scale, const int8_t *wq, const float *w_scale, int M,
                           int N, int K, const YDest &dst, int64_t ldy, void *workspace, cudaStream_t st) {
+  CUtensorMap tmW, tmX;
+  if (!make_tmap_i8(&tmW, wq, N, K, kDecRows)) return cudaErrorInvalidValue;
+  if (!make_tmap_i8(&tmX, xq, M, K, MP)) return cudaErrorInvalidValue;
+  const DecodePlan plan = plan_decode<MP>(M, N, K);
+  if (plan.cluster) {
+    prepare_decode_cluster_kernel<MP, KIND, F8>();
+    return launch_pdl(w8a8_gemm_decode_cluster_kernel<MP, KIND, F8>, dim3(plan.C * plan.S), dim3(kThreads),
+                      DecClusterSmem<MP>::kTotal, st, (unsigned)plan.S, tmW, tmX, x_scale, w_scale, dst, ldy, M, N,
+                      K, plan.S, plan.C, plan.tcols, device_error_word());
+  }
   using L = DecSmem<MP>;
   auto kern = w8a8_gemm_decode_kernel<MP, KIND, F8>;
   static bool attr_set[64] = {};
@@ -1088,22 +1321,12 @@ cudaError_t launch_decode(const int8_t *xq, const float *x_scale, const int8_t *
     if (e != cudaSuccess) return e;
     attr_set[dev & 63] = true;
   }
-  CUtensorMap tmW, tmX;
-  if (!make_tmap_i8(&tmW, wq, N, K, kDecRows)) return cudaErrorInvalidValue;
-  if (!make_tmap_i8(&tmX, xq, M, K, MP)) return cudaErrorInvalidValue;
   const int nt = (N + kDecRows - 1) / kDecRows, nk = (K + kBK - 1) / kBK;
-  if (nt <= num_sms()) {
-    // one wave of tiles: split K across a cluster of S CTAs per tile
-    int S = 1;
-    for (int cand = 2; cand <= 16; cand *= 2)
-      if (cand <= nk && (int64_t)nt * cand <= num_sms() && cluster_capacity<MP, KIND, F8>(cand) >= nt) S = cand;
-    return launch_decode_cluster<MP, KIND, F8>(tmW, tmX, x_scale, w_scale, M, N, K, dst, ldy, nt, S, st);
-  }
   const int64_t items = (int64_t)nt * nk;
   const int grid = (int)(items < num_sms() ? items : num_sms());
   int32_t *ws = static_cast<int32_t *>(workspace);
   unsigned *counts = reinterpret_cast<unsigned *>(static_cast<uint8_t *>(workspace) + decode_ws_elems(M, N) * 4);
-return launch_pdl(kern, dim3(grid), dim3(kThreads), L::kTotal, st, 1, tmW, tmX, x_scale, w_scale, dst, ldy, M, N, K,
+  return launch_pdl(kern, dim3(grid), dim3(kThreads), L::kTotal, st, 1, tmW, tmX, x_scale, w_scale, dst, ldy, M, N, K,
                     ws, counts, device_error_word());
 }
 
@@ -1139,8 +1362,18 @@ cudaError_t gemm_dispatch(const int8_t *xq, const float *x_scale, const int8_t *
 
 }  // namespace
 
-size_t w8a8_workspace_bytes(int64_t M, int64_t N, int64_t) {
-  if (M <= 0 || M > kDecodeMaxM) return 0;
+bool w8a8_decode_uses_workspace(int64_t M, int64_t N, int64_t K) {
+  if (M <= 0 || M > kDecodeMaxM) return false;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return true;  // no device to plan for: assume the workspace path
+  }
+  return decode_plan_uses_workspace((int)M, (int)N, (int)K);
+}
+
+size_t w8a8_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+  if (!w8a8_decode_uses_workspace(M, N, K)) return 0;
   return decode_ws_elems(M, N) * 4 + decode_counter_bytes(N);
 }
 
@@ -1206,6 +1439,8 @@ bool is_aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u)
 
 }  // namespace
 
+extern "C" size_t sq_decode_static_scratch_bytes(void) { return SQ_DECODE_STATIC_SCRATCH_BYTES; }
+
 extern "C" sq_status sq_w8a8_linear_decode_noalloc(const int8_t *xq, const float *x_scale, const int8_t *wq,
                                                    const float *w_scale, int64_t M, int64_t N, int64_t K, void *y,
                                                    sq_dtype yt, int64_t ldy, sq_stream_t stream) {
@@ -1223,14 +1458,19 @@ extern "C" sq_status sq_w8a8_linear_decode_noalloc(const int8_t *xq, const float
     return SQ_ERR_INVALID_ARG;
   if (M > sq::kDecodeMaxM) return SQ_ERR_UNSUPPORTED;
   const size_t need = sq::w8a8_workspace_bytes(M, N, K);
-  if (need == 0 || need > SQ_DECODE_STATIC_SCRATCH_BYTES) return SQ_ERR_UNSUPPORTED;
+  if (need > SQ_DECODE_STATIC_SCRATCH_BYTES) return SQ_ERR_UNSUPPORTED;
   cudaError_t e = cudaSuccess;
-  void *scratch = decode_scratch_address(&e);
-  if (scratch == nullptr) return SQ_ERR_CUDA;
+  void *scratch = nullptr;
+  if (need > 0) {  // a shape on the cluster split uses no scratch at all
+    scratch = decode_scratch_address(&e);
+    if (scratch == nullptr) return SQ_ERR_CUDA;
+  }
   cudaStream_t st = (cudaStream_t)stream;
-  // the decode kernel expects zero partial sums and zero tile counters
-  if (cudaMemsetAsync(scratch, 0, need, st) != cudaSuccess) return SQ_ERR_CUDA;
   const sq::OutKind kind = yt == SQ_F32 ? sq::OutKind::F32 : yt == SQ_F16 ? sq::OutKind::F16 : sq::OutKind::BF16;
+  // the stream-K decode kernel expects zero partial sums and zero tile
+  // counters (cleared on every call: a call that timed out may have left
+  // them dirty)
+  if (need > 0 && cudaMemsetAsync(scratch, 0, need, st) != cudaSuccess) return SQ_ERR_CUDA;
   e = sq::launch_w8a8_gemm(xq, x_scale, wq, w_scale, M, N, K, y, kind, ldy, scratch, need, st, sq::QFmt::I8);
   return e == cudaSuccess ? SQ_OK : SQ_ERR_CUDA;
 }

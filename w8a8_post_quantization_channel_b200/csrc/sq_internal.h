@@ -99,6 +99,13 @@ cudaError_t launch_w8a8_gemm_dest(const int8_t *xq, const float *x_scale, const 
 cudaError_t launch_w8a8_gemm(const int8_t *xq, const float *x_scale, const int8_t *wq, const float *w_scale,
                              int64_t M, int64_t N, int64_t K, void *y, OutKind kind, int64_t ldy, void *workspace,
                              size_t workspace_bytes, cudaStream_t st, QFmt fmt);
+// Workspace bytes the product of this shape needs on the current device:
+// the stream-K decode kernel's partial sums and tile counters, or 0 (the
+// cluster split and the prefill kernels use none).  Without a device to plan
+// for, the stream-K kernel's need for any decode-shaped M.
 size_t w8a8_workspace_bytes(int64_t M, int64_t N, int64_t K);
+// Whether the decode-shaped product (1 <= M <= 64) of this shape takes the
+// stream-K kernel on the current device.
+bool w8a8_decode_uses_workspace(int64_t M, int64_t N, int64_t K);
 
 }  // namespace sq
