@@ -235,6 +235,34 @@ def step(layers, sq, world: int, ev=None):
         timed("linear", lambda: sq.sq_w8a8_linear(L.xq, L.xs, L.wq, L.ws, torch.float16, y=L.y))
 
 
+def row_graph_ms(layers, sq) -> dict:
+    """Per-step time of each row, its calls (one per linear) replayed back to
+    back from a CUDA graph.  The activation rows rotate over extra copies of
+    the four inputs, so that the replayed inputs exceed 2 x L2 as the other
+    rows' already do (3.8 GB of calibration tokens, 0.4 GB of weights, 0.26
+    GB of codes and weights per step)."""
+    out = {}
+    calls = {"calib": [], "weight": [], "act": [], "linear": []}
+    copies = []
+    for L in layers:
+        calls["calib"].append(lambda L=L: sq.sq_calib_absmax(L.calib, L.amax))
+        calls["weight"].append(lambda L=L: sq.sq_smooth_quant_weight(L.w, sq.SQ_W_NK, L.amax, 0.5, wq=L.wq,
+                                                                      w_scale=L.ws, smooth=L.s, inv_smooth=L.inv))
+        calls["linear"].append(lambda L=L: sq.sq_w8a8_linear(L.xq, L.xs, L.wq, L.ws, torch.float16, y=L.y))
+    act_bytes = sum(L.x.numel() * L.x.element_size() for L in layers)
+    reps = max(1, -(-(2 * L2_BYTES + 1) // act_bytes))
+    for _ in range(reps):
+        for L in layers:
+            x = L.x.clone()
+            copies.append(x)
+            calls["act"].append(lambda L=L, x=x: sq.sq_quant_act(x, L.inv, xq=L.xq, x_scale=L.xs))
+    for row, cs in calls.items():
+        secs, _ = graph_seconds_per_call(cs, min_calls=40, max_calls=400)
+        out[row] = secs * len(layers) * 1e3
+    del copies
+    return out
+
+
 def row_work(layers):
     """Algorithmic bytes / ops per step for each row (one rank)."""
     calib = sum(L.calib.shape[0] * L.K * 2 + 8 * L.K for L in layers)
@@ -409,7 +437,12 @@ def bench_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     if sq.sq_check_device_error() != sq.SQ_OK:
         raise RuntimeError("device-side timeout during the per-row pass")
-    row_ms = {r: sum(a.elapsed_time(b) for a, b in v) / row_steps for r, v in ev.items()}
+    row_ms_isolated = {r: sum(a.elapsed_time(b) for a, b in v) / row_steps for r, v in ev.items()}
+    # -- and each row's calls back to back, as they run inside a step (a CUDA
+    # graph per row, replayed; no event between the calls) ------------------
+    row_ms = row_graph_ms(layers, sq)
+    if sq.sq_check_device_error() != sq.SQ_OK:
+        raise RuntimeError("device-side timeout during the per-row graphs")
 
     if world > 1:
         t = torch.tensor([ms_total], device=device, dtype=torch.float64)
@@ -461,7 +494,11 @@ def bench_ours(args, rank, world, local_rank):
                            "peak_note": "INT8 = 2 x measured bf16 (nominal dense ratio 4.5/2.25)"},
            "act_quant": {"GB/s": rows["act"]["GB/s"], "frac_of_hbm": rows["act"]["frac_of_hbm"],
                          "shapes": "2048 tokens x K = 4096 (x3), 16384 (x1), fp16"},
-           "rows": rows, "rows_timing": f"per-call CUDA events over {row_steps} further steps",
+           "rows": rows,
+           "rows_timing": "each row's calls for the four linears captured in a CUDA graph and replayed back to back "
+                          "(inputs rotate over copies larger than 2 x L2), CUDA events around the replays",
+           "rows_isolated_ms_per_step": {r: round(v, 4) for r, v in row_ms_isolated.items()},
+           "rows_isolated_timing": f"each call bracketed by CUDA events, {row_steps} further steps",
            "gpu_launches": LAUNCHES_PER_LINEAR * nlin * args.steps}
     if not args.no_extra_rows:
         out["decode"] = decode_rows(sq, pk, device)

@@ -247,8 +247,9 @@ def test_accumulate_exact(M, N, K):
 
 # Shapes with at least one round of 256 x 256 tiles for every CTA pair, which
 # the library runs on CTA pairs (tcgen05 cta_group::2) with tile widths 160,
-# 192, 224 and 256 (chosen per shape): tails in M, N and K, including tiles
-# whose second CTA's half of Xq or Wq lies entirely past the matrix edge.
+# 224 or 256, whichever fills the last round of tiles best (on 74 pairs:
+# 160, 160, 224, 256 below): tails in M, N and K, including tiles whose
+# second CTA's half of Xq or Wq lies entirely past the matrix edge.
 PAIR_SHAPES = [(1000, 8464, 272), (2304, 4160, 144), (300, 16384, 256), (256, 18944, 256)]
 
 

@@ -270,28 +270,30 @@ __global__ void __launch_bounds__(kThreads, 1)
 // and of its Wq block into its own shared memory; both loads count bytes on
 // the leader CTA's (rank 0) full barrier.  The leader's single MMA thread
 // drives the pair; its commits arrive on the matching barriers of both
-// CTAs.  Each CTA's epilogue reads its own TMEM: 128 rows x 256 columns.
-// Per CTA and k-block this moves 32 KB for 128 x 256 x 128 MACs, a third
-// less operand traffic than the single-CTA 128 x 256 tile.
+// CTAs.  Each CTA's epilogue reads its own TMEM: 128 rows x BN columns.
+// With BN = 256, per CTA and k-block this moves 32 KB for 128 x 256 x 128
+// MACs, a third less operand traffic than the single-CTA 128 x 256 tile.
+// Narrower tiles (BN = 224, 160) fill the last wave of tiles better on some
+// shapes; the dispatcher picks the width.
 // ---------------------------------------------------------------------------
-constexpr int kPairBN = 256;
-
-template <int STAGES>
+template <int BN, int STAGES>
 struct PairSmem {
-  static constexpr uint32_t kA = kBM * kBK;           // 16 KB: this CTA's 128 rows of Xq
-  static constexpr uint32_t kB = (kPairBN / 2) * kBK;  // 16 KB: this CTA's 128 rows of Wq
+  static_assert(BN % 32 == 0 && BN >= 128 && BN <= 256, "pair tile width");
+  static constexpr uint32_t kA = kBM * kBK;       // 16 KB: this CTA's 128 rows of Xq
+  static constexpr uint32_t kB = (BN / 2) * kBK;  // this CTA's BN / 2 rows of Wq (a multiple of 1 KB)
   static constexpr uint32_t kRing = STAGES * (kA + kB);
   static constexpr uint32_t kBars = (2 * STAGES + 5) * 8 + 16;
   static constexpr uint32_t kTotal = kRing + kBars + 1024;
-  static constexpr uint32_t kTmemCols = 2 * kPairBN;  // two 256-column accumulators
+  static constexpr uint32_t kTmemCols = 512;  // two BN-column accumulators
 };
 
-template <int STAGES, OutKind KIND, bool F8>
+template <int BN, int STAGES, OutKind KIND, bool F8>
 __global__ void __launch_bounds__(kThreads, 1)
     w8a8_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                           const float *__restrict__ x_scale, const float *__restrict__ w_scale,
                           const YDest dst, int64_t ldy, int M, int N, int K, unsigned *err) {
-  using L = PairSmem<STAGES>;
+  using L = PairSmem<BN, STAGES>;
+  constexpr int kPairBN = BN;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *sA = smem;
@@ -384,7 +386,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int tile = pair; tile < tiles && ok; tile += npairs) {
         if (!mbar_wait(&tempty[ab], aphase ^ 1, abort_flag, err)) break;
         tc_fence_after();
-        const uint32_t d = tmem_base + ab * kPairBN;
+        const uint32_t d = tmem_base + ab * 256;  // accumulators at columns 0 and 256
         for (int kb = 0; kb < nk; ++kb) {
           if (!mbar_wait(&full[stage], phase, abort_flag, err)) {
             ok = false;
@@ -430,7 +432,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 1
       for (int c = 0; c < kPairBN / 32; ++c) {
         uint32_t r[32];
-        tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + ab * kPairBN + c * 32, r);
+        tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + ab * 256 + c * 32, r);
         tmem_ld_wait();
         const int n0 = nb * kPairBN + c * 32;
         if (row_ok && n0 < N) store_chunk<KIND, F8>(r, dst, ldy, row, n0, N, dx, w_scale);
@@ -1142,27 +1144,27 @@ cudaError_t launch_tc(const CUtensorMap &tmA, const CUtensorMap &tmB, const floa
                     device_error_word());
 }
 
-template <int STAGES, OutKind KIND, bool F8>
+template <int BN, int STAGES, OutKind KIND, bool F8>
 cudaError_t launch_pair(const CUtensorMap &tmA, const CUtensorMap &tmB, const float *x_scale, const float *w_scale,
                         const YDest &dst, int64_t ldy, int M, int N, int K, int max_clusters, cudaStream_t st) {
-  using L = PairSmem<STAGES>;
-  auto kern = w8a8_gemm_pair_kernel<STAGES, KIND, F8>;
-  const int tiles = ((M + 2 * kBM - 1) / (2 * kBM)) * ((N + kPairBN - 1) / kPairBN);
+  using L = PairSmem<BN, STAGES>;
+  auto kern = w8a8_gemm_pair_kernel<BN, STAGES, KIND, F8>;
+  const int tiles = ((M + 2 * kBM - 1) / (2 * kBM)) * ((N + BN - 1) / BN);
   const int clusters = tiles < max_clusters ? tiles : max_clusters;
   return launch_pdl(kern, dim3(2 * clusters), dim3(kThreads), L::kTotal, st, 2, tmA, tmB, x_scale, w_scale, dst, ldy, M,
                     N, K, device_error_word());
 }
 
 // Clusters of two 1-CTA-per-SM blocks that fit on the device at once.
-template <int STAGES, OutKind KIND, bool F8>
+template <int BN, int STAGES, OutKind KIND, bool F8>
 int pair_capacity() {
-  using L = PairSmem<STAGES>;
+  using L = PairSmem<BN, STAGES>;
   static int cache[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   int &c = cache[dev & 63];
   if (c == 0) {
-    auto kern = w8a8_gemm_pair_kernel<STAGES, KIND, F8>;
+    auto kern = w8a8_gemm_pair_kernel<BN, STAGES, KIND, F8>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::kTotal) != cudaSuccess)
       return -1;
     cudaLaunchConfig_t cfg = {};
@@ -1183,7 +1185,42 @@ int pair_capacity() {
   return c;
 }
 
-constexpr int kPairStages = 7;
+// Ring depths that fill ~224 KB of shared memory at each tile width.
+template <int BN>
+constexpr int pair_stages() {
+  return (int)((224u * 1024u) / PairSmem<BN, 1>::kRing);
+}
+
+// The pair-tile width whose rounds of tiles take the least time: the number
+// of rounds over `pairs` CTA pairs times the width (a tile's MMA time grows
+// with it); ties go to the wider tile, which moves fewer operand bytes per
+// MAC.
+inline int pair_width(int M, int N, int pairs) {
+  const int widths[3] = {256, 224, 160};
+  int best = 256;
+  int64_t best_cost = INT64_MAX;
+  for (int w : widths) {
+    const int64_t tiles = (int64_t)((M + 255) / 256) * ((N + w - 1) / w);
+    const int64_t cost = (tiles + pairs - 1) / pairs * w;
+    if (cost < best_cost) {
+      best_cost = cost;
+      best = w;
+    }
+  }
+  return best;
+}
+
+template <int BN, OutKind KIND, bool F8>
+cudaError_t run_pair(const int8_t *xq, const float *x_scale, const int8_t *wq, const float *w_scale, int M, int N,
+                     int K, const YDest &dst, int64_t ldy, int pairs, cudaStream_t st) {
+  CUtensorMap tmA, tmB;
+  if (!make_tmap_i8(&tmA, xq, M, K, kBM)) return cudaErrorInvalidValue;
+  if (!make_tmap_i8(&tmB, wq, N, K, BN / 2)) return cudaErrorInvalidValue;
+  constexpr int S = pair_stages<BN>();
+  const int cap = pair_capacity<BN, S, KIND, F8>();
+  if (cap <= 0) return cudaErrorLaunchOutOfResources;
+  return launch_pair<BN, S, KIND, F8>(tmA, tmB, x_scale, w_scale, dst, ldy, M, N, K, cap < pairs ? cap : pairs, st);
+}
 
 template <int MP, OutKind KIND, bool F8>
 void prepare_decode_cluster_kernel() {
@@ -1240,9 +1277,11 @@ struct DecodePlan {
   uint32_t tcols = 32;  // TMEM columns per CTA of the cluster kernel
 };
 
-// Extra cost of a split tile (cluster barriers, partials through distributed
-// shared memory), in k-blocks streamed by one CTA.
-constexpr int kDecSplitCost = 6;
+// Extra cost of splitting tiles across a cluster (two cluster barriers, and
+// partial sums of M tokens through distributed shared memory), in k-blocks
+// streamed by one CTA: 6 + M / 4, fitted to timed launches of the Llama-2
+// decode shapes (M = 1 .. 64).
+inline int dec_split_cost(int M) { return 6 + M / 4; }
 
 // The plan for a decode-shaped product of M tokens on the current device.
 //  - More tiles than SMs and at most 32 tokens: the stream-K kernel.  Every
@@ -1250,7 +1289,7 @@ constexpr int kDecSplitCost = 6;
 //    has at most two contributors: their int32 partials, and E4M3 (f32)
 //    ones too, add to the same value in either order.
 //  - Otherwise the cluster split with the least cost: the k-blocks its
-//    busiest CTA streams, plus kDecSplitCost when tiles are split (ties:
+//    busiest CTA streams, plus dec_split_cost(M) when tiles are split (ties:
 //    fewer CTAs per cluster), among the splits whose segments fit one CTA;
 //    the stream-K kernel if none fits and tiles outnumber the SMs.
 // Residency is taken from one instantiation of the cluster kernel: all of
@@ -1273,7 +1312,7 @@ DecodePlan plan_decode(int M, int N, int K) {
     int64_t segs = items == 0 ? 0 : (items + nk - 1) / nk + 1;
     if (segs > tmax) segs = tmax;
     if (segs > dec_max_segs<MP>()) continue;
-    const int64_t cost = items + (S > 1 ? kDecSplitCost : 0);
+    const int64_t cost = items + (S > 1 ? dec_split_cost(M) : 0);
     if (cost < best_cost) {
       best_cost = cost;
       best.cluster = true;
@@ -1343,11 +1382,13 @@ cudaError_t gemm_dispatch(const int8_t *xq, const float *x_scale, const int8_t *
   CUtensorMap tmA, tmB;
   // CTA pairs once there are enough 256 x 256 tiles to occupy every pair
   const int tiles_pair = ((M + 255) / 256) * ((N + 255) / 256);
-  const int cap = pair_capacity<kPairStages, KIND, F8>();
+  const int cap = pair_capacity<256, pair_stages<256>(), KIND, F8>();
   if (cap > 0 && tiles_pair >= cap) {
-    if (!make_tmap_i8(&tmA, xq, M, K, kBM)) return cudaErrorInvalidValue;
-    if (!make_tmap_i8(&tmB, wq, N, K, kPairBN / 2)) return cudaErrorInvalidValue;
-    return launch_pair<kPairStages, KIND, F8>(tmA, tmB, x_scale, w_scale, dst, ldy, M, N, K, cap, st);
+    switch (pair_width(M, N, cap)) {
+      case 160: return run_pair<160, KIND, F8>(xq, x_scale, wq, w_scale, M, N, K, dst, ldy, cap, st);
+      case 224: return run_pair<224, KIND, F8>(xq, x_scale, wq, w_scale, M, N, K, dst, ldy, cap, st);
+      default: return run_pair<256, KIND, F8>(xq, x_scale, wq, w_scale, M, N, K, dst, ldy, cap, st);
+    }
   }
   const int tiles256 = ((M + kBM - 1) / kBM) * ((N + 255) / 256);
   const bool wide = tiles256 >= sms || (N % 256 == 0 && tiles256 * 2 > sms);
