@@ -89,3 +89,18 @@ def test_profile_sweeps_name_known_ops():
             assert dt in pc.DT and K % 16 == 0, (name, op, K, dt)
             if op == "rot":
                 assert N & (N - 1) == 0 and K % N == 0, (name, K, N)
+
+
+def test_both_arms_share_the_config_and_the_reference_is_labelled():
+    import bench as b  # by its module name: the oracle processes are spawned and import it again
+    c1, c2 = b.config_dict(1), b.config_dict(2)
+    assert set(c1) == {"workload", "global_batch", "seq_len", "parallelism", "l2"}
+    assert c2["global_batch"] == 2 * c1["global_batch"] and c2["parallelism"] == "dp2"
+
+    class A:
+        oracle_procs, warmup, steps = 2, 3, 1
+    out = b.bench_reference(A, 0, 1)
+    assert out["impl"] == "reference" and out["config"] == c1
+    assert out["ms_per_step_kind"].startswith("extrapolated")
+    assert out["cpu_baseline"]["cores"] == 2 and out["e2e"]["h2d_bytes_per_step"] == 0
+    assert b.bench_reference(A, 1, 2) is None  # other ranks do no work

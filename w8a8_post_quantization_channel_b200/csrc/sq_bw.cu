@@ -229,6 +229,92 @@ __global__ void __launch_bounds__(kRowMaxThreads)
   }
 }
 
+// The same row quantizer with its row loads staged in shared memory: each
+// thread copies its own 16-byte vectors of the next D rows with cp.async
+// (no registers held for them), so a CTA keeps D + 1 rows in flight; the
+// copies are the thread's own, so reading them back needs no barrier.
+template <typename T, int kVPT, int D, typename F>
+__global__ void __launch_bounds__(kRowMaxThreads)
+    quant_rows_async_kernel(const T *__restrict__ x, int64_t rows, int64_t nvec, int64_t ld,
+                            const float *__restrict__ col_scale, int8_t *__restrict__ q,
+                            float *__restrict__ row_scale_out) {
+  pdl_wait();  // the previous kernel's results are visible from here on
+  pdl_trigger();
+  constexpr int V = Vec<T>::N;
+  extern __shared__ uint4 stage[];  // [D][kVPT][blockDim]
+  __shared__ float red[2][kRowMaxThreads / 32];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int nwarps = blockDim.x >> 5, nt = blockDim.x;
+  const int64_t K = nvec * V;
+
+  float sc[kVPT][V];
+#pragma unroll
+  for (int i = 0; i < kVPT; ++i) {
+    const int64_t v = tid + (int64_t)i * nt;
+#pragma unroll
+    for (int e = 0; e < V; ++e) sc[i][e] = v < nvec ? __ldg(col_scale + v * V + e) : 0.0f;
+  }
+  const uint64_t policy = policy_evict_first();  // every row is read exactly once
+  auto issue = [&](int64_t rr, int slot) {
+#pragma unroll
+    for (int i = 0; i < kVPT; ++i) {
+      const int64_t v = tid + (int64_t)i * nt;
+      if (rr < rows && v < nvec) cp_async_16(&stage[(slot * kVPT + i) * nt + tid], x + rr * ld + v * V, policy);
+    }
+    cp_async_commit();  // one group per row, empty past the last row
+  };
+  int64_t r = blockIdx.x;
+#pragma unroll
+  for (int d = 0; d < D; ++d) issue(r + (int64_t)d * gridDim.x, d);
+  int slot = 0, rslot = 0;
+  for (; r < rows; r += gridDim.x) {
+    cp_async_wait<D - 1>();  // this row's copies (the oldest group) have landed
+    uint4 cur[kVPT];
+#pragma unroll
+    for (int i = 0; i < kVPT; ++i) cur[i] = stage[(slot * kVPT + i) * nt + tid];
+    issue(r + (int64_t)D * gridDim.x, slot);  // the slot's next row
+    slot = slot + 1 == D ? 0 : slot + 1;
+    float val[kVPT][V];
+    float m = 0.0f;
+#pragma unroll
+    for (int i = 0; i < kVPT; ++i) {
+      float f[V];
+      Vec<T>::to_f32(cur[i], f);
+#pragma unroll
+      for (int e = 0; e < V; e += 2) {
+        const float2 p = fmul2_rn(make_float2(f[e], f[e + 1]), make_float2(sc[i][e], sc[i][e + 1]));
+        val[i][e] = p.x;
+        val[i][e + 1] = p.y;
+      }
+#pragma unroll
+      for (int e = 0; e < V; e += 2) m = fmax3(m, fabsf(val[i][e]), fabsf(val[i][e + 1]));
+    }
+    m = warp_max(m);
+    if (lane == 0) red[rslot][warp] = m;
+    __syncthreads();
+    m = 0.0f;
+    for (int w = 0; w < nwarps; ++w) m = fmaxf(m, red[rslot][w]);
+    rslot ^= 1;
+    // scale delta = m / Q; codes of fl(v / delta) (rcp = 0 for a zero row)
+    const float delta = __fdiv_rn(m, F::kMax);
+    const float rcp = m > 0.0f ? __frcp_rn(delta) : 0.0f;
+    if (tid == 0) row_scale_out[r] = delta;
+    int8_t *qrow = q + r * K;
+#pragma unroll
+    for (int i = 0; i < kVPT; ++i) {
+      const int64_t v = tid + (int64_t)i * nt;
+      if (v < nvec) {
+        if constexpr (V == 8) {
+          *reinterpret_cast<uint2 *>(qrow + v * V) = F::codes8(val[i], delta, rcp);
+        } else {
+          *reinterpret_cast<uint32_t *>(qrow + v * V) = F::codes4(val[i], delta, rcp);
+        }
+      }
+    }
+  }
+  cp_async_wait<0>();  // no copy may land after the CTA exits
+}
+
 // Row quantizer for long rows (persistent, one CTA of 512 threads per SM):
 // whole rows are staged in shared memory by bulk async copies into
 // kStages buffers (one mbarrier each), issued kStages rows ahead; the
@@ -506,6 +592,30 @@ cudaError_t launch_quant_rows_persistent(const T *x, int64_t rows, int64_t nvec,
                     col_scale, q, row_scale_out);
 }
 
+template <typename T, int kVPT, int D, typename F>
+cudaError_t launch_quant_rows_async(const T *x, int64_t rows, int64_t nvec, int64_t ld, const float *col_scale,
+                                    int8_t *q, float *row_scale_out, int threads, cudaStream_t st) {
+  static int per_sm[64][5] = {};  // [device][threads / 128], per instantiation
+  auto kern = quant_rows_async_kernel<T, kVPT, D, F>;
+  const size_t smem = (size_t)D * kVPT * threads * 16;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  int &cached = per_sm[dev & 63][(threads - 1) / 128];
+  if (cached == 0) {
+    if (smem > 48 * 1024) {
+      cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e != cudaSuccess) return e;
+    }
+    int n = 0;
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, threads, smem);
+    if (e != cudaSuccess) return e;
+    cached = n > 0 ? n : 1;
+  }
+  const int64_t grid = std::min<int64_t>(rows, (int64_t)cached * num_sms());
+  return launch_pdl(kern, dim3((unsigned)grid), dim3(threads), smem, st, 1, x, rows, nvec, ld, col_scale, q,
+                    row_scale_out);
+}
+
 template <typename T, int kVPT, int kStages, typename F>
 cudaError_t launch_quant_rows_smem(const T *x, int64_t rows, int64_t nvec, int64_t ld, const float *col_scale,
                                    int8_t *q, float *row_scale_out, uint32_t row_bytes, uint32_t smem_bytes,
@@ -524,6 +634,11 @@ cudaError_t launch_quant_rows_smem(const T *x, int64_t rows, int64_t nvec, int64
                     q, row_scale_out, row_bytes, device_error_word());
 }
 
+// Which of the two register-row quantizers serves rows of 129..2048 16-byte
+// vectors: the one whose row loads are staged with cp.async (true), or the
+// one that keeps the next row in registers.
+inline bool quant_rows_async_enabled() { return false; }
+
 template <typename T, typename F>
 cudaError_t quant_rows_t(const void *x, int64_t rows, int64_t cols, int64_t ld, const float *col_scale, int8_t *q,
                          float *row_scale_out, cudaStream_t st) {
@@ -538,6 +653,8 @@ cudaError_t quant_rows_t(const void *x, int64_t rows, int64_t cols, int64_t ld, 
     return launch_quant_rows_persistent<T, 1, F>(xp, rows, nvec, ld, col_scale, q, row_scale_out, threads_for(1), st);
   }
   if (nvec <= 4 * kRowMaxThreads) {
+    if (quant_rows_async_enabled())
+      return launch_quant_rows_async<T, 4, 3, F>(xp, rows, nvec, ld, col_scale, q, row_scale_out, threads_for(4), st);
     return launch_quant_rows_persistent<T, 4, F>(xp, rows, nvec, ld, col_scale, q, row_scale_out, threads_for(4), st);
   }
   const uint32_t row_bytes = (uint32_t)(cols * sizeof(T));

@@ -124,6 +124,21 @@ __device__ __forceinline__ uint4 ld_policy_v4(const void *p, uint64_t policy) {
   return r;
 }
 
+// 16-byte asynchronous copy global -> this thread's shared memory (through
+// L2 only), with an L2 eviction policy; completion in commit groups.
+__device__ __forceinline__ void cp_async_16(void *smem_dst, const void *gsrc, uint64_t policy) {
+  asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2;" ::"r"(
+                   static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst))),
+               "l"(gsrc), "l"(policy)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+// Waits until at most n of this thread's most recent commit groups are pending.
+template <int n>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(n) : "memory");
+}
+
 // ---------------------------------------------------------------------------
 // The quantizer: code = rne(fl(v / delta)) for a row with scale delta =
 // absmax / Q (Q = 127 for INT8, 448 for E4M3), clamped to [-127, 127] for
