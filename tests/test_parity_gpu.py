@@ -141,10 +141,12 @@ def test_quant_act(dt, K, M):
     no_device_error()
 
 
-# Heavy-tailed batches of a few hundred and a few thousand tokens: rows per
-# CTA from one to dozens, a zero row among them.
+# Heavy-tailed batches of a few hundred to ten thousand tokens: rows per CTA
+# from one to dozens, a zero row among them.  Batches of 8192 rows or more
+# run on the row kernel whose next rows are staged by cp.async, shorter ones
+# on the one that holds the next row in registers.
 @pytest.mark.parametrize("dt,K", [("bf16", 4096), ("bf16", 7168), ("f16", 16384), ("f32", 8192), ("f16", 1040)])
-@pytest.mark.parametrize("M", [300, 5000])
+@pytest.mark.parametrize("M", [300, 5000, 9000])
 def test_quant_act_batch_kernels(dt, K, M):
     o = synth.outliers(K, frac=0.01, mult=100.0, seed=K + 1)
     x = synth.activations(M, K, o, seed=K + M + 1, dtype=TORCH_DT[dt], kind="student_t3")
@@ -246,10 +248,9 @@ def test_accumulate_exact(M, N, K):
 
 
 # Shapes with at least one round of 256 x 256 tiles for every CTA pair, which
-# the library runs on CTA pairs (tcgen05 cta_group::2) with tile widths 160,
-# 224 or 256, whichever fills the last round of tiles best (on 74 pairs:
-# 160, 160, 224, 256 below): tails in M, N and K, including tiles whose
-# second CTA's half of Xq or Wq lies entirely past the matrix edge.
+# the library runs on CTA pairs (tcgen05 cta_group::2): tails in M, N and K,
+# including tiles whose second CTA's half of Xq or Wq lies entirely past the
+# matrix edge.
 PAIR_SHAPES = [(1000, 8464, 272), (2304, 4160, 144), (300, 16384, 256), (256, 18944, 256)]
 
 

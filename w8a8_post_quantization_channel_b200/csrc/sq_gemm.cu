@@ -273,8 +273,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 // CTAs.  Each CTA's epilogue reads its own TMEM: 128 rows x BN columns.
 // With BN = 256, per CTA and k-block this moves 32 KB for 128 x 256 x 128
 // MACs, a third less operand traffic than the single-CTA 128 x 256 tile.
-// Narrower tiles (BN = 224, 160) fill the last wave of tiles better on some
-// shapes; the dispatcher picks the width.
+// (Narrower pair tiles, 160 or 224 wide, chosen to fill the last round of
+// tiles, measured 15-37% slower per launch on every shape that took them;
+// the library runs BN = 256.)
 // ---------------------------------------------------------------------------
 template <int BN, int STAGES>
 struct PairSmem {
@@ -1191,25 +1192,6 @@ constexpr int pair_stages() {
   return (int)((224u * 1024u) / PairSmem<BN, 1>::kRing);
 }
 
-// The pair-tile width whose rounds of tiles take the least time: the number
-// of rounds over `pairs` CTA pairs times the width (a tile's MMA time grows
-// with it); ties go to the wider tile, which moves fewer operand bytes per
-// MAC.
-inline int pair_width(int M, int N, int pairs) {
-  const int widths[3] = {256, 224, 160};
-  int best = 256;
-  int64_t best_cost = INT64_MAX;
-  for (int w : widths) {
-    const int64_t tiles = (int64_t)((M + 255) / 256) * ((N + w - 1) / w);
-    const int64_t cost = (tiles + pairs - 1) / pairs * w;
-    if (cost < best_cost) {
-      best_cost = cost;
-      best = w;
-    }
-  }
-  return best;
-}
-
 template <int BN, OutKind KIND, bool F8>
 cudaError_t run_pair(const int8_t *xq, const float *x_scale, const int8_t *wq, const float *w_scale, int M, int N,
                      int K, const YDest &dst, int64_t ldy, int pairs, cudaStream_t st) {
@@ -1384,11 +1366,7 @@ cudaError_t gemm_dispatch(const int8_t *xq, const float *x_scale, const int8_t *
   const int tiles_pair = ((M + 255) / 256) * ((N + 255) / 256);
   const int cap = pair_capacity<256, pair_stages<256>(), KIND, F8>();
   if (cap > 0 && tiles_pair >= cap) {
-    switch (pair_width(M, N, cap)) {
-      case 160: return run_pair<160, KIND, F8>(xq, x_scale, wq, w_scale, M, N, K, dst, ldy, cap, st);
-      case 224: return run_pair<224, KIND, F8>(xq, x_scale, wq, w_scale, M, N, K, dst, ldy, cap, st);
-      default: return run_pair<256, KIND, F8>(xq, x_scale, wq, w_scale, M, N, K, dst, ldy, cap, st);
-    }
+    return run_pair<256, KIND, F8>(xq, x_scale, wq, w_scale, M, N, K, dst, ldy, cap, st);
   }
   const int tiles256 = ((M + kBM - 1) / kBM) * ((N + 255) / 256);
   const bool wide = tiles256 >= sms || (N % 256 == 0 && tiles256 * 2 > sms);
