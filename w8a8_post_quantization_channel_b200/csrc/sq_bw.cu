@@ -577,10 +577,10 @@ cudaError_t absmax_rows_t(const void *x, int64_t rows, int64_t cols, int64_t ld,
 template <typename T, int kVPT, typename F>
 cudaError_t launch_quant_rows_persistent(const T *x, int64_t rows, int64_t nvec, int64_t ld, const float *col_scale,
                                          int8_t *q, float *row_scale_out, int threads, cudaStream_t st) {
-  static int per_sm[64][5] = {};  // [device][threads / 128], per instantiation
+  static int per_sm[64][kRowMaxThreads / 32 + 1] = {};  // [device][warps], per instantiation
   int dev = 0;
   cudaGetDevice(&dev);
-  int &cached = per_sm[dev & 63][(threads - 1) / 128];
+  int &cached = per_sm[dev & 63][threads / 32];
   if (cached == 0) {
     int n = 0;
     cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, quant_rows_kernel<T, kVPT, F>, threads, 0);
@@ -595,19 +595,23 @@ cudaError_t launch_quant_rows_persistent(const T *x, int64_t rows, int64_t nvec,
 template <typename T, int kVPT, int D, typename F>
 cudaError_t launch_quant_rows_async(const T *x, int64_t rows, int64_t nvec, int64_t ld, const float *col_scale,
                                     int8_t *q, float *row_scale_out, int threads, cudaStream_t st) {
-  static int per_sm[64][5] = {};  // [device][threads / 128], per instantiation
+  static int per_sm[64][kRowMaxThreads / 32 + 1] = {};  // [device][warps], per instantiation
+  static int attr_bytes[64] = {};
   auto kern = quant_rows_async_kernel<T, kVPT, D, F>;
   const size_t smem = (size_t)D * kVPT * threads * 16;
   int dev = 0;
   cudaGetDevice(&dev);
-  int &cached = per_sm[dev & 63][(threads - 1) / 128];
-  if (cached == 0) {
+  if (attr_bytes[dev & 63] < (int)smem) {
     // (the dynamic share plus the kernel's static reduction array may pass
     // the 48 KB available without opting in)
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
+    attr_bytes[dev & 63] = (int)smem;
+  }
+  int &cached = per_sm[dev & 63][threads / 32];
+  if (cached == 0) {
     int n = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, threads, smem);
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, threads, smem);
     if (e != cudaSuccess) return e;
     cached = n > 0 ? n : 1;
   }
