@@ -151,7 +151,7 @@ def _check_acc(acc_gpu, xq, wq):
 
 
 SHAPES = [(1, 256, 4096), (16, 4096, 4096), (33, 1024, 11008), (64, 28672, 1024), (8, 19968, 256),
-          (200, 512, 4096), (300, 2048, 272), (1024, 4096, 2048)]
+          (200, 512, 4096), (300, 2048, 272), (1024, 4096, 2048), (300, 10000, 1040)]
 
 
 @pytest.mark.parametrize("M,N,K", SHAPES)

@@ -251,7 +251,8 @@ def test_accumulate_exact(M, N, K):
 # the library runs on CTA pairs (tcgen05 cta_group::2): tails in M, N and K,
 # including tiles whose second CTA's half of Xq or Wq lies entirely past the
 # matrix edge.
-PAIR_SHAPES = [(1000, 8464, 272), (2304, 4160, 144), (300, 16384, 256), (256, 18944, 256)]
+PAIR_SHAPES = [(1000, 8464, 272), (2304, 4160, 144), (300, 16384, 256), (256, 18944, 256),
+               (300, 10000, 1040), (512, 19200, 512)]
 
 
 @pytest.mark.parametrize("M,N,K", PAIR_SHAPES)
@@ -314,6 +315,22 @@ def test_decode_shapes_exact_and_workspace_clean(M, N, K):
     assert_y(y, y_ref, "bf16")
     if work is not None:
         assert int(work.count_nonzero()) == 0
+    no_device_error()
+
+
+def test_binding_workspace_is_kept_per_stream_and_left_zero():
+    # without a caller workspace the binding keeps one zeroed buffer per
+    # (device, stream); the stream-K decode kernel leaves it zero, so calls
+    # of different shapes reuse it
+    shapes = [(8, 19968, 1040), (3, 32768, 512), (8, 19968, 1040)]
+    for i, (M, N, K) in enumerate(shapes):
+        assert sq.sq_w8a8_linear_workspace_size(M, N, K) > 0
+        xq, wq = _rand_codes((M, K), 40 + i), _rand_codes((N, K), 50 + i)
+        acc = sq.sq_w8a8_accumulate(xq.to(DEV), wq.to(DEV))
+        np.testing.assert_array_equal(acc.cpu().numpy(), oracle.gemm_i8(xq.numpy(), wq.numpy()))
+    key = (torch.device(DEV).index or 0, torch.cuda.current_stream().cuda_stream)
+    cached = [w for k, w in sq._WORKSPACES.items() if k[1] == key[1]]
+    assert len(cached) == 1 and int(cached[0].count_nonzero()) == 0
     no_device_error()
 
 

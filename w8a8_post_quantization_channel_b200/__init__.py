@@ -140,6 +140,25 @@ def _ptr(t) -> ctypes.c_void_p:
     return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
 
 
+# Zeroed workspaces of the linear entry points, one per (device, stream).
+# Every call leaves its workspace zero again and calls on one stream run in
+# order, so one buffer serves them all; it grows to the largest need seen.
+_WORKSPACES: dict = {}
+
+
+def _workspace(need: int, device, stream):
+    if need == 0:
+        return None
+    s = stream if stream is not None else torch.cuda.current_stream(device)
+    key = (torch.device(device).index, s.cuda_stream)
+    w = _WORKSPACES.get(key)
+    if w is None or w.numel() < need:
+        with torch.cuda.stream(s):  # allocated on the stream that uses it
+            w = torch.zeros(need, dtype=torch.uint8, device=device)
+        _WORKSPACES[key] = w
+    return w
+
+
 def _rowmajor(t: torch.Tensor, name: str) -> None:
     if t.dim() != 2 or t.stride(1) != 1:
         raise ValueError(f"{name} must be a 2-D tensor with unit column stride")
@@ -272,7 +291,8 @@ def sq_quant_act_static(x: torch.Tensor, inv_smooth: torch.Tensor, delta: torch.
 
 
 def sq_w8a8_linear_workspace_size(M: int, N: int, K: int) -> int:
-    """Workspace bytes sq_w8a8_linear needs for this shape (0 outside decode shapes)."""
+    """Workspace bytes sq_w8a8_linear needs for this shape on the current device
+    (the stream-K decode shapes; 0 for every other shape)."""
     return int(lib().sq_w8a8_linear_workspace_size(M, N, K))
 
 
@@ -284,8 +304,8 @@ def sq_w8a8_linear(xq: torch.Tensor, x_scale: torch.Tensor, wq: torch.Tensor, w_
     y = torch.empty((M, N), dtype=out_dtype, device=xq.device) if y is None else y
     _rowmajor(y, "y")
     need = sq_w8a8_linear_workspace_size(M, N, K)
-    if workspace is None and need > 0:
-        workspace = torch.zeros(need, dtype=torch.uint8, device=xq.device)
+    if workspace is None:
+        workspace = _workspace(need, xq.device, stream)
     wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib().sq_w8a8_linear(_ptr(xq), _ptr(x_scale), _ptr(wq), _ptr(w_scale), M, N, K, _ptr(y),
                                 _dtype(y, "y"), y.stride(0), _ptr(workspace), wbytes, _stream(stream)),
@@ -311,8 +331,8 @@ def sq_w8a8_linear_scatter(xq: torch.Tensor, x_scale: torch.Tensor, wq: torch.Te
     esz = y0.element_size()
     ptrs = (ctypes.c_void_p * len(ys))(*[y.data_ptr() + col0 * esz for y in ys])
     need = sq_w8a8_linear_workspace_size(M, N, K)
-    if workspace is None and need > 0:
-        workspace = torch.zeros(need, dtype=torch.uint8, device=xq.device)
+    if workspace is None:
+        workspace = _workspace(need, xq.device, stream)
     wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib().sq_w8a8_linear_scatter(_ptr(xq), _ptr(x_scale), _ptr(wq), _ptr(w_scale), M, N, K, ptrs, len(ys),
                                         _dtype(y0, "y"), y0.stride(0), _ptr(workspace), wbytes, _stream(stream)),
@@ -325,8 +345,8 @@ def sq_w8a8_accumulate(xq: torch.Tensor, wq: torch.Tensor, acc=None, workspace=N
     N = wq.shape[0]
     acc = torch.empty((M, N), dtype=torch.int32, device=xq.device) if acc is None else acc
     need = sq_w8a8_linear_workspace_size(M, N, K)
-    if workspace is None and need > 0:
-        workspace = torch.zeros(need, dtype=torch.uint8, device=xq.device)
+    if workspace is None:
+        workspace = _workspace(need, xq.device, stream)
     wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib().sq_w8a8_accumulate(_ptr(xq), _ptr(wq), M, N, K, _ptr(acc), acc.stride(0), _ptr(workspace),
                                     wbytes, _stream(stream)), "sq_w8a8_accumulate")
@@ -372,8 +392,8 @@ def sq_w8a8_linear_e4m3(xq: torch.Tensor, x_scale: torch.Tensor, wq: torch.Tenso
     y = torch.empty((M, N), dtype=out_dtype, device=xq.device) if y is None else y
     _rowmajor(y, "y")
     need = sq_w8a8_linear_workspace_size(M, N, K)
-    if workspace is None and need > 0:
-        workspace = torch.zeros(need, dtype=torch.uint8, device=xq.device)
+    if workspace is None:
+        workspace = _workspace(need, xq.device, stream)
     wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib().sq_w8a8_linear_e4m3(_ptr(xq), _ptr(x_scale), _ptr(wq), _ptr(w_scale), M, N, K, _ptr(y),
                                      _dtype(y, "y"), y.stride(0), _ptr(workspace), wbytes, _stream(stream)),
@@ -388,8 +408,8 @@ def sq_w8a8_accumulate_e4m3(xq: torch.Tensor, wq: torch.Tensor, acc=None, worksp
     N = wq.shape[0]
     acc = torch.empty((M, N), dtype=torch.float32, device=xq.device) if acc is None else acc
     need = sq_w8a8_linear_workspace_size(M, N, K)
-    if workspace is None and need > 0:
-        workspace = torch.zeros(need, dtype=torch.uint8, device=xq.device)
+    if workspace is None:
+        workspace = _workspace(need, xq.device, stream)
     wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib().sq_w8a8_accumulate_e4m3(_ptr(xq), _ptr(wq), M, N, K, _ptr(acc), acc.stride(0), _ptr(workspace),
                                          wbytes, _stream(stream)), "sq_w8a8_accumulate_e4m3")
@@ -432,5 +452,10 @@ def sq_selftest_wait_timeout(limit_ms: int = 100, stream=None) -> int:
 
 
 def sq_check_device_error(stream=None) -> int:
-    """Synchronises the stream; returns SQ_OK or SQ_ERR_TIMEOUT (and clears it)."""
-    return int(lib().sq_check_device_error(_stream(stream)))
+    """Synchronises the stream; returns SQ_OK or SQ_ERR_TIMEOUT (and clears it).
+    After a timeout the cached workspaces are dropped: a kernel that stopped
+    early may have left tile counts in them."""
+    status = int(lib().sq_check_device_error(_stream(stream)))
+    if status != SQ_OK:
+        _WORKSPACES.clear()
+    return status
