@@ -1290,6 +1290,10 @@ DecodePlan plan_decode(int M, int N, int K) {
     if (cap < C) C = cap;
     if (C <= 0) continue;
     const int64_t tmax = (nt + C - 1) / C;              // tiles of the largest cluster
+    // every CTA of the smallest cluster gets items, so that a split tile's
+    // contributors are consecutive ranks (the split cost keeps such plans
+    // out anyway; this states it)
+    if (S > 1 && (nt / C) * nk < S) continue;
     const int64_t items = (tmax * nk + S - 1) / S;       // k-blocks of its busiest CTA
     int64_t segs = items == 0 ? 0 : (items + nk - 1) / nk + 1;
     if (segs > tmax) segs = tmax;
