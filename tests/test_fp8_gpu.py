@@ -107,6 +107,22 @@ def test_quant_act_e4m3(dt, K, M):
     assert sq.sq_check_device_error() == sq.SQ_OK
 
 
+# Long batches (8192 tokens or more) run on the staged row kernel, with eight
+# vectors per thread at these 16-bit widths and four at 16384.
+@pytest.mark.parametrize("dt,K", [("bf16", 4096), ("f16", 7168), ("bf16", 16384)])
+def test_quant_act_e4m3_long_batches(dt, K):
+    M = 8200
+    o = synth.outliers(K, frac=0.01, mult=80.0, seed=K + 11)
+    x = synth.activations(M, K, o, seed=K + M, dtype=TORCH_DT[dt], kind="student_t3")
+    x[9] = 0  # all-zero token
+    inv = torch.exp(torch.randn(K, generator=synth.gen(K + 13)))
+    xq, xs = sq.sq_quant_act_e4m3(x.to(DEV), inv.to(DEV))
+    xq_ref, xs_ref = oracle.quant_act_e4m3(f32(x), inv.numpy())
+    np.testing.assert_array_equal(xs.cpu().numpy(), xs_ref)
+    np.testing.assert_array_equal(xq.cpu().numpy(), xq_ref)
+    assert sq.sq_check_device_error() == sq.SQ_OK
+
+
 @pytest.mark.parametrize("layout", ["kn", "nk"])
 @pytest.mark.parametrize("dt", ["f32", "bf16"])
 @pytest.mark.parametrize("K,N", [(48, 80), (1040, 528)])

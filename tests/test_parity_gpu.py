@@ -144,8 +144,11 @@ def test_quant_act(dt, K, M):
 # Heavy-tailed batches of a few hundred to ten thousand tokens: rows per CTA
 # from one to dozens, a zero row among them.  Batches of 8192 rows or more
 # run on the row kernel whose next rows are staged by cp.async, shorter ones
-# on the one that holds the next row in registers.
-@pytest.mark.parametrize("dt,K", [("bf16", 4096), ("bf16", 7168), ("f16", 16384), ("f32", 8192), ("f16", 1040)])
+# on the one that holds the next row in registers.  The staged kernel takes
+# eight vectors per thread at 16-bit K = 4096, 5120, 7168 and 11008 (two or
+# more CTAs per SM) and four at K = 16384 and for fp32 rows.
+@pytest.mark.parametrize("dt,K", [("bf16", 4096), ("bf16", 7168), ("f16", 16384), ("f32", 8192), ("f16", 1040),
+                                  ("bf16", 11008), ("f16", 5120)])
 @pytest.mark.parametrize("M", [300, 5000, 9000])
 def test_quant_act_batch_kernels(dt, K, M):
     o = synth.outliers(K, frac=0.01, mult=100.0, seed=K + 1)

@@ -233,8 +233,11 @@ __global__ void __launch_bounds__(kRowMaxThreads)
 // thread copies its own 16-byte vectors of the next D rows with cp.async
 // (no registers held for them), so a CTA keeps D + 1 rows in flight; the
 // copies are the thread's own, so reading them back needs no barrier.
+// With eight vectors a thread holds 64 values and their column scales, so
+// that form is launched with at most 256 threads (registers up to 255).
+constexpr int kRowAsync8Threads = 256;
 template <typename T, int kVPT, int D, typename F>
-__global__ void __launch_bounds__(kRowMaxThreads)
+__global__ void __launch_bounds__(kVPT == 8 ? kRowAsync8Threads : kRowMaxThreads)
     quant_rows_async_kernel(const T *__restrict__ x, int64_t rows, int64_t nvec, int64_t ld,
                             const float *__restrict__ col_scale, int8_t *__restrict__ q,
                             float *__restrict__ row_scale_out) {
@@ -592,9 +595,10 @@ cudaError_t launch_quant_rows_persistent(const T *x, int64_t rows, int64_t nvec,
                     col_scale, q, row_scale_out);
 }
 
+// Sets the staged row kernel's shared-memory limit for `threads` and
+// returns how many of its CTAs an SM holds (cached per device and warps).
 template <typename T, int kVPT, int D, typename F>
-cudaError_t launch_quant_rows_async(const T *x, int64_t rows, int64_t nvec, int64_t ld, const float *col_scale,
-                                    int8_t *q, float *row_scale_out, int threads, cudaStream_t st) {
+cudaError_t quant_rows_async_occupancy(int threads, int *per_sm_out) {
   static int per_sm[64][kRowMaxThreads / 32 + 1] = {};  // [device][warps], per instantiation
   static int attr_bytes[64] = {};
   auto kern = quant_rows_async_kernel<T, kVPT, D, F>;
@@ -615,9 +619,20 @@ cudaError_t launch_quant_rows_async(const T *x, int64_t rows, int64_t nvec, int6
     if (e != cudaSuccess) return e;
     cached = n > 0 ? n : 1;
   }
-  const int64_t grid = std::min<int64_t>(rows, (int64_t)cached * num_sms());
-  return launch_pdl(kern, dim3((unsigned)grid), dim3(threads), smem, st, 1, x, rows, nvec, ld, col_scale, q,
-                    row_scale_out);
+  *per_sm_out = cached;
+  return cudaSuccess;
+}
+
+template <typename T, int kVPT, int D, typename F>
+cudaError_t launch_quant_rows_async(const T *x, int64_t rows, int64_t nvec, int64_t ld, const float *col_scale,
+                                    int8_t *q, float *row_scale_out, int threads, cudaStream_t st) {
+  int per_sm = 0;
+  cudaError_t e = quant_rows_async_occupancy<T, kVPT, D, F>(threads, &per_sm);
+  if (e != cudaSuccess) return e;
+  const size_t smem = (size_t)D * kVPT * threads * 16;
+  const int64_t grid = std::min<int64_t>(rows, (int64_t)per_sm * num_sms());
+  return launch_pdl(quant_rows_async_kernel<T, kVPT, D, F>, dim3((unsigned)grid), dim3(threads), smem, st, 1, x, rows,
+                    nvec, ld, col_scale, q, row_scale_out);
 }
 
 template <typename T, int kVPT, int kStages, typename F>
@@ -660,8 +675,21 @@ cudaError_t quant_rows_t(const void *x, int64_t rows, int64_t cols, int64_t ld, 
     return launch_quant_rows_persistent<T, 1, F>(xp, rows, nvec, ld, col_scale, q, row_scale_out, threads_for(1), st);
   }
   if (nvec <= 4 * kRowMaxThreads) {
-    if (quant_rows_async_enabled(rows))
+    if (quant_rows_async_enabled(rows)) {
+      // eight vectors per thread (half the threads per row) where that
+      // still leaves two or more CTAs on an SM: more rows in flight per SM
+      // at the same thread count (16384 tokens, bf16: K = 7168 0.76 -> 0.86
+      // of HBM, K = 11008 0.67 -> 0.87); with one CTA per SM it loses
+      if (V == 8 && nvec >= 8 * 32 && nvec <= 8 * kRowAsync8Threads) {  // 16-bit rows, as measured
+        int per_sm = 0;
+        cudaError_t e = quant_rows_async_occupancy<T, 8, 3, F>(threads_for(8), &per_sm);
+        if (e != cudaSuccess) return e;
+        if (per_sm >= 2)
+          return launch_quant_rows_async<T, 8, 3, F>(xp, rows, nvec, ld, col_scale, q, row_scale_out, threads_for(8),
+                                                     st);
+      }
       return launch_quant_rows_async<T, 4, 3, F>(xp, rows, nvec, ld, col_scale, q, row_scale_out, threads_for(4), st);
+    }
     return launch_quant_rows_persistent<T, 4, F>(xp, rows, nvec, ld, col_scale, q, row_scale_out, threads_for(4), st);
   }
   const uint32_t row_bytes = (uint32_t)(cols * sizeof(T));
