@@ -658,8 +658,13 @@ cudaError_t launch_quant_rows_smem(const T *x, int64_t rows, int64_t nvec, int64
 // rows staged by cp.async (measured on 16384-token batches: 0.81 against
 // 0.77 of HBM at K = 4096, 0.75 against 0.70 at K = 7168); shorter ones with
 // the next row in registers, whose smaller shared-memory share lets the
-// neighbouring kernels overlap it (at 2048 tokens: 8.0 against 9.1 us).
-inline bool quant_rows_async_enabled(int64_t rows) { return rows >= 8192; }
+// neighbouring kernels overlap it (at 2048 tokens: 8.0 against 9.1 us), but
+// only while rows are short: 16-bit rows of 7168 values or more stage better
+// from 2048 rows up (2048 x 11008: 18.2 against 20.5 us; 6144 x 7168: 28.9
+// against 31.9; 4096 x 16384: 45.1 against 46.2).
+inline bool quant_rows_async_enabled(int64_t rows, int64_t cols, int elem_bytes) {
+  return rows >= 8192 || (elem_bytes == 2 && rows >= 2048 && cols >= 7168);
+}
 
 template <typename T, typename F>
 cudaError_t quant_rows_t(const void *x, int64_t rows, int64_t cols, int64_t ld, const float *col_scale, int8_t *q,
@@ -675,7 +680,7 @@ cudaError_t quant_rows_t(const void *x, int64_t rows, int64_t cols, int64_t ld, 
     return launch_quant_rows_persistent<T, 1, F>(xp, rows, nvec, ld, col_scale, q, row_scale_out, threads_for(1), st);
   }
   if (nvec <= 4 * kRowMaxThreads) {
-    if (quant_rows_async_enabled(rows)) {
+    if (quant_rows_async_enabled(rows, cols, (int)sizeof(T))) {
       // eight vectors per thread (half the threads per row) where that
       // still leaves two or more CTAs on an SM: more rows in flight per SM
       // at the same thread count (16384 tokens, bf16: K = 7168 0.76 -> 0.86
