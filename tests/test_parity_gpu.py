@@ -162,6 +162,23 @@ def test_quant_act_batch_kernels(dt, K, M):
     no_device_error()
 
 
+# Both sides of the row quantizers' routing: 2047 / 2048 rows of 7168 values
+# (register / staged kernel), 7152 / 7168 values at 2048 rows, and the
+# staged kernel's eight / four vectors per thread at 12288 / 13824 values.
+@pytest.mark.parametrize("M,K,dt", [(2047, 7168, "bf16"), (2048, 7168, "bf16"), (2048, 7152, "f16"),
+                                    (8192, 12288, "f16"), (8192, 13824, "bf16")])
+def test_quant_act_routing_boundaries(M, K, dt):
+    o = synth.outliers(K, frac=0.01, mult=100.0, seed=K + 3)
+    x = synth.activations(M, K, o, seed=K + M + 3, dtype=TORCH_DT[dt], kind="student_t3")
+    x[M - 1] = 0  # all-zero last token
+    inv = torch.exp(torch.randn(K, generator=synth.gen(K + 7)))
+    xq, xs = sq.sq_quant_act(x.to(DEV), inv.to(DEV))
+    xq_ref, xs_ref = oracle.quant_act(f32(x), inv.numpy())
+    np.testing.assert_array_equal(xs.cpu().numpy(), xs_ref)
+    np.testing.assert_array_equal(xq.cpu().numpy(), xq_ref)
+    no_device_error()
+
+
 def _near_boundary_rows(n_rows, K, seed):
     """fp32 rows whose first value is the row's absmax m and whose other
     values sit within a few ulps of (k + 1/2) * delta, delta = fl(m / 127):
