@@ -107,8 +107,8 @@ def test_quant_act_e4m3(dt, K, M):
     assert sq.sq_check_device_error() == sq.SQ_OK
 
 
-# Long batches (8192 tokens or more) run on the staged row kernel, with eight
-# vectors per thread at these 16-bit widths and four at 16384.
+# Long batches (8192 tokens or more) run on the staged row kernel (four
+# vectors per thread for E4M3 codes).
 @pytest.mark.parametrize("dt,K", [("bf16", 4096), ("f16", 7168), ("bf16", 16384)])
 def test_quant_act_e4m3_long_batches(dt, K):
     M = 8200

@@ -11,6 +11,7 @@
 // per-thread partial maxima in registers and merges them with warp
 // shuffles; results are independent of the launch shape (max is exact).
 #include <algorithm>
+#include <type_traits>
 
 #include "sq_common.cuh"
 #include "sq_internal.h"
@@ -680,12 +681,15 @@ cudaError_t quant_rows_t(const void *x, int64_t rows, int64_t cols, int64_t ld, 
     return launch_quant_rows_persistent<T, 1, F>(xp, rows, nvec, ld, col_scale, q, row_scale_out, threads_for(1), st);
   }
   if (nvec <= 4 * kRowMaxThreads) {
-    if (quant_rows_async_enabled(rows, cols, (int)sizeof(T))) {
+    // the routing below was measured with INT8 codes; E4M3 codes keep the
+    // 8192-row rule and four vectors per thread
+    constexpr bool kI8 = std::is_same<F, FmtI8>::value;
+    if (quant_rows_async_enabled(rows, kI8 ? cols : 0, (int)sizeof(T))) {
       // eight vectors per thread (half the threads per row) where that
       // still leaves two or more CTAs on an SM: more rows in flight per SM
       // at the same thread count (16384 tokens, bf16: K = 7168 0.76 -> 0.86
       // of HBM, K = 11008 0.67 -> 0.87); with one CTA per SM it loses
-      if (V == 8 && nvec >= 8 * 32 && nvec <= 8 * kRowAsync8Threads) {  // 16-bit rows, as measured
+      if (kI8 && V == 8 && nvec >= 8 * 32 && nvec <= 8 * kRowAsync8Threads) {  // 16-bit rows, as measured
         int per_sm = 0;
         cudaError_t e = quant_rows_async_occupancy<T, 8, 3, F>(threads_for(8), &per_sm);
         if (e != cudaSuccess) return e;
