@@ -26,6 +26,10 @@ def test_defining_values():
     assert np.isnan(oracle.e4m3_decode(np.array([int(c) for c in g["nan_codes"]], np.uint8))).all()
     # exactly two NaN codes; every other code is finite
     assert int(np.isnan(oracle.e4m3_decode(CODES)).sum()) == 2
+    # and the encoder maps NaN onto the format's NaN pattern S.1111.111
+    # (the quantizers never meet one: their inputs are finite)
+    enc = oracle.e4m3_encode(np.array([np.nan, -np.nan], np.float32))
+    assert all(int(c) & 0x7F == 0x7F for c in enc)
 
 
 def test_hand_worked_rounding():
